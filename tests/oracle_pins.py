@@ -1,0 +1,287 @@
+"""Pins that tie the CPU oracle to something other than itself.
+
+Each ``pin_*`` takes the oracle module as ``o`` and raises AssertionError when
+the oracle disagrees with an independent fact: a hand-worked fixture, an
+explicit mask built from the row-coverage definition, exact integer
+arithmetic, a ReLU identity, brute-force scalar loops, dense masked attention
+or torch's causal scaled_dot_product_attention. ``test_oracle_pins.py`` runs
+them on the real oracle; ``test_oracle_mutations.py`` runs them on copies with a
+planted mistake and expects at least one to fail.
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+import torch
+
+from sparse_mla_prefill_b200.inputs import generate_small
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _np(inputs):
+    return {k: v.numpy() for k, v in inputs.items()}
+
+
+# ----------------------------------------------------------------- visibility
+
+def pin_visibility_mask(o, n_c: int = 12):
+    """n_vis(t) equals the row count of a mask built from row coverage, and the rows form a prefix."""
+    T = 4 * n_c + 8
+    mask = np.zeros((T, n_c), dtype=bool)
+    for t in range(T):
+        for j in range(n_c):
+            mask[t, j] = max(4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3) <= t
+    assert np.array_equal(o.explicit_visibility_mask(T, n_c), mask)
+    for t in range(T):
+        nv = min(o.n_vis(t), n_c)
+        assert nv == int(mask[t].sum()), (t, nv, int(mask[t].sum()))
+        assert mask[t, :nv].all() and not mask[t, nv:].any()
+        for j in range(n_c):
+            assert o.is_visible(t, j) == bool(mask[t, j])
+
+
+def pin_visibility_golden(o):
+    with open(os.path.join(GOLDEN, "visibility_ratio4.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            t, nv, rows = line.split()
+            t, nv = int(t), int(nv)
+            assert o.n_vis(t) == nv, (t, o.n_vis(t), nv)
+            want = [] if rows == "-" else [int(x) for x in rows.split(",")]
+            got = [j for j in range(nv + 3) if o.is_visible(t, j)]
+            assert got == want, (t, got, want)
+
+
+# -------------------------------------------------------------------- indexer
+
+def _indexer_case(T=96, H_i=4, D_i=64, seed=11):
+    return _np(generate_small(T, H_i, D_i, seed))
+
+
+def pin_scores_exact(o, inp=None, tokens=None):
+    """float64 scores equal exact int64 scores (integer-valued inputs)."""
+    inp = inp or _indexer_case()
+    tokens = range(inp["q_idx"].shape[0]) if tokens is None else tokens
+    for t in tokens:
+        f = o.indexer_scores_token(inp["q_idx"][t], inp["k_idx"], inp["w"][t], t)
+        e = o.indexer_scores_token_exact(inp["q_idx"][t], inp["k_idx"], inp["w"][t], t)
+        assert f.shape == e.shape == (o.n_vis(t),)
+        assert np.array_equal(f, e.astype(np.float64)), t
+
+
+def pin_scores_relu_identities(o, inp=None, tokens=None):
+    """relu(x)-relu(-x) = x and relu(x)+relu(-x) = |x| give two closed forms.
+
+    s(q) - s(-q) = sum_h w_h (q_h . k_j)   and   s(q) + s(-q) = sum_h w_h |q_h . k_j|,
+    each a single matrix product with no ReLU; together they fix s(q).
+    """
+    inp = inp or _indexer_case()
+    tokens = range(inp["q_idx"].shape[0]) if tokens is None else tokens
+    k = inp["k_idx"].astype(np.float64)
+    for t in tokens:
+        q = inp["q_idx"][t].astype(np.float64)
+        w = inp["w"][t].astype(np.float64)
+        nv = o.n_vis(t)
+        sp = o.indexer_scores_token(q, k, w, t)
+        sm = o.indexer_scores_token(-q, k, w, t)
+        x = q @ k[:nv].T
+        assert np.array_equal(sp - sm, w @ x), t
+        assert np.array_equal(sp + sm, w @ np.abs(x)), t
+
+
+def pin_scores_bruteforce(o):
+    """Pure-Python loops over (h, d) on a tiny case."""
+    inp = _indexer_case(T=24, H_i=3, D_i=5, seed=5)
+    q, k, w = inp["q_idx"], inp["k_idx"], inp["w"]
+    for t in range(24):
+        got = o.indexer_scores_token(q[t], k, w[t], t)
+        want = []
+        for j in range(k.shape[0]):
+            if 4 * j + 3 > t:
+                continue
+            s = 0.0
+            for h in range(q.shape[1]):
+                dot = 0.0
+                for d in range(q.shape[2]):
+                    dot += float(q[t, h, d]) * float(k[j, d])
+                s += float(w[t, h]) * (dot if dot > 0 else 0.0)
+            want.append(s)
+        assert got.tolist() == want, (t, got.tolist(), want)
+
+
+# ---------------------------------------------------------------------- top-k
+
+def pin_topk_golden(o):
+    with open(os.path.join(GOLDEN, "topk_ties.txt")) as f:
+        lines = [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+    scores = np.array([float(x) for x in lines[0].split(":")[1].split()])
+    for ln in lines[1:]:
+        k, row = ln.split("|")
+        want = [int(x) for x in row.split()]
+        got = o.topk_row(scores, int(k)).tolist()
+        assert got == want, (k, got, want)
+
+
+def _topk_brute(scores, k):
+    cands = sorted(range(len(scores)), key=lambda j: (-scores[j], j))[:min(k, len(scores))]
+    cands.sort()
+    return cands + [-1] * (k - len(cands))
+
+
+def pin_topk_bruteforce(o, trials: int = 300, seed: int = 3):
+    """Brute force by sorted() plus the defining properties, on rows rich in ties."""
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        n = int(rng.integers(0, 70))
+        k = int(rng.integers(0, 40))
+        scores = rng.integers(-3, 6, n).astype(np.float64) * float(rng.choice([1.0, 0.5, 1e3]))
+        got = o.topk_row(scores, k)
+        assert got.dtype == np.int32 and got.shape == (k,)
+        assert got.tolist() == _topk_brute(scores.tolist(), k), (scores.tolist(), k)
+        m = min(k, n)
+        sel = got[:m]
+        assert (got[m:] == -1).all() and (np.diff(sel) > 0).all()
+        rest = np.setdiff1d(np.arange(n), sel)
+        if m and len(rest):
+            assert scores[sel].min() >= scores[rest].max()
+            thr = scores[sel].min()
+            if (scores[rest] == thr).any():
+                assert sel[scores[sel] == thr].max() < rest[scores[rest] == thr].min()
+
+
+# ------------------------------------------------------------------ attention
+
+def _attn_case(T=48, n_c=None, seed=21):
+    g = torch.Generator("cpu").manual_seed(seed)
+    n_c = T // 4 if n_c is None else n_c
+    q = torch.randn(T, 16, 576, generator=g).half().double().numpy()
+    kv_raw = torch.randn(T, 576, generator=g).half().double().numpy()
+    kv_cmp = torch.randn(n_c, 576, generator=g).half().double().numpy()
+    return q, kv_raw, kv_cmp
+
+
+def pin_attention_sdpa_causal(o, T: int = 48):
+    """k = 0 and n_swa >= T reduce to causal attention with one shared KV head."""
+    q, kv_raw, kv_cmp = _attn_case(T)
+    scale = 1.0 / 24.0
+    got = o.sparse_mla_attention(q, kv_raw, kv_cmp, np.zeros((T, 0), np.int32), 0, T, scale)
+    Q = torch.from_numpy(q).permute(1, 0, 2)[None]                 # [1,16,T,576]
+    K = torch.from_numpy(kv_raw)[None, None].expand(1, 16, T, 576)
+    V = torch.from_numpy(kv_raw[:, :512])[None, None].expand(1, 16, T, 512)
+    ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, is_causal=True, scale=scale)
+    ref = ref[0].permute(1, 0, 2).numpy()
+    assert got.shape == ref.shape
+    assert np.abs(got - ref).max() < 1e-12, np.abs(got - ref).max()
+
+
+def pin_attention_sdpa_window(o, T: int = 48, n_swa: int = 7):
+    """k = 0 reduces to sliding-window attention over raw rows (banded boolean mask)."""
+    q, kv_raw, kv_cmp = _attn_case(T, seed=22)
+    scale = 0.05
+    got = o.sparse_mla_attention(q, kv_raw, kv_cmp, np.zeros((T, 0), np.int32), 0, n_swa, scale)
+    t = torch.arange(T)
+    allowed = (t[None, :] <= t[:, None]) & (t[None, :] > t[:, None] - n_swa)
+    Q = torch.from_numpy(q).permute(1, 0, 2)[None]
+    K = torch.from_numpy(kv_raw)[None, None].expand(1, 16, T, 576)
+    V = torch.from_numpy(kv_raw[:, :512])[None, None].expand(1, 16, T, 512)
+    ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=allowed, scale=scale)
+    ref = ref[0].permute(1, 0, 2).numpy()
+    assert np.abs(got - ref).max() < 1e-12, np.abs(got - ref).max()
+
+
+def pin_attention_dense_mask(o, T: int = 64, n_swa: int = 9):
+    """With k >= n_vis(t) for every t the output is dense masked attention over
+    [all compressed rows ; all raw rows], whatever the indexer scores are."""
+    q, kv_raw, kv_cmp = _attn_case(T, seed=23)
+    n_c = kv_cmp.shape[0]
+    k = n_c
+    scale = 1.0 / 24.0
+    # Any scores: selection keeps every visible row because k >= n_vis.
+    rng = np.random.default_rng(0)
+    idx = np.stack([o.topk_row(rng.standard_normal(o.n_vis(t)), k) for t in range(T)])
+    got = o.sparse_mla_attention(q, kv_raw, kv_cmp, idx, 0, n_swa, scale)
+    keys = np.concatenate([kv_cmp, kv_raw])                      # [n_c + T, 576]
+    for t in range(T):
+        cmp_ok = np.array([4 * j + 3 <= t for j in range(n_c)])
+        raw_ok = np.array([t - n_swa < s <= t for s in range(T)])
+        ok = np.concatenate([cmp_ok, raw_ok])
+        logits = scale * (q[t] @ keys.T)
+        logits[:, ~ok] = -np.inf
+        p = np.exp(logits - logits.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        ref = p @ keys[:, :512]
+        assert np.abs(got[t] - ref).max() < 1e-12, t
+
+
+def pin_attention_bruteforce(o, tokens=(0, 3, 9, 30, 47)):
+    """Scalar loops with math.exp for a few tokens of a small case (k=5, n_swa=6)."""
+    T, k, n_swa = 48, 5, 6
+    q, kv_raw, kv_cmp = _attn_case(T, seed=24)
+    rng = np.random.default_rng(1)
+    idx = np.stack([o.topk_row(rng.integers(0, 4, o.n_vis(t)).astype(float), k) for t in range(T)])
+    scale = 1.0 / 24.0
+    got = o.sparse_mla_attention(q, kv_raw, kv_cmp, idx, 0, n_swa, scale)
+    for t in tokens:
+        rows = [kv_cmp[j] for j in idx[t] if j >= 0]
+        rows += [kv_raw[s] for s in range(max(0, t - n_swa + 1), t + 1)]
+        for h in range(16):
+            logits = [scale * sum(float(a) * float(b) for a, b in zip(q[t, h], r)) for r in rows]
+            mx = max(logits)
+            e = [math.exp(x - mx) for x in logits]
+            z = sum(e)
+            for d in range(0, 512, 37):
+                want = sum(ei * float(r[d]) for ei, r in zip(e, rows)) / z
+                assert abs(got[t, h, d] - want) < 1e-12, (t, h, d)
+
+
+def pin_attention_closed_forms(o):
+    """scale = 0 gives the plain mean of the attended rows' values; token 0 alone
+    attends only raw row 0, so its output is that row's first 512 values."""
+    T, k, n_swa = 40, 4, 5
+    q, kv_raw, kv_cmp = _attn_case(T, seed=25)
+    rng = np.random.default_rng(2)
+    idx = np.stack([o.topk_row(rng.standard_normal(o.n_vis(t)), k) for t in range(T)])
+    got0 = o.sparse_mla_attention(q, kv_raw, kv_cmp, idx, 0, n_swa, 0.0)
+    for t in range(T):
+        nsel = min(k, (t + 1) // 4)
+        members = [kv_cmp[j] for j in idx[t][:nsel]] + [kv_raw[s] for s in range(max(0, t - n_swa + 1), t + 1)]
+        want = np.mean(np.stack(members)[:, :512], axis=0)
+        assert np.abs(got0[t] - want[None, :]).max() < 1e-12, t
+    got = o.sparse_mla_attention(q, kv_raw, kv_cmp, idx, 0, n_swa, 1.0 / 24.0)
+    assert np.abs(got[0] - kv_raw[0, :512][None, :]).max() < 1e-12
+
+
+# ---------------------------------------------------------------------- bands
+
+def pin_bands_equal_oneshot(o):
+    """Band-by-band equals one pass over all tokens, exactly."""
+    inp = _np(generate_small(160, 4, 64, seed=31))
+    one = o.prefill_tokens(inp, range(160), top_k=8, n_swa=12)
+    bands = o.prefill_bands(inp, 160, top_k=8, n_swa=12, band=64)
+    assert np.array_equal(one["topk"], bands["topk"])
+    assert np.array_equal(one["out"], bands["out"])
+
+
+ALL_PINS = [
+    pin_visibility_mask, pin_visibility_golden,
+    pin_scores_exact, pin_scores_relu_identities, pin_scores_bruteforce,
+    pin_topk_golden, pin_topk_bruteforce,
+    pin_attention_sdpa_causal, pin_attention_sdpa_window, pin_attention_dense_mask,
+    pin_attention_bruteforce, pin_attention_closed_forms,
+    pin_bands_equal_oneshot,
+]
+
+
+def failing_pins(o):
+    """Names of the pins the given oracle fails (used by the mutation tests)."""
+    bad = []
+    for p in ALL_PINS:
+        try:
+            p(o)
+        except (AssertionError, ValueError, IndexError):
+            bad.append(p.__name__)
+    return bad

@@ -1,0 +1,125 @@
+"""Plant a plausible mistake in a private copy of the oracle (CPU only) and check
+that the pins catch it. This shows the pins constrain every step of the oracle."""
+import importlib.util
+import os
+
+import numpy as np
+import pytest
+
+import oracle_pins as P
+
+ORACLE_SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                          "oracle", "ds4sp_oracle.py")
+
+
+def fresh_oracle():
+    spec = importlib.util.spec_from_file_location("oracle_mutant", ORACLE_SRC)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _mut_visibility_first_token(o):
+    o.n_vis = lambda t, ratio=4: (t + ratio) // ratio          # row visible at its first token
+
+
+def _mut_no_relu(o):
+    def f(q, k, w, t, ratio=4):
+        nv = o.n_vis(t, ratio)
+        return np.asarray(w, float) @ (np.asarray(q, float) @ np.asarray(k[:nv], float).T)
+    o.indexer_scores_token = f
+
+
+def _mut_relu_after_head_sum(o):
+    def f(q, k, w, t, ratio=4):
+        nv = o.n_vis(t, ratio)
+        return np.maximum(np.asarray(w, float) @ (np.asarray(q, float) @ np.asarray(k[:nv], float).T), 0)
+    o.indexer_scores_token = f
+
+
+def _mut_unweighted_heads(o):
+    def f(q, k, w, t, ratio=4):
+        nv = o.n_vis(t, ratio)
+        return np.maximum(np.asarray(q, float) @ np.asarray(k[:nv], float).T, 0).sum(axis=0)
+    o.indexer_scores_token = f
+
+
+def _mut_ties_to_higher_j(o):
+    def f(scores, k):
+        nv = len(scores)
+        out = np.full(k, -1, dtype=np.int32)
+        m = min(k, nv)
+        if m:
+            order = np.lexsort((-np.arange(nv), -np.asarray(scores, float)))
+            out[:m] = np.sort(order[:m])
+        return out
+    o.topk_row = f
+
+
+def _mut_score_order_listing(o):
+    def f(scores, k):
+        nv = len(scores)
+        out = np.full(k, -1, dtype=np.int32)
+        m = min(k, nv)
+        if m:
+            out[:m] = np.lexsort((np.arange(nv), -np.asarray(scores, float)))[:m]
+        return out
+    o.topk_row = f
+
+
+def _mut_value_last_dims(o):
+    def f(q_t, rows, scale, d_v):
+        logits = scale * (np.asarray(q_t, float) @ rows.T)
+        p = np.exp(logits - logits.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        return p @ rows[:, -d_v:]
+    o.attention_token = f
+
+
+def _mut_window_excludes_self(o):
+    o.window = lambda t, n_swa: np.arange(max(0, t - n_swa), t, dtype=np.int64)
+
+
+def _mut_scale_ignored(o):
+    orig = o.attention_token
+    o.attention_token = lambda q_t, rows, scale, d_v: orig(q_t, rows, 1.0, d_v)
+
+
+def _mut_dedup_window(o):
+    # Drops raw rows whose index coincides with a selected compressed row index.
+    orig = o.attended_rows
+    def f(t, topk_t, kv_raw, kv_cmp, n_swa):
+        sel = topk_t[topk_t >= 0]
+        win = [s for s in o.window(t, n_swa) if s not in set(sel.tolist())]
+        return np.concatenate([np.asarray(kv_cmp[sel], float), np.asarray(kv_raw[win], float)])
+    o.attended_rows = f
+
+
+MUTATIONS = [
+    (_mut_visibility_first_token, [P.pin_visibility_mask, P.pin_visibility_golden]),
+    (_mut_no_relu, [P.pin_scores_exact, P.pin_scores_relu_identities, P.pin_scores_bruteforce]),
+    (_mut_relu_after_head_sum, [P.pin_scores_relu_identities, P.pin_scores_bruteforce]),
+    (_mut_unweighted_heads, [P.pin_scores_relu_identities, P.pin_scores_bruteforce]),
+    (_mut_ties_to_higher_j, [P.pin_topk_golden, P.pin_topk_bruteforce]),
+    (_mut_score_order_listing, [P.pin_topk_golden, P.pin_topk_bruteforce]),
+    (_mut_value_last_dims, [P.pin_attention_sdpa_causal, P.pin_attention_closed_forms]),
+    (_mut_window_excludes_self, [P.pin_attention_sdpa_causal, P.pin_attention_sdpa_window]),
+    (_mut_scale_ignored, [P.pin_attention_sdpa_causal, P.pin_attention_bruteforce]),
+    (_mut_dedup_window, [P.pin_attention_dense_mask, P.pin_attention_closed_forms]),
+]
+
+
+@pytest.mark.parametrize("mutate,pins", MUTATIONS, ids=[m[0].__name__ for m in MUTATIONS])
+def test_planted_mistake_is_caught(mutate, pins):
+    o = fresh_oracle()
+    for p in pins:            # the unmutated copy passes these pins
+        p(o)
+    mutate(o)
+    caught = []
+    for p in pins:
+        try:
+            with np.errstate(all="ignore"):
+                p(o)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(p.__name__)
+    assert caught, f"{mutate.__name__} slipped past {[p.__name__ for p in pins]}"
