@@ -1,0 +1,337 @@
+"""Benchmark: DS4 sparse-prefill tokens/s on the 10,240-token frontier workload.
+
+One step = one whole prefill of T = 10,240 tokens: five 2,048-token bands in
+chronological order, each running indexer -> top-k -> streaming sparse MLA
+attention through the C ABI (ds4sp_prefill_band). Inputs are seeded synthetic
+tensors resident in HBM before the timed region; per step the inputs read
+(q 189 MB, q_idx 168 MB) and the output written (335 MB) exceed the 126 MB L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
+
+N > 1 runs under torchrun: each rank prefills its own sequence (weak scaling, no
+collective on the data path); timing is the max over ranks. ``--impl reference``
+times the CPU oracle (the only reference this method has) on a bounded token
+sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_mla_prefill_b200 import ds4sp as D  # noqa: E402
+from sparse_mla_prefill_b200.inputs import generate, workload  # noqa: E402
+
+WORKLOAD = "10k"
+METRIC = "sparse-prefill attention tokens/s at 8K/10K; HBM GB/s and % of roofline"
+
+
+# ------------------------------------------------------------------ algorithmic work
+
+def n_vis(t, ratio=4):
+    return (t + 1) // ratio
+
+
+def attn_rows(T, k, n_swa, t0=0, t1=None):
+    t1 = T if t1 is None else t1
+    return sum(min(k, n_vis(t)) + min(n_swa, t + 1) for t in range(t0, t1))
+
+
+def algorithmic(wl):
+    """Per-step algorithmic bytes / FLOPs of each kernel (per-unit figures in the design doc)."""
+    T, k, n_swa = wl.T, wl.top_k, wl.n_swa
+    rows = attn_rows(T, k, n_swa)
+    sum_vis = sum(n_vis(t) for t in range(T))
+    return {
+        "attention_bytes": 1152 * rows + (18432 + 32768 + 4 * k) * T,
+        "attention_flops": 2 * 16 * (576 + 512) * rows,
+        "indexer_flops": 2 * wl.H_i * wl.D_i * sum_vis,
+        "indexer_bytes": 2 * wl.H_i * wl.D_i * T + 4 * wl.H_i * T + 4 * sum_vis,
+        "topk_bytes": 4 * sum_vis + 4 * k * T,
+        "rows": rows,
+    }
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in out.splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ reference arm (oracle)
+
+def cpu_oracle_sample(wl, n_sample, inputs_np=None):
+    """Time the float64 CPU oracle on a spread sample of tokens; tokens/s."""
+    import numpy as np
+    import oracle
+    if inputs_np is None:
+        inputs_np = {k: v.numpy() for k, v in generate(wl).items()}
+    stride = max(1, wl.T // n_sample)
+    toks = list(range(stride - 1, wl.T, stride))[:n_sample]
+    t0 = time.perf_counter()
+    oracle.prefill_tokens(inputs_np, toks, wl.top_k, wl.n_swa)
+    dt = time.perf_counter() - t0
+    return {"value": len(toks) / dt, "unit": "tokens/s", "cores": torch.get_num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(toks)} of {wl.T} tokens (every {stride}th), float64 NumPy, "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    wl = workload(WORKLOAD)
+    if rank != 0:
+        return
+    inputs_np = {k: v.numpy() for k, v in generate(wl).items()}
+    per_step = 256
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, 32, inputs_np)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(cpu_oracle_sample(wl, per_step, inputs_np))
+    wall = time.perf_counter() - t0
+    value = args.steps * len(range(0, per_step)) / wall
+    cb = dict(vals[-1])
+    cb["value"] = value
+    cb["sample"] = f"{args.steps} steps x {per_step} tokens spread over the {wl.T}-token sequence"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * wall / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": config_name(wl), "sample_tokens_per_step": per_step},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def config_name(wl):
+    return (f"{wl.name}: T={wl.T} as {wl.n_bands} bands of {wl.band}, 16 heads, d_qk 576 / d_v 512 "
+            f"fp16, indexer {wl.H_i}x{wl.D_i}, top_k {wl.top_k}, n_swa {wl.n_swa}, seed {wl.seed}")
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = workload(WORKLOAD)
+    alg = algorithmic(wl)
+    pk = peaks()
+
+    host = generate(wl)
+    inputs = {k: v.to(dev) for k, v in host.items()}
+    cfg = D.make_config(n_idx_heads=wl.H_i, d_idx=wl.D_i, top_k=wl.top_k, n_swa=wl.n_swa,
+                        max_tokens=wl.T, band=wl.band)
+    h = D.ds4sp_create(cfg)
+    topk = torch.empty((wl.T, wl.top_k), dtype=torch.int32, device=dev)
+    out = torch.empty((wl.T, 16, 512), dtype=torch.float32, device=dev)
+    ws = D.band_workspace(h, wl.T, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        D.prefill(h, inputs, wl.T, topk, out, ws, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.item()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, bits = D.ds4sp_device_status(h)
+    if st != D.OK:
+        raise RuntimeError(f"device status {bits:#x} after warm-up")
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    D.ds4sp_profile_enable(h, True)
+    D.ds4sp_profile_read(h)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    prof = D.ds4sp_profile_read(h)
+    D.ds4sp_profile_enable(h, False)
+    clk = clocks.stop()
+    ms_max = max_over_ranks(ms)
+
+    # end to end through the public API: pinned host inputs -> device, prefill, out -> host
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out.numel() * out.element_size()
+    e2e_steps = max(1, min(args.steps, 5))
+    D.prefill_host(h, pinned, inputs, wl.T, topk, out, ws, out_host, stream)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        D.prefill_host(h, pinned, inputs, wl.T, topk, out, ws, out_host, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    st, bits = D.ds4sp_device_status(h)
+    if st != D.OK:
+        raise RuntimeError(f"device status {bits:#x} after timing")
+
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_base = cpu_oracle_sample(wl, args.cpu_sample, {k: v.numpy() for k, v in host.items()})
+
+    if rank == 0:
+        tokens = world * wl.T * args.steps
+        value = tokens / (ms_max / 1e3)
+        attn_ms, attn_n = prof["attention"]
+        idx_ms, idx_n = prof["indexer"]
+        topk_ms, topk_n = prof["topk"]
+        steps = args.steps
+        attn_achieved = alg["attention_bytes"] * steps / (attn_ms / 1e3) / 1e9
+        idx_achieved = alg["indexer_flops"] * steps / (idx_ms / 1e3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": ms_max / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16", "data": "synthetic",
+            "config": {"workload": config_name(wl), "parallelism": f"dp{world} (one sequence per rank)",
+                       "l2": "inputs larger than L2: q+q_idx read and out written per step = 692 MB > 126 MB"},
+            "roofline": {"bound": "hbm", "achieved": attn_achieved, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": attn_achieved / pk["hbm_gbs"],
+                         "traffic": None, "kernel": "sparse_attn_mma_kernel",
+                         "peak_source": f"{pk['source']} hbm_gbs (of {pk['source']})"},
+            "kernels": {
+                "attention": {"ms_per_step": attn_ms / steps, "launches": attn_n,
+                              "alg_GBps": attn_achieved,
+                              "frac_hbm": attn_achieved / pk["hbm_gbs"],
+                              "alg_bytes_per_step": alg["attention_bytes"]},
+                "indexer": {"ms_per_step": idx_ms / steps, "launches": idx_n,
+                            "TFLOPs": idx_achieved,
+                            "frac_tensor": idx_achieved / pk["bf16_tflops"],
+                            "alg_flops_per_step": alg["indexer_flops"]},
+                "topk": {"ms_per_step": topk_ms / steps, "launches": topk_n,
+                         "alg_GBps": alg["topk_bytes"] * steps / (topk_ms / 1e3) / 1e9},
+            },
+            "gpu_launches": attn_n + idx_n + topk_n,
+            "e2e": {"value": world * wl.T * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "clocks": clk,
+            "cpu_baseline": cpu_base,
+        }
+        print(json.dumps(line), flush=True)
+    D.ds4sp_destroy(h)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-sample", type=int, default=2048)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,156 @@
+/*
+ * ds4sp.h -- C ABI of libds4sp: DS4 sparse-prefill attention on NVIDIA B200 (sm_100a).
+ *
+ * Per query token t the library runs three steps:
+ *   1. indexer:   score(t, j) = sum_h w[t,h] * ReLU(q_idx[t,h,:] . k_idx[j,:])
+ *                 for every compressed row j visible to t (4j + 3 <= t);
+ *   2. top-k:     keep the min(k, n_vis(t)) best rows, equal scores to the lower j,
+ *                 listed by ascending j, unused slots -1;
+ *   3. attention: one softmax of 16 query heads over the selected compressed rows
+ *                 and the raw rows max(0, t-n_swa+1) .. t; key = all 576 dims of a
+ *                 row, value = its first 512 dims.
+ * Tokens are processed in 2048-token bands in chronological order.
+ *
+ * Sources: "perf(ds4): extend sparse prefill scheduling to 10K", Summary (five
+ * 2,048-token bands up to a 10,240-token frontier; ratio-4 causal visibility derived
+ * in the kernel instead of a stored quadratic mask; top-k rows handed directly to
+ * attention; F16 transport of selected rows; each selected latent row streamed once
+ * across sixteen heads; chronological state commit) and Qualification (ratio-4
+ * boundary formula; explicit-mask versus analytic-mask oracle). The pages do not
+ * define the indexer score, the tie rule or the window; this library fixes them as
+ * written above.
+ *
+ * Conventions for every entry point
+ *   - Tensors are caller-owned device memory, contiguous and row-major, and every
+ *     pointer is 16-byte aligned. fp16 means IEEE binary16; fp32 means IEEE binary32.
+ *   - Per-token tensors (q, q_idx, w, topk, out) start at token t0: row 0 is token t0.
+ *     KV tensors (kv_raw, kv_cmp, k_idx) are whole-sequence base pointers holding at
+ *     least max_tokens (raw) or max_tokens/4 (compressed) rows.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream). The library launches kernels only; it never allocates, frees or copies
+ *     caller memory, and never synchronises the caller's stream except where stated.
+ *   - Argument, shape, order and workspace errors are returned before any launch.
+ *     A failed launch returns DS4SP_ERR_CUDA. Index checks inside the kernels never
+ *     fault: an out-of-range index is skipped and recorded in a device status word
+ *     that ds4sp_device_status() reads.
+ *   - No C++ exception crosses this ABI. A handle is not thread-safe; use one handle
+ *     per host thread, or serialise calls.
+ */
+#ifndef DS4SP_H
+#define DS4SP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ds4sp_handle ds4sp_handle; /* opaque, owned by the library */
+
+typedef enum {
+    DS4SP_OK = 0,
+    DS4SP_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad range or size */
+    DS4SP_ERR_UNSUPPORTED = 2,   /* shape outside what the kernels implement */
+    DS4SP_ERR_ORDER = 3,         /* band called out of chronological order */
+    DS4SP_ERR_WORKSPACE = 4,     /* workspace smaller than ds4sp_workspace_bytes() */
+    DS4SP_ERR_CUDA = 5,          /* a CUDA call or kernel launch failed */
+    DS4SP_ERR_DEVICE_BOUNDS = 6, /* a kernel met an out-of-range index or gave up a wait */
+} ds4sp_status;
+
+/* Model and schedule constants, fixed at ds4sp_create. Supported: n_heads = 16,
+ * d_qk = 576, d_v = 512, ratio = 4, d_idx in {64, 128}, n_idx_heads a power of two
+ * in [1, 64], top_k >= 0, n_swa >= 1, band >= 1, 1 <= max_tokens <= 2^24. */
+typedef struct {
+    int n_heads;         /* query heads sharing each latent row (16) */
+    int d_qk;            /* latent row width used as key: 512 latent + 64 rope (576) */
+    int d_v;             /* leading dims of the row used as value (512) */
+    int ratio;           /* raw tokens per compressed row (4) */
+    int n_idx_heads;     /* indexer heads H_i */
+    int d_idx;           /* indexer head dim D_i */
+    int top_k;           /* compressed rows kept per token, k */
+    int n_swa;           /* raw-row sliding window, inclusive of the token itself */
+    int band;            /* tokens per band (2048) */
+    int max_tokens;      /* sequence length T the KV buffers hold */
+    float softmax_scale; /* <= 0 selects 1/sqrt(d_qk) */
+} ds4sp_config;
+
+/* Validate cfg and create a handle bound to the current CUDA device. The handle owns
+ * a 4-byte device status word and some host state. *out is NULL on error. */
+ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out);
+
+/* Wait for every launch this handle made (it records an event after each call), then
+ * free the handle's own memory. Caller memory is never touched. NULL is accepted. */
+ds4sp_status ds4sp_destroy(ds4sp_handle* h);
+
+/* Bytes of scratch ds4sp_indexer_topk needs for query tokens [t0, t0+n_q): the fp32
+ * score rows [n_q, ld] with ld = n_vis(t0+n_q-1) rounded up to 4 floats. Returns 0 for
+ * an invalid handle or range. The scratch is caller-owned, 256-byte aligned, and may
+ * be reused as soon as the call's kernels have run. */
+size_t ds4sp_workspace_bytes(const ds4sp_handle* h, int t0, int n_q);
+
+/* Steps 1-2 for tokens [t0, t0+n_q).
+ *   q_idx [n_q, H_i, D_i] fp16, k_idx [max_tokens/4, D_i] fp16, w [n_q, H_i] fp32,
+ *   topk  [n_q, top_k] int32 (output; may be NULL when top_k == 0),
+ *   ws    scratch of ws_bytes >= ds4sp_workspace_bytes(h, t0, n_q).
+ * Scores are fp32, accumulated from fp16 products on the tensor cores; integer-valued
+ * inputs with |score| < 2^24 therefore give exact scores and exact indices. */
+ds4sp_status ds4sp_indexer_topk(ds4sp_handle* h, const void* q_idx, const void* k_idx,
+                                const float* w, int t0, int n_q, int32_t* topk,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* Step 3 for tokens [t0, t0+n_q).
+ *   q [n_q, 16, 576] fp16, kv_raw [max_tokens, 576] fp16, kv_cmp [max_tokens/4, 576]
+ *   fp16, topk [n_q, top_k] int32 as written by ds4sp_indexer_topk (entries
+ *   0 .. min(k, n_vis(t))-1 hold visible rows), out [n_q, 16, 512] fp32 (output).
+ * Rows are fp16; logits, softmax and accumulation are fp32; probabilities enter the
+ * value product as fp16. */
+ds4sp_status ds4sp_sparse_attn(ds4sp_handle* h, const void* q, const void* kv_raw,
+                               const void* kv_cmp, const int32_t* topk, int t0, int n_q,
+                               float* out, void* stream);
+
+/* Steps 1-3 for band b, tokens [b*band, min((b+1)*band, n_tokens)). Bands must come in
+ * order: b must equal the handle's next band (0 after create or ds4sp_reset), else
+ * DS4SP_ERR_ORDER; on success the next band becomes b+1. All tensor arguments are
+ * whole-sequence base pointers: q [n_tokens,16,576], q_idx [n_tokens,H_i,D_i],
+ * w [n_tokens,H_i], topk [n_tokens,top_k], out [n_tokens,16,512]; KV as above.
+ * n_tokens <= max_tokens. ws_bytes >= ds4sp_workspace_bytes(h, b*band, band-length). */
+ds4sp_status ds4sp_prefill_band(ds4sp_handle* h, int b, int n_tokens, const void* q,
+                                const void* q_idx, const float* w, const void* kv_raw,
+                                const void* kv_cmp, const void* k_idx, int32_t* topk,
+                                float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Set the band the next ds4sp_prefill_band call must name (resume or restart). */
+ds4sp_status ds4sp_reset(ds4sp_handle* h, int next_band);
+
+/* The band the next ds4sp_prefill_band call must name, or -1 for a NULL handle. */
+int ds4sp_next_band(const ds4sp_handle* h);
+
+/* Synchronise `stream`, then read and clear the handle's device status word:
+ * DS4SP_OK, or DS4SP_ERR_DEVICE_BOUNDS if a kernel skipped an out-of-range index or
+ * gave up a bounded wait since the last read. *bits (may be NULL) receives the raw
+ * word: bit 0 = index out of range, bit 1 = wait gave up. */
+ds4sp_status ds4sp_device_status(ds4sp_handle* h, void* stream, uint32_t* bits);
+
+/* Per-kernel timing. When enabled, the handle records CUDA events around each of its
+ * kernels on the launch stream. ds4sp_profile_read synchronises those events and
+ * returns, per kernel kind (0 = indexer, 1 = top-k, 2 = attention), the summed
+ * milliseconds and launch counts since the last read; then it clears them. */
+ds4sp_status ds4sp_profile_enable(ds4sp_handle* h, int enable);
+ds4sp_status ds4sp_profile_read(ds4sp_handle* h, double ms[3], int launches[3]);
+
+/* Host-side fault injection for tests: the next n kernel launches of this handle are
+ * not made, and the call that would make them returns DS4SP_ERR_CUDA. */
+ds4sp_status ds4sp_debug_fail_launches(ds4sp_handle* h, int n);
+
+/* Static description of a status code. */
+const char* ds4sp_status_string(ds4sp_status s);
+
+/* Details of the most recent error on the calling host thread ("" if none). */
+const char* ds4sp_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DS4SP_H */

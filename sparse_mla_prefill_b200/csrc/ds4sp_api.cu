@@ -1,0 +1,525 @@
+// C ABI of libds4sp (declared in include/ds4sp.h): argument checks, band order,
+// workspace sizing, TMA descriptors and kernel launches. Everything the path
+// computes runs in the kernels included below; this file only validates and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "ds4sp.h"
+#include "indexer_tcgen05.cuh"
+#include "sparse_attn_mma.cuh"
+#include "topk_radix.cuh"
+
+using namespace ds4sp;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+ds4sp_status fail(ds4sp_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+ds4sp_status fail(ds4sp_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+ds4sp_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(DS4SP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxTopkCandidates = 51200;  // top-k keeps a token's row in shared memory
+
+enum Kind { kIndexer = 0, kTopk = 1, kAttn = 2 };
+
+struct TimedLaunch {
+    int kind;
+    cudaEvent_t start, stop;
+};
+
+}  // namespace
+
+struct ds4sp_handle {
+    ds4sp_config cfg;
+    int device = 0;
+    int sm_count = 148;
+    uint32_t* d_status = nullptr;
+    cudaEvent_t last = nullptr;
+    int next_band = 0;
+    int fail_launches = 0;
+    bool profiling = false;
+    std::vector<TimedLaunch> timed;
+    std::vector<cudaEvent_t> event_pool;
+    bool smem_set[3] = {false, false, false};
+};
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int nvis(int t, int ratio) { return (t + 1) / ratio; }
+
+int score_ld(int t_last, int ratio) {
+    const int nv = nvis(t_last, ratio);
+    return ((nv > 0 ? nv : 1) + 3) / 4 * 4;
+}
+
+float scale_of(const ds4sp_config& c) {
+    return c.softmax_scale > 0.f ? c.softmax_scale : 1.0f / std::sqrt((float)c.d_qk);
+}
+
+cudaEvent_t pooled_event(ds4sp_handle* h) {
+    if (!h->event_pool.empty()) {
+        cudaEvent_t e = h->event_pool.back();
+        h->event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// Runs `launch` on `stream`, honouring the fault-injection counter and recording
+// timing events when profiling is on.
+template <class F>
+ds4sp_status launch(ds4sp_handle* h, int kind, cudaStream_t stream, F&& f) {
+    if (h->fail_launches > 0) {
+        --h->fail_launches;
+        return fail(DS4SP_ERR_CUDA, "launch suppressed by ds4sp_debug_fail_launches");
+    }
+    TimedLaunch tl{kind, nullptr, nullptr};
+    if (h->profiling) {
+        tl.start = pooled_event(h);
+        tl.stop = pooled_event(h);
+        if (!tl.start || !tl.stop) return fail(DS4SP_ERR_CUDA, "cudaEventCreate failed");
+        cudaEventRecord(tl.start, stream);
+    }
+    f();
+    const cudaError_t e = cudaGetLastError();
+    if (h->profiling) {
+        cudaEventRecord(tl.stop, stream);
+        h->timed.push_back(tl);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return DS4SP_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (EncodeTiledFn) nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// 2-D fp16 row-major [rows, cols] map with a (64 x box_rows) box and 128-byte swizzle.
+bool make_tmap_2d(CUtensorMap* m, const void* base, int cols, int rows, int box_rows) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- launchers
+
+template <int D_I, int H_I>
+ds4sp_status launch_indexer(ds4sp_handle* h, const void* q_idx, const void* k_idx, const float* w,
+                            int t0, int n_q, float* scores, int ld, cudaStream_t stream) {
+    using C = IndexerTile<D_I, H_I>;
+    const int ratio = h->cfg.ratio;
+    const int t_last = t0 + n_q - 1;
+    const int n_rows = nvis(t_last, ratio);
+    if (n_rows == 0) return DS4SP_OK;  // no token of the range sees a compressed row
+    CUtensorMap tk, tq;
+    if (!make_tmap_2d(&tk, k_idx, D_I, n_rows, C::BM) ||
+        !make_tmap_2d(&tq, q_idx, D_I, n_q * H_I, C::BN))
+        return fail(DS4SP_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    static bool attr_done[2][65] = {};  // per instantiation; the attribute is per function
+    if (!attr_done[D_I / 128][H_I]) {
+        const cudaError_t e = cudaFuncSetAttribute(indexer_tcgen05_kernel<D_I, H_I>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   C::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(indexer)");
+        attr_done[D_I / 128][H_I] = true;
+    }
+    IndexerParams p;
+    p.w = w;
+    p.scores = scores;
+    p.status = h->d_status;
+    p.t0 = t0;
+    p.n_q = n_q;
+    p.ld = ld;
+    p.ratio = ratio;
+    p.n_tb = (n_q + C::TB - 1) / C::TB;
+    const int n_jt_max = (n_rows + C::BM - 1) / C::BM;
+    int nsplit = 1;
+    if (p.n_tb < h->sm_count) nsplit = std::min(n_jt_max, (h->sm_count + p.n_tb - 1) / p.n_tb);
+    p.nsplit = nsplit;
+    const dim3 grid(p.n_tb * nsplit);
+    return launch(h, kIndexer, stream, [&] {
+        indexer_tcgen05_kernel<D_I, H_I><<<grid, 192, C::SMEM_BYTES, stream>>>(tk, tq, p);
+    });
+}
+
+template <int D_I>
+ds4sp_status dispatch_indexer_h(ds4sp_handle* h, const void* q_idx, const void* k_idx,
+                                const float* w, int t0, int n_q, float* scores, int ld,
+                                cudaStream_t s) {
+    switch (h->cfg.n_idx_heads) {
+        case 4: return launch_indexer<D_I, 4>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
+        case 8: return launch_indexer<D_I, 8>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
+        case 16: return launch_indexer<D_I, 16>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
+        case 32: return launch_indexer<D_I, 32>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
+        case 64: return launch_indexer<D_I, 64>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
+    }
+    return fail(DS4SP_ERR_UNSUPPORTED, "n_idx_heads %d", h->cfg.n_idx_heads);
+}
+
+ds4sp_status launch_topk(ds4sp_handle* h, const float* scores, int ld, int t0, int n_q,
+                         int32_t* topk, cudaStream_t stream) {
+    const size_t smem = (size_t)ld * 4;
+    const bool big = ld > 4096;
+    if (!h->smem_set[kTopk]) {
+        cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel<256>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kMaxTopkCandidates * 4 + 64);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(topk_radix_kernel<1024>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kMaxTopkCandidates * 4 + 64);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(topk)");
+        h->smem_set[kTopk] = true;
+    }
+    const int k = h->cfg.top_k, ratio = h->cfg.ratio;
+    return launch(h, kTopk, stream, [&] {
+        if (big)
+            topk_radix_kernel<1024><<<n_q, 1024, smem, stream>>>(scores, ld, t0, n_q, k, ratio, topk);
+        else
+            topk_radix_kernel<256><<<n_q, 256, smem, stream>>>(scores, ld, t0, n_q, k, ratio, topk);
+    });
+}
+
+ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, const void* kv_cmp,
+                         const int32_t* topk, int t0, int n_q, float* out, cudaStream_t stream) {
+    if (!h->smem_set[kAttn]) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            sparse_attn_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, attn::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention)");
+        h->smem_set[kAttn] = true;
+    }
+    AttnParams p;
+    p.q = static_cast<const __half*>(q);
+    p.kv_raw = static_cast<const __half*>(kv_raw);
+    p.kv_cmp = static_cast<const __half*>(kv_cmp);
+    p.topk = topk;
+    p.out = out;
+    p.status = h->d_status;
+    p.t0 = t0;
+    p.n_q = n_q;
+    p.k = h->cfg.top_k;
+    p.n_swa = h->cfg.n_swa;
+    p.ratio = h->cfg.ratio;
+    p.scale_log2 = scale_of(h->cfg) * 1.4426950408889634f;
+    return launch(h, kAttn, stream, [&] {
+        sparse_attn_mma_kernel<<<n_q, attn::THREADS, attn::SMEM_BYTES, stream>>>(p);
+    });
+}
+
+ds4sp_status check_handle(const ds4sp_handle* h) {
+    if (!h) return fail(DS4SP_ERR_INVALID_ARG, "null handle");
+    return DS4SP_OK;
+}
+
+ds4sp_status check_range(const ds4sp_handle* h, int t0, int n_q) {
+    if (t0 < 0 || n_q < 0 || (long long)t0 + n_q > h->cfg.max_tokens)
+        return fail(DS4SP_ERR_INVALID_ARG, "token range [%d, %d+%d) outside [0, %d)", t0, t0, n_q,
+                    h->cfg.max_tokens);
+    return DS4SP_OK;
+}
+
+ds4sp_status check_ptr(const void* p, const char* name) {
+    if (!p) return fail(DS4SP_ERR_INVALID_ARG, "%s is null", name);
+    if (!aligned16(p)) return fail(DS4SP_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return DS4SP_OK;
+}
+
+#define DS4SP_TRY(x)                      \
+    do {                                  \
+        const ds4sp_status s_ = (x);      \
+        if (s_ != DS4SP_OK) return s_;    \
+    } while (0)
+
+ds4sp_status record_last(ds4sp_handle* h, cudaStream_t stream) {
+    const cudaError_t e = cudaEventRecord(h->last, stream);
+    return e == cudaSuccess ? DS4SP_OK : cuda_fail(e, "cudaEventRecord");
+}
+
+ds4sp_status indexer_topk_impl(ds4sp_handle* h, const void* q_idx, const void* k_idx,
+                               const float* w, int t0, int n_q, int32_t* topk, void* ws,
+                               size_t ws_bytes, cudaStream_t stream) {
+    DS4SP_TRY(check_range(h, t0, n_q));
+    if (n_q == 0) return DS4SP_OK;
+    const int k = h->cfg.top_k;
+    if (k == 0) return DS4SP_OK;  // nothing to select, nothing to write
+    const int t_last = t0 + n_q - 1;
+    DS4SP_TRY(check_ptr(q_idx, "q_idx"));
+    if (nvis(t_last, h->cfg.ratio) > 0) DS4SP_TRY(check_ptr(k_idx, "k_idx"));
+    DS4SP_TRY(check_ptr(w, "w"));
+    DS4SP_TRY(check_ptr(topk, "topk"));
+    DS4SP_TRY(check_ptr(ws, "ws"));
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return fail(DS4SP_ERR_INVALID_ARG, "ws is not 256-byte aligned");
+    if (nvis(t_last, h->cfg.ratio) > kMaxTopkCandidates)
+        return fail(DS4SP_ERR_UNSUPPORTED, "%d candidate rows exceed the top-k limit %d",
+                    nvis(t_last, h->cfg.ratio), kMaxTopkCandidates);
+    const size_t need = ds4sp_workspace_bytes(h, t0, n_q);
+    if (ws_bytes < need)
+        return fail(DS4SP_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    const int ld = score_ld(t_last, h->cfg.ratio);
+    float* scores = static_cast<float*>(ws);
+    const ds4sp_status s =
+        h->cfg.d_idx == 64
+            ? dispatch_indexer_h<64>(h, q_idx, k_idx, w, t0, n_q, scores, ld, stream)
+            : dispatch_indexer_h<128>(h, q_idx, k_idx, w, t0, n_q, scores, ld, stream);
+    DS4SP_TRY(s);
+    DS4SP_TRY(launch_topk(h, scores, ld, t0, n_q, topk, stream));
+    return record_last(h, stream);
+}
+
+ds4sp_status sparse_attn_impl(ds4sp_handle* h, const void* q, const void* kv_raw,
+                              const void* kv_cmp, const int32_t* topk, int t0, int n_q,
+                              float* out, cudaStream_t stream) {
+    DS4SP_TRY(check_range(h, t0, n_q));
+    if (n_q == 0) return DS4SP_OK;
+    DS4SP_TRY(check_ptr(q, "q"));
+    DS4SP_TRY(check_ptr(kv_raw, "kv_raw"));
+    DS4SP_TRY(check_ptr(out, "out"));
+    if (h->cfg.top_k > 0) {
+        DS4SP_TRY(check_ptr(topk, "topk"));
+        if (nvis(t0 + n_q - 1, h->cfg.ratio) > 0) DS4SP_TRY(check_ptr(kv_cmp, "kv_cmp"));
+    }
+    DS4SP_TRY(launch_attn(h, q, kv_raw, kv_cmp, topk, t0, n_q, out, stream));
+    return record_last(h, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
+    if (!out) return fail(DS4SP_ERR_INVALID_ARG, "out is null");
+    *out = nullptr;
+    if (!cfg) return fail(DS4SP_ERR_INVALID_ARG, "cfg is null");
+    const ds4sp_config& c = *cfg;
+    if (c.n_heads != 16 || c.d_qk != 576 || c.d_v != 512 || c.ratio != 4)
+        return fail(DS4SP_ERR_UNSUPPORTED, "supported: n_heads 16, d_qk 576, d_v 512, ratio 4");
+    if (c.d_idx != 64 && c.d_idx != 128)
+        return fail(DS4SP_ERR_UNSUPPORTED, "d_idx %d (supported: 64, 128)", c.d_idx);
+    if (c.n_idx_heads < 4 || c.n_idx_heads > 64 || (c.n_idx_heads & (c.n_idx_heads - 1)))
+        return fail(DS4SP_ERR_UNSUPPORTED, "n_idx_heads %d (supported: 4, 8, 16, 32, 64)",
+                    c.n_idx_heads);
+    if (c.top_k < 0 || c.n_swa < 1 || c.band < 1 || c.max_tokens < 1 || c.max_tokens > (1 << 24) ||
+        !(c.softmax_scale == c.softmax_scale))
+        return fail(DS4SP_ERR_INVALID_ARG, "top_k >= 0, n_swa >= 1, band >= 1, "
+                                           "1 <= max_tokens <= 2^24 and a finite scale required");
+    ds4sp_handle* h = new (std::nothrow) ds4sp_handle();
+    if (!h) return fail(DS4SP_ERR_INVALID_ARG, "out of host memory");
+    h->cfg = c;
+    cudaError_t e = cudaGetDevice(&h->device);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, h->device);
+    if (e == cudaSuccess) e = cudaMalloc(&h->d_status, sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMemset(h->d_status, 0, sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->last, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+        ds4sp_destroy(h);
+        return cuda_fail(e, "ds4sp_create");
+    }
+    *out = h;
+    return DS4SP_OK;
+}
+
+ds4sp_status ds4sp_destroy(ds4sp_handle* h) {
+    if (!h) return DS4SP_OK;
+    ds4sp_status s = DS4SP_OK;
+    if (h->last && cudaEventSynchronize(h->last) != cudaSuccess)
+        s = fail(DS4SP_ERR_CUDA, "pending work failed before destroy");
+    for (auto& tl : h->timed) {
+        cudaEventSynchronize(tl.stop);
+        cudaEventDestroy(tl.start);
+        cudaEventDestroy(tl.stop);
+    }
+    for (auto e : h->event_pool) cudaEventDestroy(e);
+    if (h->last) cudaEventDestroy(h->last);
+    if (h->d_status) cudaFree(h->d_status);
+    delete h;
+    return s;
+}
+
+size_t ds4sp_workspace_bytes(const ds4sp_handle* h, int t0, int n_q) {
+    if (!h || t0 < 0 || n_q <= 0 || (long long)t0 + n_q > h->cfg.max_tokens) return 0;
+    const int ld = score_ld(t0 + n_q - 1, h->cfg.ratio);
+    const size_t bytes = (size_t)n_q * ld * sizeof(float);
+    return (bytes + 255) / 256 * 256;
+}
+
+ds4sp_status ds4sp_indexer_topk(ds4sp_handle* h, const void* q_idx, const void* k_idx,
+                                const float* w, int t0, int n_q, int32_t* topk, void* ws,
+                                size_t ws_bytes, void* stream) {
+    DS4SP_TRY(check_handle(h));
+    return indexer_topk_impl(h, q_idx, k_idx, w, t0, n_q, topk, ws, ws_bytes,
+                             static_cast<cudaStream_t>(stream));
+}
+
+ds4sp_status ds4sp_sparse_attn(ds4sp_handle* h, const void* q, const void* kv_raw,
+                               const void* kv_cmp, const int32_t* topk, int t0, int n_q,
+                               float* out, void* stream) {
+    DS4SP_TRY(check_handle(h));
+    return sparse_attn_impl(h, q, kv_raw, kv_cmp, topk, t0, n_q, out,
+                            static_cast<cudaStream_t>(stream));
+}
+
+ds4sp_status ds4sp_prefill_band(ds4sp_handle* h, int b, int n_tokens, const void* q,
+                                const void* q_idx, const float* w, const void* kv_raw,
+                                const void* kv_cmp, const void* k_idx, int32_t* topk,
+                                float* out, void* ws, size_t ws_bytes, void* stream) {
+    DS4SP_TRY(check_handle(h));
+    const ds4sp_config& c = h->cfg;
+    if (n_tokens < 1 || n_tokens > c.max_tokens)
+        return fail(DS4SP_ERR_INVALID_ARG, "n_tokens %d outside [1, %d]", n_tokens, c.max_tokens);
+    if (b < 0 || (long long)b * c.band >= n_tokens)
+        return fail(DS4SP_ERR_INVALID_ARG, "band %d outside the %d-token sequence", b, n_tokens);
+    if (b != h->next_band)
+        return fail(DS4SP_ERR_ORDER, "band %d called, band %d expected next", b, h->next_band);
+    DS4SP_TRY(check_ptr(q, "q"));
+    DS4SP_TRY(check_ptr(q_idx, "q_idx"));
+    DS4SP_TRY(check_ptr(w, "w"));
+    DS4SP_TRY(check_ptr(kv_raw, "kv_raw"));
+    DS4SP_TRY(check_ptr(out, "out"));
+    const int t0 = b * c.band;
+    const int n_q = std::min(c.band, n_tokens - t0);
+    if (c.top_k > 0) {
+        DS4SP_TRY(check_ptr(topk, "topk"));
+        if (nvis(t0 + n_q - 1, c.ratio) > 0) {   // some token of the band sees a compressed row
+            DS4SP_TRY(check_ptr(kv_cmp, "kv_cmp"));
+            DS4SP_TRY(check_ptr(k_idx, "k_idx"));
+        }
+    }
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto* qh = static_cast<const __half*>(q) + (size_t)t0 * c.n_heads * c.d_qk;
+    auto* qi = static_cast<const __half*>(q_idx) + (size_t)t0 * c.n_idx_heads * c.d_idx;
+    const float* wt = w + (size_t)t0 * c.n_idx_heads;
+    int32_t* tk = c.top_k > 0 ? topk + (size_t)t0 * c.top_k : nullptr;
+    float* ot = out + (size_t)t0 * c.n_heads * c.d_v;
+    if (c.top_k > 0) {
+        if (ws_bytes < ds4sp_workspace_bytes(h, t0, n_q))
+            return fail(DS4SP_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes,
+                        ds4sp_workspace_bytes(h, t0, n_q));
+        DS4SP_TRY(indexer_topk_impl(h, qi, k_idx, wt, t0, n_q, tk, ws, ws_bytes, s));
+    }
+    DS4SP_TRY(sparse_attn_impl(h, qh, kv_raw, kv_cmp, tk, t0, n_q, ot, s));
+    h->next_band = b + 1;
+    return DS4SP_OK;
+}
+
+ds4sp_status ds4sp_reset(ds4sp_handle* h, int next_band) {
+    DS4SP_TRY(check_handle(h));
+    if (next_band < 0) return fail(DS4SP_ERR_INVALID_ARG, "next_band %d < 0", next_band);
+    h->next_band = next_band;
+    return DS4SP_OK;
+}
+
+int ds4sp_next_band(const ds4sp_handle* h) { return h ? h->next_band : -1; }
+
+ds4sp_status ds4sp_device_status(ds4sp_handle* h, void* stream, uint32_t* bits) {
+    DS4SP_TRY(check_handle(h));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemcpy(&word, h->d_status, sizeof(word), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(h->d_status, 0, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "ds4sp_device_status");
+    if (bits) *bits = word;
+    if (word) return fail(DS4SP_ERR_DEVICE_BOUNDS, "device status word 0x%x", word);
+    return DS4SP_OK;
+}
+
+ds4sp_status ds4sp_profile_enable(ds4sp_handle* h, int enable) {
+    DS4SP_TRY(check_handle(h));
+    h->profiling = enable != 0;
+    return DS4SP_OK;
+}
+
+ds4sp_status ds4sp_profile_read(ds4sp_handle* h, double ms[3], int launches[3]) {
+    DS4SP_TRY(check_handle(h));
+    if (!ms || !launches) return fail(DS4SP_ERR_INVALID_ARG, "null output");
+    for (int k = 0; k < 3; ++k) {
+        ms[k] = 0.0;
+        launches[k] = 0;
+    }
+    ds4sp_status st = DS4SP_OK;
+    for (auto& tl : h->timed) {
+        float m = 0.f;
+        cudaError_t e = cudaEventSynchronize(tl.stop);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&m, tl.start, tl.stop);
+        if (e != cudaSuccess && st == DS4SP_OK) st = cuda_fail(e, "ds4sp_profile_read");
+        ms[tl.kind] += m;
+        launches[tl.kind] += 1;
+        h->event_pool.push_back(tl.start);
+        h->event_pool.push_back(tl.stop);
+    }
+    h->timed.clear();
+    return st;
+}
+
+ds4sp_status ds4sp_debug_fail_launches(ds4sp_handle* h, int n) {
+    DS4SP_TRY(check_handle(h));
+    if (n < 0) return fail(DS4SP_ERR_INVALID_ARG, "n < 0");
+    h->fail_launches = n;
+    return DS4SP_OK;
+}
+
+const char* ds4sp_status_string(ds4sp_status s) {
+    switch (s) {
+        case DS4SP_OK: return "ok";
+        case DS4SP_ERR_INVALID_ARG: return "invalid argument";
+        case DS4SP_ERR_UNSUPPORTED: return "unsupported shape";
+        case DS4SP_ERR_ORDER: return "band out of order";
+        case DS4SP_ERR_WORKSPACE: return "workspace too small";
+        case DS4SP_ERR_CUDA: return "CUDA error";
+        case DS4SP_ERR_DEVICE_BOUNDS: return "device index or wait check failed";
+    }
+    return "unknown status";
+}
+
+const char* ds4sp_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"
