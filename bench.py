@@ -87,7 +87,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -144,7 +144,8 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     inputs_np = {k: v.numpy() for k, v in generate(wl).items()}
-    per_step = 256
+    # a bounded sample per step, so that the whole run stays within a few minutes
+    per_step = max(8, min(256, 8192 // max(1, args.steps)))
     for _ in range(args.warmup):
         cpu_oracle_sample(wl, 32, inputs_np)
     vals = []
@@ -152,7 +153,7 @@ def run_reference(args, rank, world):
     for _ in range(args.steps):
         vals.append(cpu_oracle_sample(wl, per_step, inputs_np))
     wall = time.perf_counter() - t0
-    value = args.steps * len(range(0, per_step)) / wall
+    value = args.steps * per_step / wall
     cb = dict(vals[-1])
     cb["value"] = value
     cb["sample"] = f"{args.steps} steps x {per_step} tokens spread over the {wl.T}-token sequence"
@@ -302,10 +303,10 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-sample", type=int, default=2048)
+    ap.add_argument("--cpu-sample", type=int, default=8192)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
