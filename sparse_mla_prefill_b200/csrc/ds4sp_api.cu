@@ -179,13 +179,15 @@ ds4sp_status launch_indexer(ds4sp_handle* h, const void* q_idx, const void* k_id
     p.ld = ld;
     p.ratio = ratio;
     p.n_tb = (n_q + C::TB - 1) / C::TB;
+    // Split the j-tiles of each token block until there are about eight units per SM,
+    // keeping at least two tiles per unit; CTAs are persistent, one per SM.
     const int n_jt_max = (n_rows + C::BM - 1) / C::BM;
     int nsplit = 1;
-    if (p.n_tb < h->sm_count) nsplit = std::min(n_jt_max, (h->sm_count + p.n_tb - 1) / p.n_tb);
+    while (p.n_tb * nsplit < 8 * h->sm_count && n_jt_max / (2 * nsplit) >= 2) nsplit *= 2;
     p.nsplit = nsplit;
-    const dim3 grid(p.n_tb * nsplit);
+    const int grid = std::min(p.n_tb * nsplit, h->sm_count);
     return launch(h, kIndexer, stream, [&] {
-        indexer_tcgen05_kernel<D_I, H_I><<<grid, 192, C::SMEM_BYTES, stream>>>(tk, tq, p);
+        indexer_tcgen05_kernel<D_I, H_I><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tq, p);
     });
 }
 
@@ -229,9 +231,11 @@ ds4sp_status launch_topk(ds4sp_handle* h, const float* scores, int ld, int t0, i
 
 ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, const void* kv_cmp,
                          const int32_t* topk, int t0, int n_q, float* out, cudaStream_t stream) {
+    const int smem = attn::smem_bytes(h->cfg.top_k);
     if (!h->smem_set[kAttn]) {
-        const cudaError_t e = cudaFuncSetAttribute(
-            sparse_attn_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, attn::SMEM_BYTES);
+        const cudaError_t e = cudaFuncSetAttribute(sparse_attn_mma_kernel,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   attn::smem_bytes(attn::MAX_TOPK));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention)");
         h->smem_set[kAttn] = true;
     }
@@ -249,7 +253,9 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
     p.ratio = h->cfg.ratio;
     p.scale_log2 = scale_of(h->cfg) * 1.4426950408889634f;
     return launch(h, kAttn, stream, [&] {
-        sparse_attn_mma_kernel<<<n_q, attn::THREADS, attn::SMEM_BYTES, stream>>>(p);
+        // persistent: one CTA per SM, each walking its share of the tokens
+        const int grid = std::min(n_q, h->sm_count);
+        sparse_attn_mma_kernel<<<grid, attn::THREADS, smem, stream>>>(p);
     });
 }
 
@@ -346,6 +352,8 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
     if (c.n_idx_heads < 4 || c.n_idx_heads > 64 || (c.n_idx_heads & (c.n_idx_heads - 1)))
         return fail(DS4SP_ERR_UNSUPPORTED, "n_idx_heads %d (supported: 4, 8, 16, 32, 64)",
                     c.n_idx_heads);
+    if (c.top_k > attn::MAX_TOPK)
+        return fail(DS4SP_ERR_UNSUPPORTED, "top_k %d (supported: up to %d)", c.top_k, attn::MAX_TOPK);
     if (c.top_k < 0 || c.n_swa < 1 || c.band < 1 || c.max_tokens < 1 || c.max_tokens > (1 << 24) ||
         !(c.softmax_scale == c.softmax_scale))
         return fail(DS4SP_ERR_INVALID_ARG, "top_k >= 0, n_swa >= 1, band >= 1, "

@@ -11,10 +11,14 @@
 // and the head sum for a token runs along that lane's columns, inside one thread:
 // no cross-lane reduction. K = D_i in steps of 16.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
-// the MMAs, warps 2-5 run the epilogue (ReLU, head weights, sum, store). Two TMEM
-// accumulators (2 x 256 columns) let the epilogue of tile i overlap the MMAs of
-// tile i+1. Every wait is bounded (device_common.cuh).
+// Work unit: one block of 256/H_i tokens and a range of its 128-row j-tiles. CTAs are
+// persistent (one per SM) and take units in snake order over a heaviest-first list.
+// Warp roles (320 threads): warp 0 issues TMA loads (q_idx block into one of two B
+// buffers, k_idx tiles as 16 KB K sub-tiles into a 4-deep ring), warp 1 owns TMEM and
+// issues the MMAs, warps 2-9 run the epilogue (ReLU, head weights, sum, store), two
+// warps per TMEM lane quarter, each on half of the columns. Two TMEM accumulators
+// (2 x 256 columns) let the epilogue of tile i overlap the MMAs of tile i+1.
+// Every wait is bounded (device_common.cuh).
 #pragma once
 
 #include <cuda.h>
@@ -29,22 +33,25 @@ struct IndexerTile {
     static constexpr int BN = 256;              // (token, head) columns per tile (UMMA N)
     static constexpr int TB = BN / H_I;         // tokens per tile
     static constexpr int KSUB = D_I / 64;       // 128-byte K sub-tiles (64 fp16 each)
-    static constexpr int A_SUB = BM * 128;      // bytes of one A sub-tile
+    static constexpr int A_SUB = BM * 128;      // bytes of one A sub-tile (one ring stage)
     static constexpr int B_SUB = BN * 128;      // bytes of one B sub-tile
-    static constexpr int A_STAGE = A_SUB * KSUB;
     static constexpr int B_BYTES = B_SUB * KSUB;
-    static constexpr int STAGES = 4;
+    static constexpr int A_STAGES = 4;
+    static constexpr int EPI_WARPS = 8;
+    static constexpr int THREADS = (2 + EPI_WARPS) * 32;
     static constexpr int TMEM_COLS = 2 * BN;
-    static constexpr int OFF_B = 0;
-    static constexpr int OFF_A = B_BYTES;
-    static constexpr int OFF_W = OFF_A + STAGES * A_STAGE;
-    static constexpr int OFF_BAR = OFF_W + BN * 4;
-    static constexpr int N_BARS = 2 * STAGES + 1 + 2 + 2 + 1;  // full, empty, b, tfull, tempty, done
+    static constexpr int OFF_B = 0;                                   // two B buffers
+    static constexpr int OFF_A = 2 * B_BYTES;
+    static constexpr int OFF_W = OFF_A + A_STAGES * A_SUB;            // two w buffers
+    static constexpr int OFF_BAR = OFF_W + 2 * BN * 4;
+    // afull[4], aempty[4], bfull[2], bempty[2], tfull[2], tempty[2], done
+    static constexpr int N_BARS = 2 * A_STAGES + 4 + 4 + 1;
     static constexpr int OFF_TMEM_PTR = OFF_BAR + N_BARS * 8;
-    static constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;  // + alignment slack
+    static constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;       // + alignment slack
     static constexpr uint32_t IDESC = umma_idesc_f16_f32(BM, BN);
     static_assert(D_I == 64 || D_I == 128, "D_i must be 64 or 128");
-    static_assert(H_I >= 1 && H_I <= 64 && (BN % H_I) == 0, "H_i must divide 256 and be <= 64");
+    static_assert(H_I >= 4 && H_I <= 64 && (BN % H_I) == 0, "H_i must be a power of two in [4, 64]");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
 struct IndexerParams {
@@ -56,29 +63,49 @@ struct IndexerParams {
     int nsplit;            // j-tile ranges per token block
 };
 
-// Wait used only while draining at exit: ignores the abort flag, still bounded.
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, uint32_t* status) {
-    bool abort = false;
-    mbar_wait(bar, parity, status, abort);
+struct IndexerUnit {
+    int tok0, tok_end, jt_begin, n_tiles;
+};
+
+template <int TB>
+__device__ __forceinline__ IndexerUnit indexer_unit(const IndexerParams& p, int u) {
+    IndexerUnit w;
+    const int tb = p.n_tb - 1 - u / p.nsplit;                 // heaviest token blocks first
+    const int split = u % p.nsplit;
+    w.tok0 = p.t0 + tb * TB;
+    w.tok_end = min(w.tok0 + TB, p.t0 + p.n_q);
+    const int n_jt = (n_vis(w.tok_end - 1, p.ratio) + 127) / 128;
+    const int chunk = (n_jt + p.nsplit - 1) / p.nsplit;
+    w.jt_begin = split * chunk;
+    w.n_tiles = max(0, min(n_jt, w.jt_begin + chunk) - w.jt_begin);
+    return w;
+}
+
+// Unit taken by CTA b in round r: snake order pairs heavy units with light ones.
+__device__ __forceinline__ int snake_unit(int r, int b, int G) {
+    return r * G + ((r & 1) ? (G - 1 - b) : b);
+}
+
+// acc.xy += a.xy * b.xy as one packed fp32x2 FMA (round-to-nearest per lane).
+__device__ __forceinline__ void ffma2(float& acc_x, float& acc_y, float a_x, float a_y, float b_x,
+                                      float b_y) {
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%0, %1};\n\t"
+        "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "+f"(acc_x), "+f"(acc_y)
+        : "f"(a_x), "f"(a_y), "f"(b_x), "f"(b_y));
 }
 
 template <int D_I, int H_I>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(IndexerTile<D_I, H_I>::THREADS, 1)
 indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_q, IndexerParams p) {
     using C = IndexerTile<D_I, H_I>;
-    // Heavy token blocks (later tokens see more rows) are launched first.
-    const int unit = blockIdx.x;
-    const int tb = p.n_tb - 1 - unit / p.nsplit;
-    const int split = unit % p.nsplit;
-    const int tok0 = p.t0 + tb * C::TB;                       // first token of the block
-    const int tok_end = min(tok0 + C::TB, p.t0 + p.n_q);
-    const int nv_last = n_vis(tok_end - 1, p.ratio);
-    const int n_jt = (nv_last + C::BM - 1) / C::BM;
-    const int chunk = (n_jt + p.nsplit - 1) / p.nsplit;
-    const int jt_begin = split * chunk;
-    const int n_tiles = min(n_jt, jt_begin + chunk) - jt_begin;
-    if (n_tiles <= 0) return;                                 // uniform across the CTA
+    const int n_units = p.n_tb * p.nsplit;
+    const int G = gridDim.x, b = blockIdx.x;
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -86,25 +113,26 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint8_t* smem = smem_raw + (base - raw_u32);
     float* sw = reinterpret_cast<float*>(smem + C::OFF_W);
     const uint32_t bar0 = base + C::OFF_BAR;
-    auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
-    const uint32_t b_bar = bar0 + 8u * (2 * C::STAGES);
-    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 1 + b); };
-    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 3 + b); };
-    const uint32_t done_bar = bar0 + 8u * (2 * C::STAGES + 5);
+    auto afull = [&](int s) { return bar0 + 8u * s; };
+    auto aempty = [&](int s) { return bar0 + 8u * (C::A_STAGES + s); };
+    auto bfull = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + i); };
+    auto bempty = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + 2 + i); };
+    auto tfull = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + 4 + i); };
+    auto tempty = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + 6 + i); };
+    const uint32_t done_bar = bar0 + 8u * (2 * C::A_STAGES + 8);
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_PTR);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);
+        for (int s = 0; s < C::A_STAGES; ++s) {
+            mbar_init(afull(s), 1);
+            mbar_init(aempty(s), 1);
         }
-        mbar_init(b_bar, 1);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), 4);   // one arrive per epilogue warp
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bfull(i), 1);
+            mbar_init(bempty(i), 1);
+            mbar_init(tfull(i), 1);
+            mbar_init(tempty(i), C::EPI_WARPS);   // one arrive per epilogue warp
         }
         mbar_init(done_bar, 1);
         fence_mbar_init();
@@ -115,11 +143,6 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         tmem_alloc(smem_u32(tmem_ptr), C::TMEM_COLS);
         tmem_relinquish();
     }
-    // Head weights of this block's tokens, in column order (col = token*H_i + h).
-    for (int c = threadIdx.x; c < C::BN; c += blockDim.x) {
-        const int tl = c / H_I;
-        sw[c] = (tok0 + tl < tok_end) ? p.w[(size_t)(tok0 - p.t0 + tl) * H_I + (c % H_I)] : 0.f;
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -127,90 +150,143 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     bool abort = false;
     if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            // B operand: the block's (token, head) rows of q_idx, loaded once.
-            mbar_arrive_expect_tx(b_bar, C::B_BYTES);
-            for (int ks = 0; ks < C::KSUB; ++ks)
-                tma_load_2d(base + C::OFF_B + ks * C::B_SUB, &tmap_q, b_bar, ks * 64,
-                            (tok0 - p.t0) * H_I);
-            int issued[C::STAGES] = {};
-            for (int it = 0; it < n_tiles; ++it) {
-                const int s = it % C::STAGES;
-                if (!mbar_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, p.status, abort)) break;
-                mbar_arrive_expect_tx(full_bar(s), C::A_STAGE);
+            int bi = 0, a_it = 0;
+            int b_issued[2] = {0, 0}, a_issued[C::A_STAGES] = {};
+            for (int r = 0; !abort; ++r) {
+                const int u = snake_unit(r, b, G);
+                if (u >= n_units) break;
+                const IndexerUnit w = indexer_unit<C::TB>(p, u);
+                if (w.n_tiles == 0) continue;
+                const int bb = bi & 1;
+                if (!mbar_wait(bempty(bb), ((bi >> 1) & 1) ^ 1, p.status, abort)) break;
+                mbar_arrive_expect_tx(bfull(bb), C::B_BYTES);
                 for (int ks = 0; ks < C::KSUB; ++ks)
-                    tma_load_2d(base + C::OFF_A + s * C::A_STAGE + ks * C::A_SUB, &tmap_k,
-                                full_bar(s), ks * 64, (jt_begin + it) * C::BM);
-                ++issued[s];
+                    tma_load_2d(base + C::OFF_B + bb * C::B_BYTES + ks * C::B_SUB, &tmap_q,
+                                bfull(bb), ks * 64, (w.tok0 - p.t0) * H_I);
+                ++b_issued[bb];
+                for (int it = 0; it < w.n_tiles && !abort; ++it) {
+                    for (int ks = 0; ks < C::KSUB; ++ks, ++a_it) {
+                        const int s = a_it % C::A_STAGES;
+                        if (!mbar_wait(aempty(s), ((a_it / C::A_STAGES) & 1) ^ 1, p.status, abort))
+                            break;
+                        mbar_arrive_expect_tx(afull(s), C::A_SUB);
+                        tma_load_2d(base + C::OFF_A + s * C::A_SUB, &tmap_k, afull(s), ks * 64,
+                                    (w.jt_begin + it) * C::BM);
+                        ++a_issued[s];
+                    }
+                }
+                ++bi;
             }
             // Every bulk copy this CTA started must land before the CTA exits.
-            mbar_drain(b_bar, 0, p.status);
-            for (int s = 0; s < C::STAGES; ++s)
-                if (issued[s]) mbar_drain(full_bar(s), (issued[s] - 1) & 1, p.status);
+            for (int i = 0; i < 2; ++i) {
+                bool d = false;
+                if (b_issued[i]) mbar_wait(bfull(i), (b_issued[i] - 1) & 1, p.status, d);
+            }
+            for (int s = 0; s < C::A_STAGES; ++s) {
+                bool d = false;
+                if (a_issued[s]) mbar_wait(afull(s), (a_issued[s] - 1) & 1, p.status, d);
+            }
         }
     } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            if (mbar_wait(b_bar, 0, p.status, abort)) {
-                for (int it = 0; it < n_tiles; ++it) {
-                    const int s = it % C::STAGES, buf = it & 1;
-                    if (!mbar_wait(tempty_bar(buf), ((it >> 1) & 1) ^ 1, p.status, abort)) break;
-                    if (!mbar_wait(full_bar(s), (it / C::STAGES) & 1, p.status, abort)) break;
-                    tc_fence_after();
+            int bi = 0, a_it = 0, tc = 0;
+            for (int r = 0; !abort; ++r) {
+                const int u = snake_unit(r, b, G);
+                if (u >= n_units) break;
+                const IndexerUnit w = indexer_unit<C::TB>(p, u);
+                if (w.n_tiles == 0) continue;
+                const int bb = bi & 1;
+                if (!mbar_wait(bfull(bb), (bi >> 1) & 1, p.status, abort)) break;
+                const uint32_t bsm = base + C::OFF_B + bb * C::B_BYTES;
+                for (int it = 0; it < w.n_tiles && !abort; ++it, ++tc) {
+                    const int buf = tc & 1;
+                    if (!mbar_wait(tempty(buf), ((tc >> 1) & 1) ^ 1, p.status, abort)) break;
                     const uint32_t d = tmem_base + buf * C::BN;
-                    const uint32_t a0 = base + C::OFF_A + s * C::A_STAGE;
-                    const uint32_t b0 = base + C::OFF_B;
+                    for (int ks = 0; ks < C::KSUB; ++ks, ++a_it) {
+                        const int s = a_it % C::A_STAGES;
+                        if (!mbar_wait(afull(s), (a_it / C::A_STAGES) & 1, p.status, abort)) break;
+                        tc_fence_after();
+                        const uint32_t asm_ = base + C::OFF_A + s * C::A_SUB;
 #pragma unroll
-                    for (int kk = 0; kk < D_I / 16; ++kk) {
-                        // k16 step kk: sub-tile kk/4, 32-byte offset inside the 128-byte row
-                        const uint32_t off = (kk % 4) * 32;
-                        const uint64_t ad = umma_desc_sw128(a0 + (kk / 4) * C::A_SUB + off);
-                        const uint64_t bd = umma_desc_sw128(b0 + (kk / 4) * C::B_SUB + off);
-                        umma_f16(d, ad, bd, C::IDESC, kk > 0);
+                        for (int kk = 0; kk < 4; ++kk)   // k16 steps: 32 bytes into the 128-byte row
+                            umma_f16(d, umma_desc_sw128(asm_ + kk * 32),
+                                     umma_desc_sw128(bsm + ks * C::B_SUB + kk * 32), C::IDESC,
+                                     ks > 0 || kk > 0);
+                        umma_commit(aempty(s));          // A sub-tile free once these finish
                     }
-                    umma_commit(empty_bar(s));     // A stage free once these MMAs finish
-                    umma_commit(tfull_bar(buf));   // accumulator ready for the epilogue
+                    umma_commit(tfull(buf));             // accumulator ready for the epilogue
                 }
+                umma_commit(bempty(bb));                 // B buffer free once the unit's MMAs finish
+                ++bi;
             }
             // All MMAs issued by this thread must finish before TMEM is released.
             umma_commit(done_bar);
-            mbar_drain(done_bar, 0, p.status);
+            bool d = false;
+            mbar_wait(done_bar, 0, p.status, d);
         }
         __syncwarp();
     } else {
-        // Epilogue: warp w reads TMEM lanes 32*(w%4) .. 32*(w%4)+31.
-        const int quarter = warp & 3;
-        const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-        for (int it = 0; it < n_tiles; ++it) {
-            const int buf = it & 1;
-            const bool ready = mbar_wait(tfull_bar(buf), (it >> 1) & 1, p.status, abort);
-            if (!__all_sync(0xffffffffu, ready)) break;   // warp-uniform before .sync.aligned loads
-            tc_fence_after();
-            // Columns are (token, head) in token-major order, so one running sum
-            // suffices: a token's sum is complete at its last head column.
-            const int j = (jt_begin + it) * C::BM + quarter * 32 + lane;
-            float acc = 0.f;
+        // ------------------------------------------------------------ epilogue
+        const int e = warp - 2;                      // 0..7
+        const int quarter = warp & 3;                // TMEM lanes 32*quarter .. +31
+        const int half = e / 4;                      // columns 128*half .. +127
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + half * 128;
+        int bi = 0, tc = 0;
+        for (int r = 0;; ++r) {
+            const int u = snake_unit(r, b, G);
+            if (u >= n_units) break;
+            const IndexerUnit w = indexer_unit<C::TB>(p, u);
+            if (w.n_tiles == 0) continue;
+            // Head weights of the unit's tokens, in column order (col = token*H_i + h).
+            float* swb = sw + (bi & 1) * C::BN;
+            {
+                const int col = e * 32 + lane, tl = col / H_I;
+                swb[col] = (w.tok0 + tl < w.tok_end)
+                               ? p.w[(size_t)(w.tok0 - p.t0 + tl) * H_I + (col % H_I)] : 0.f;
+            }
+            named_barrier(1, C::EPI_WARPS * 32);
+            const float* wh = swb + half * 128;
+            // After a wait gives up this warp keeps walking the units (waits then return at
+            // once) so that it still meets every named barrier of the epilogue warps.
+            for (int it = 0; it < w.n_tiles; ++it, ++tc) {
+                const int buf = tc & 1;
+                const bool ready = mbar_wait(tfull(buf), (tc >> 1) & 1, p.status, abort);
+                if (!__all_sync(0xffffffffu, ready)) continue;   // warp-uniform skip
+                tc_fence_after();
+                const int j = (w.jt_begin + it) * C::BM + quarter * 32 + lane;
+                float ax = 0.f, ay = 0.f;                // running sum (even, odd heads)
 #pragma unroll
-            for (int ch = 0; ch < C::BN / 32; ++ch) {
-                uint32_t v[32];
-                tmem_ld_x32(lane_addr + buf * C::BN + ch * 32, v);
-                tmem_ld_wait();
-                if (ch == C::BN / 32 - 1) {        // all of this buffer is in registers
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(tempty_bar(buf));
-                }
+                for (int pass = 0; pass < 2; ++pass) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld_x32(lane_addr + buf * C::BN + pass * 64, v0);
+                    tmem_ld_x32(lane_addr + buf * C::BN + pass * 64 + 32, v1);
+                    tmem_ld_wait();
+                    if (pass == 1) {                     // the whole accumulator is in registers
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(tempty(buf));
+                    }
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int col = ch * 32 + c;
-                    acc = fmaf(sw[col], fmaxf(__uint_as_float(v[c]), 0.f), acc);
-                    if (col % H_I == H_I - 1) {
-                        const int t = tok0 + col / H_I;
-                        if (t < tok_end && j < n_vis(t, p.ratio))
-                            p.scores[(size_t)(t - p.t0) * p.ld + j] = acc;
-                        acc = 0.f;
+                    for (int c = 0; c < 64; c += 2) {
+                        const uint32_t x0 = c < 32 ? v0[c] : v1[c - 32];
+                        const uint32_t x1 = c < 32 ? v0[c + 1] : v1[c - 31];
+                        const int col = pass * 64 + c;   // column within this warp's half
+                        const float2 wv = *reinterpret_cast<const float2*>(wh + col);
+                        ffma2(ax, ay, wv.x, wv.y, fmaxf(__uint_as_float(x0), 0.f),
+                              fmaxf(__uint_as_float(x1), 0.f));
+                        if ((col + 2) % H_I == 0) {
+                            const int t = w.tok0 + (half * 128 + col) / H_I;
+                            if (t < w.tok_end && j < n_vis(t, p.ratio))
+                                p.scores[(size_t)(t - p.t0) * p.ld + j] = ax + ay;
+                            ax = ay = 0.f;
+                        }
                     }
                 }
             }
+            ++bi;
         }
     }
 
