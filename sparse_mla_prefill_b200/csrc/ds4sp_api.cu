@@ -179,11 +179,11 @@ ds4sp_status launch_indexer(ds4sp_handle* h, const void* q_idx, const void* k_id
     p.ld = ld;
     p.ratio = ratio;
     p.n_tb = (n_q + C::TB - 1) / C::TB;
-    // Split the j-tiles of each token block until there are about eight units per SM,
-    // keeping at least two tiles per unit; CTAs are persistent, one per SM.
+    // Split the j-tiles of each token block until there are about four units per SM,
+    // keeping at least four tiles per unit; CTAs are persistent, one per SM.
     const int n_jt_max = (n_rows + C::BM - 1) / C::BM;
     int nsplit = 1;
-    while (p.n_tb * nsplit < 8 * h->sm_count && n_jt_max / (2 * nsplit) >= 2) nsplit *= 2;
+    while (p.n_tb * nsplit < 4 * h->sm_count && n_jt_max / (2 * nsplit) >= 4) nsplit *= 2;
     p.nsplit = nsplit;
     const int grid = std::min(p.n_tb * nsplit, h->sm_count);
     return launch(h, kIndexer, stream, [&] {

@@ -13,9 +13,10 @@
 //
 // Work unit: one block of 256/H_i tokens and a range of its 128-row j-tiles. CTAs are
 // persistent (one per SM) and take units in snake order over a heaviest-first list.
-// Warp roles (320 threads): warp 0 issues TMA loads (q_idx block into one of two B
-// buffers, k_idx tiles as 16 KB K sub-tiles into a 4-deep ring), warp 1 owns TMEM and
-// issues the MMAs, warps 2-9 run the epilogue (ReLU, head weights, sum, store), two
+// Warp roles (352 threads): warp 10 loads q_idx blocks into two B buffers, up to two
+// units ahead; warp 0 streams k_idx tiles as 16 KB K sub-tiles into a 4-deep ring;
+// warp 1 owns TMEM and issues the MMAs; warps 2-9 run the epilogue (ReLU, head
+// weights, sum, store), two
 // warps per TMEM lane quarter, each on half of the columns. Two TMEM accumulators
 // (2 x 256 columns) let the epilogue of tile i overlap the MMAs of tile i+1.
 // Every wait is bounded (device_common.cuh).
@@ -38,7 +39,8 @@ struct IndexerTile {
     static constexpr int B_BYTES = B_SUB * KSUB;
     static constexpr int A_STAGES = 4;
     static constexpr int EPI_WARPS = 8;
-    static constexpr int THREADS = (2 + EPI_WARPS) * 32;
+    static constexpr int B_WARP = 2 + EPI_WARPS;                      // q_idx loader
+    static constexpr int THREADS = (3 + EPI_WARPS) * 32;
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int OFF_B = 0;                                   // two B buffers
     static constexpr int OFF_A = 2 * B_BYTES;
@@ -64,7 +66,13 @@ struct IndexerParams {
 };
 
 struct IndexerUnit {
-    int tok0, tok_end, jt_begin, n_tiles;
+    int tok0, tok_end, jt_begin, n_tiles, rot;
+    // j-tile of the unit's it-th tile. Each CTA starts at its own offset so that the SMs do
+    // not all fetch the same k_idx tile from L2 at the same moment.
+    __device__ __forceinline__ int jt(int it) const {
+        const int k = it + rot;
+        return jt_begin + (k >= n_tiles ? k - n_tiles : k);
+    }
 };
 
 template <int TB>
@@ -78,6 +86,7 @@ __device__ __forceinline__ IndexerUnit indexer_unit(const IndexerParams& p, int 
     const int chunk = (n_jt + p.nsplit - 1) / p.nsplit;
     w.jt_begin = split * chunk;
     w.n_tiles = max(0, min(n_jt, w.jt_begin + chunk) - w.jt_begin);
+    w.rot = w.n_tiles > 0 ? (int)(blockIdx.x % (unsigned)w.n_tiles) : 0;
     return w;
 }
 
@@ -149,11 +158,13 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const uint32_t tmem_base = *tmem_ptr;
 
     bool abort = false;
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int bi = 0, a_it = 0;
-            int b_issued[2] = {0, 0}, a_issued[C::A_STAGES] = {};
+    if (warp == C::B_WARP || warp == 0) {
+        // ------------------------------------------------------------ TMA producers
+        // The last warp loads the q_idx blocks (B) and runs up to two units ahead; warp 0
+        // streams the k_idx sub-tiles (A). Each waits only on the ring it fills.
+        if (warp == C::B_WARP && lane == 0) {
+            int bi = 0;
+            int b_issued[2] = {0, 0};
             for (int r = 0; !abort; ++r) {
                 const int u = snake_unit(r, b, G);
                 if (u >= n_units) break;
@@ -166,17 +177,6 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     tma_load_2d(base + C::OFF_B + bb * C::B_BYTES + ks * C::B_SUB, &tmap_q,
                                 bfull(bb), ks * 64, (w.tok0 - p.t0) * H_I);
                 ++b_issued[bb];
-                for (int it = 0; it < w.n_tiles && !abort; ++it) {
-                    for (int ks = 0; ks < C::KSUB; ++ks, ++a_it) {
-                        const int s = a_it % C::A_STAGES;
-                        if (!mbar_wait(aempty(s), ((a_it / C::A_STAGES) & 1) ^ 1, p.status, abort))
-                            break;
-                        mbar_arrive_expect_tx(afull(s), C::A_SUB);
-                        tma_load_2d(base + C::OFF_A + s * C::A_SUB, &tmap_k, afull(s), ks * 64,
-                                    (w.jt_begin + it) * C::BM);
-                        ++a_issued[s];
-                    }
-                }
                 ++bi;
             }
             // Every bulk copy this CTA started must land before the CTA exits.
@@ -184,11 +184,31 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 bool d = false;
                 if (b_issued[i]) mbar_wait(bfull(i), (b_issued[i] - 1) & 1, p.status, d);
             }
+        } else if (warp == 0 && lane == 0) {
+            int a_it = 0;
+            int a_issued[C::A_STAGES] = {};
+            for (int r = 0; !abort; ++r) {
+                const int u = snake_unit(r, b, G);
+                if (u >= n_units) break;
+                const IndexerUnit w = indexer_unit<C::TB>(p, u);
+                for (int it = 0; it < w.n_tiles && !abort; ++it) {
+                    for (int ks = 0; ks < C::KSUB; ++ks, ++a_it) {
+                        const int s = a_it % C::A_STAGES;
+                        if (!mbar_wait(aempty(s), ((a_it / C::A_STAGES) & 1) ^ 1, p.status, abort))
+                            break;
+                        mbar_arrive_expect_tx(afull(s), C::A_SUB);
+                        tma_load_2d(base + C::OFF_A + s * C::A_SUB, &tmap_k, afull(s), ks * 64,
+                                    w.jt(it) * C::BM);
+                        ++a_issued[s];
+                    }
+                }
+            }
             for (int s = 0; s < C::A_STAGES; ++s) {
                 bool d = false;
                 if (a_issued[s]) mbar_wait(afull(s), (a_issued[s] - 1) & 1, p.status, d);
             }
         }
+        __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -256,33 +276,35 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const bool ready = mbar_wait(tfull(buf), (tc >> 1) & 1, p.status, abort);
                 if (!__all_sync(0xffffffffu, ready)) continue;   // warp-uniform skip
                 tc_fence_after();
-                const int j = (w.jt_begin + it) * C::BM + quarter * 32 + lane;
+                const int j = w.jt(it) * C::BM + quarter * 32 + lane;
+                // All 128 columns of this warp into registers, then release the accumulator
+                // at once so the next tile's MMAs never wait on this epilogue's arithmetic.
+                uint32_t v[4][32];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) tmem_ld_x32(lane_addr + buf * C::BN + q * 32, v[q]);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty(buf));
                 float ax = 0.f, ay = 0.f;                // running sum (even, odd heads)
 #pragma unroll
-                for (int pass = 0; pass < 2; ++pass) {
-                    uint32_t v0[32], v1[32];
-                    tmem_ld_x32(lane_addr + buf * C::BN + pass * 64, v0);
-                    tmem_ld_x32(lane_addr + buf * C::BN + pass * 64 + 32, v1);
-                    tmem_ld_wait();
-                    if (pass == 1) {                     // the whole accumulator is in registers
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(tempty(buf));
+                for (int c = 0; c < 128; c += 4) {
+                    const float4 wv = *reinterpret_cast<const float4*>(wh + c);
+                    ffma2(ax, ay, wv.x, wv.y, fmaxf(__uint_as_float(v[c / 32][c % 32]), 0.f),
+                          fmaxf(__uint_as_float(v[c / 32][c % 32 + 1]), 0.f));
+                    if ((c + 2) % H_I == 0) {
+                        const int t = w.tok0 + (half * 128 + c) / H_I;
+                        if (t < w.tok_end && j < n_vis(t, p.ratio))
+                            p.scores[(size_t)(t - p.t0) * p.ld + j] = ax + ay;
+                        ax = ay = 0.f;
                     }
-#pragma unroll
-                    for (int c = 0; c < 64; c += 2) {
-                        const uint32_t x0 = c < 32 ? v0[c] : v1[c - 32];
-                        const uint32_t x1 = c < 32 ? v0[c + 1] : v1[c - 31];
-                        const int col = pass * 64 + c;   // column within this warp's half
-                        const float2 wv = *reinterpret_cast<const float2*>(wh + col);
-                        ffma2(ax, ay, wv.x, wv.y, fmaxf(__uint_as_float(x0), 0.f),
-                              fmaxf(__uint_as_float(x1), 0.f));
-                        if ((col + 2) % H_I == 0) {
-                            const int t = w.tok0 + (half * 128 + col) / H_I;
-                            if (t < w.tok_end && j < n_vis(t, p.ratio))
-                                p.scores[(size_t)(t - p.t0) * p.ld + j] = ax + ay;
-                            ax = ay = 0.f;
-                        }
+                    ffma2(ax, ay, wv.z, wv.w, fmaxf(__uint_as_float(v[c / 32][c % 32 + 2]), 0.f),
+                          fmaxf(__uint_as_float(v[c / 32][c % 32 + 3]), 0.f));
+                    if ((c + 4) % H_I == 0) {
+                        const int t = w.tok0 + (half * 128 + c + 2) / H_I;
+                        if (t < w.tok_end && j < n_vis(t, p.ratio))
+                            p.scores[(size_t)(t - p.t0) * p.ld + j] = ax + ay;
+                        ax = ay = 0.f;
                     }
                 }
             }
