@@ -72,6 +72,23 @@ def peaks():
             "source": "fallback"}
 
 
+# ------------------------------------------------------------------ ranks
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value (every rank takes part in the same all-reduce)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_throughput(tokens_per_rank: int, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -200,13 +217,6 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return t.item()
-
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -231,7 +241,7 @@ def run_ours(args, rank, world, local_rank):
     prof = D.ds4sp_profile_read(h)
     D.ds4sp_profile_enable(h, False)
     clk = clocks.stop()
-    ms_max = max_over_ranks(ms)
+    ms_max = max_over_ranks(ms, world, dev)
 
     # end to end through the public API: pinned host inputs -> device, prefill, out -> host
     pinned = {k: v.pin_memory() for k, v in host.items()}
@@ -249,7 +259,7 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     st, bits = D.ds4sp_device_status(h)
     if st != D.OK:
         raise RuntimeError(f"device status {bits:#x} after timing")
@@ -259,8 +269,7 @@ def run_ours(args, rank, world, local_rank):
         cpu_base = cpu_oracle_sample(wl, args.cpu_sample, {k: v.numpy() for k, v in host.items()})
 
     if rank == 0:
-        tokens = world * wl.T * args.steps
-        value = tokens / (ms_max / 1e3)
+        value = job_throughput(wl.T, world, args.steps, ms_max)
         attn_ms, attn_n = prof["attention"]
         idx_ms, idx_n = prof["indexer"]
         topk_ms, topk_n = prof["topk"]
@@ -291,7 +300,7 @@ def run_ours(args, rank, world, local_rank):
                          "alg_GBps": alg["topk_bytes"] * steps / (topk_ms / 1e3) / 1e9},
             },
             "gpu_launches": attn_n + idx_n + topk_n,
-            "e2e": {"value": world * wl.T * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+            "e2e": {"value": job_throughput(wl.T, world, e2e_steps, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "clocks": clk,
             "cpu_baseline": cpu_base,
