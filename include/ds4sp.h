@@ -143,6 +143,29 @@ ds4sp_status ds4sp_profile_read(ds4sp_handle* h, double ms[3], int launches[3]);
  * not made, and the call that would make them returns DS4SP_ERR_CUDA. */
 ds4sp_status ds4sp_debug_fail_launches(ds4sp_handle* h, int n);
 
+/* Steps 1-2 like ds4sp_indexer_topk, for callers that cannot allocate device memory.
+ * The paper has no counterpart to this entry point; it exists for the host side only.
+ * Some callers cannot call cudaMalloc: a framework whose allocator reserves all device
+ * memory up front (a raw cudaMalloc then fails or splits its pool), or a latency-bound
+ * loop where cudaMalloc/cudaFree would synchronise the device. This entry point needs
+ * no handle and no workspace, and calls no cudaMalloc, cudaFree or allocating library
+ * routine. Its score scratch is a fixed 8 MiB array inside the library (2^21 fp32
+ * scores); every GPU that loads the library holds that array until the process exits.
+ *   cfg     the same configuration ds4sp_create takes (validated the same way);
+ *   q_idx, k_idx, w, t0, n_q, topk, stream  as for ds4sp_indexer_topk.
+ * n_q * ld must be <= 2^21, with ld = n_vis(t0+n_q-1) rounded up to 4 (for example, a
+ * 2048-token band whose last token sees up to 1024 rows, or up to 5 tokens at a
+ * 122,880-token context); larger ranges return DS4SP_ERR_WORKSPACE before any launch.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture. All calls
+ * share the one array, which keeps the last call's scores: calls whose kernels overlap on
+ * the GPU (other streams, other threads) race on it, so serialise them. Device-side index
+ * and wait checks of this path are recorded in a library-internal word that each call
+ * clears; they are not reported to the caller. */
+ds4sp_status ds4sp_indexer_topk_noalloc(const ds4sp_config* cfg, const void* q_idx,
+                                        const void* k_idx, const float* w, int t0, int n_q,
+                                        int32_t* topk, void* stream);
+
 /* Static description of a status code. */
 const char* ds4sp_status_string(ds4sp_status s);
 

@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -531,3 +532,111 @@ const char* ds4sp_status_string(ds4sp_status s) {
 const char* ds4sp_last_error(void) { return g_last_error.c_str(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Indexer + top-k without any device allocation.
+//
+// The score scratch of ds4sp_indexer_topk_noalloc lives in the fixed-size array below,
+// which the library image carries: every GPU that loads the library holds these 8 MiB
+// (plus one status word) until the process exits. In host code `g_static_scores` is only
+// a host-side stand-in for the symbol, not a device address; the device address comes
+// from cudaGetSymbolAddress, looked up once per device with that device current.
+// ---------------------------------------------------------------------------------
+
+namespace {
+
+constexpr size_t kStaticScoreFloats = size_t(1) << 21;   // 8 MiB of fp32 scores
+
+__device__ __align__(256) float g_static_scores[kStaticScoreFloats];
+__device__ __align__(256) uint32_t g_static_status[4];
+
+struct StaticScratch {
+    float* scores = nullptr;
+    uint32_t* status = nullptr;
+    int sm_count = 0;
+    bool ready = false;
+};
+
+constexpr int kMaxDevices = 64;
+StaticScratch g_static[kMaxDevices];
+std::mutex g_static_mu;
+
+// Device addresses of the static arrays on the current device (set-up on first use).
+ds4sp_status static_scratch(StaticScratch* out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(DS4SP_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    StaticScratch& s = g_static[dev];
+    if (!s.ready) {
+        e = cudaGetSymbolAddress(reinterpret_cast<void**>(&s.scores), g_static_scores);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scores)");
+        e = cudaGetSymbolAddress(reinterpret_cast<void**>(&s.status), g_static_status);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+        e = cudaDeviceGetAttribute(&s.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        s.ready = true;
+    }
+    *out = s;
+    return DS4SP_OK;
+}
+
+ds4sp_status check_static_config(const ds4sp_config* cfg) {
+    if (!cfg) return fail(DS4SP_ERR_INVALID_ARG, "cfg is null");
+    const ds4sp_config& c = *cfg;
+    if (c.n_heads != 16 || c.d_qk != 576 || c.d_v != 512 || c.ratio != 4)
+        return fail(DS4SP_ERR_UNSUPPORTED, "supported: n_heads 16, d_qk 576, d_v 512, ratio 4");
+    if (c.d_idx != 64 && c.d_idx != 128)
+        return fail(DS4SP_ERR_UNSUPPORTED, "d_idx %d (supported: 64, 128)", c.d_idx);
+    if (c.n_idx_heads < 4 || c.n_idx_heads > 64 || (c.n_idx_heads & (c.n_idx_heads - 1)))
+        return fail(DS4SP_ERR_UNSUPPORTED, "n_idx_heads %d (supported: 4, 8, 16, 32, 64)",
+                    c.n_idx_heads);
+    if (c.top_k < 0 || c.top_k > attn::MAX_TOPK || c.max_tokens < 1 || c.max_tokens > (1 << 24))
+        return fail(DS4SP_ERR_INVALID_ARG, "0 <= top_k <= %d and 1 <= max_tokens <= 2^24 required",
+                    attn::MAX_TOPK);
+    return DS4SP_OK;
+}
+
+}  // namespace
+
+extern "C" ds4sp_status ds4sp_indexer_topk_noalloc(const ds4sp_config* cfg, const void* q_idx,
+                                                   const void* k_idx, const float* w, int t0,
+                                                   int n_q, int32_t* topk, void* stream) {
+    DS4SP_TRY(check_static_config(cfg));
+    if (t0 < 0 || n_q < 0 || (long long)t0 + n_q > cfg->max_tokens)
+        return fail(DS4SP_ERR_INVALID_ARG, "token range [%d, %d+%d) outside [0, %d)", t0, t0, n_q,
+                    cfg->max_tokens);
+    if (n_q == 0 || cfg->top_k == 0) return DS4SP_OK;
+    const int ld = score_ld(t0 + n_q - 1, cfg->ratio);
+    if ((size_t)n_q * ld > kStaticScoreFloats)
+        return fail(DS4SP_ERR_WORKSPACE,
+                    "%d tokens x %d score columns exceed the static scratch of %zu floats (8 MiB)",
+                    n_q, ld, kStaticScoreFloats);
+    StaticScratch sc;
+    DS4SP_TRY(static_scratch(&sc));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // The status word steers the kernels' bounded waits, so each call starts it at zero.
+    const cudaError_t e = cudaMemsetAsync(sc.status, 0, sizeof(uint32_t), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+    // A handle on the stack carries the launch settings; it owns no device memory.
+    ds4sp_handle tmp;
+    tmp.cfg = *cfg;
+    tmp.d_status = sc.status;
+    tmp.sm_count = sc.sm_count;
+    ds4sp_status st = DS4SP_OK;
+    const int t_last = t0 + n_q - 1;
+    st = check_ptr(q_idx, "q_idx");
+    if (st == DS4SP_OK && nvis(t_last, cfg->ratio) > 0) st = check_ptr(k_idx, "k_idx");
+    if (st == DS4SP_OK) st = check_ptr(w, "w");
+    if (st == DS4SP_OK) st = check_ptr(topk, "topk");
+    if (st == DS4SP_OK && nvis(t_last, cfg->ratio) > kMaxTopkCandidates)
+        st = fail(DS4SP_ERR_UNSUPPORTED, "%d candidate rows exceed the top-k limit %d",
+                  nvis(t_last, cfg->ratio), kMaxTopkCandidates);
+    if (st != DS4SP_OK) return st;
+    st = cfg->d_idx == 64
+             ? dispatch_indexer_h<64>(&tmp, q_idx, k_idx, w, t0, n_q, sc.scores, ld, s)
+             : dispatch_indexer_h<128>(&tmp, q_idx, k_idx, w, t0, n_q, sc.scores, ld, s);
+    if (st != DS4SP_OK) return st;
+    return launch_topk(&tmp, sc.scores, ld, t0, n_q, topk, s);
+}

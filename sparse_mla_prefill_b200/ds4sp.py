@@ -51,6 +51,8 @@ _SIGS = {
     "ds4sp_profile_enable": (_i32, [_vp, _i32]),
     "ds4sp_profile_read": (_i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i32)]),
     "ds4sp_debug_fail_launches": (_i32, [_vp, _i32]),
+    "ds4sp_indexer_topk_noalloc": (_i32, [ctypes.POINTER(ds4sp_config), _vp, _vp, _vp, _i32,
+                                          _i32, _vp, _vp]),
     "ds4sp_status_string": (ctypes.c_char_p, [_i32]),
     "ds4sp_last_error": (ctypes.c_char_p, []),
 }
@@ -160,6 +162,18 @@ def ds4sp_indexer_topk(h: Handle, q_idx, k_idx, w, t0: int, n_q: int, topk, ws, 
                                   _ptr(topk, "topk", torch.int32), _ptr(ws, "ws"),
                                   ws.numel() * ws.element_size() if ws is not None else 0,
                                   _stream(stream)), "ds4sp_indexer_topk")
+
+
+def ds4sp_indexer_topk_noalloc(cfg: ds4sp_config, q_idx, k_idx, w, t0: int, n_q: int, topk,
+                               stream=None):
+    """Indexer + top-k with the library's fixed 8 MiB score scratch: no handle, no
+    workspace, no device allocation (see include/ds4sp.h)."""
+    lib = load_library()
+    _check(lib.ds4sp_indexer_topk_noalloc(ctypes.byref(cfg), _ptr(q_idx, "q_idx", torch.float16),
+                                          _ptr(k_idx, "k_idx", torch.float16),
+                                          _ptr(w, "w", torch.float32), t0, n_q,
+                                          _ptr(topk, "topk", torch.int32), _stream(stream)),
+           "ds4sp_indexer_topk_noalloc")
 
 
 def ds4sp_sparse_attn(h: Handle, q, kv_raw, kv_cmp, topk, t0: int, n_q: int, out, stream=None):
