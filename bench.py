@@ -72,6 +72,26 @@ def peaks():
             "source": "fallback"}
 
 
+def attention_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, or None when the
+    kernel's sources changed after that capture (the figure would no longer apply)."""
+    import hashlib
+    import re
+    prof = os.path.join(ROOT, "profiles", "sparse_attn_mma_kernel_10k_band4.md")
+    csrc = os.path.join(ROOT, "sparse_mla_prefill_b200", "csrc")
+    try:
+        text = open(prof).read()
+        src = b"".join(open(os.path.join(csrc, f), "rb").read()
+                       for f in ("sparse_attn_mma.cuh", "device_common.cuh"))
+    except OSError:
+        return None
+    want = re.search(r"kernel_source_sha256: ([0-9a-f]+)", text)
+    val = re.search(r"traffic_bytes_per_launch: ([0-9]+)", text)
+    if not want or not val or hashlib.sha256(src).hexdigest()[:16] != want.group(1):
+        return None
+    return int(val.group(1))
+
+
 # ------------------------------------------------------------------ ranks
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -285,7 +305,7 @@ def run_ours(args, rank, world, local_rank):
                        "l2": "inputs larger than L2: q+q_idx read and out written per step = 692 MB > 126 MB"},
             "roofline": {"bound": "hbm", "achieved": attn_achieved, "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": attn_achieved / pk["hbm_gbs"],
-                         "traffic": None, "kernel": "sparse_attn_mma_kernel",
+                         "traffic": attention_traffic(), "kernel": "sparse_attn_mma_kernel",
                          "peak_source": f"{pk['source']} hbm_gbs (of {pk['source']})"},
             "kernels": {
                 "attention": {"ms_per_step": attn_ms / steps, "launches": attn_n,
