@@ -60,7 +60,8 @@ typedef enum {
 
 /* Model and schedule constants, fixed at ds4sp_create. Supported: n_heads = 16,
  * d_qk = 576, d_v = 512, ratio = 4, d_idx in {64, 128}, n_idx_heads a power of two
- * in [1, 64], top_k >= 0, n_swa >= 1, band >= 1, 1 <= max_tokens <= 2^24. */
+ * in [4, 64], 0 <= top_k <= 2048, n_swa >= 1, band >= 1, 1 <= max_tokens <= 2^24;
+ * a token may see at most 51,200 compressed rows (top-k keeps a row in shared memory). */
 typedef struct {
     int n_heads;         /* query heads sharing each latent row (16) */
     int d_qk;            /* latent row width used as key: 512 latent + 64 rope (576) */

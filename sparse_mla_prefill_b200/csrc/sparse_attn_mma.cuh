@@ -8,22 +8,26 @@
 // heads". The per-token visibility (n_vis = (t+1)/4, window bounds) is computed
 // here from t; no mask is stored.
 //
-// Persistent CTAs (one per SM) walk their tokens heaviest first. Warp 8 is the
-// producer: while it issues one token's rows it prefetches the next token's top-k
-// row into shared memory (4-byte cp.async), so resolving a row never waits on global
-// memory. Per 32-row block each lane resolves one row (top-k entry or window
-// position), checks it, and copies its 1152 bytes into a 4-stage shared-memory ring
-// with one cp.async.bulk; an mbarrier per stage counts the bytes in. It runs ahead
-// across token boundaries and also fetches each token's Q. Warps 0-7 consume, with
-// the 16 heads as the M of mma.sync.m16n8k16:
-//   S = Q . R^T  warp w: rows 8(w%4) .. +7 of the block, dims 288(w/4) .. +287, with
-//                its half of Q held in registers; the two K halves meet in shared memory;
-//   softmax      per-head block max across warps, online rescaling in fp32, P to
-//                shared memory as fp16;
-//   O += P . V   warp w owns value dims 64w .. 64w+63 over all 32 rows of the block.
-// fp32 logits, max, sums and output; probabilities enter P . V as fp16.
-// Waits are bounded; a wait that gives up is turned into an abort that all consumer
-// warps take together at the next named barrier, so no warp is left waiting.
+// Persistent CTAs (one per SM) walk their tokens heaviest first as a flat sequence of
+// units: per token, one unit holding its Q (16 rows), then its rows in blocks of 32.
+// Units stream through a 5-slot shared-memory ring with one mbarrier pair per slot.
+//   * Warps 8-11 produce. They stage each token's top-k row in shared memory one
+//     token ahead, resolve and check every row, and copy it in 16-byte chunks with
+//     cp.async; cp.async.mbarrier.arrive.noinc lets the slot's barrier count the copies
+//     without the producer waiting for them. Each producer warp also publishes which of
+//     its 8 rows are valid. Producers never take part in the consumers' barriers.
+//   * Warps 0-7 consume, with the 16 heads as the M of mma.sync.m16n8k16. Warp w owns
+//     row tile nt = w%4 (8 rows) and K half kh = w/4 (288 dims) of S = Q . R^T, Q held
+//     in registers; the two K halves meet in shared memory. Softmax runs against a
+//     running reference max that is raised only when a block's max exceeds it by more
+//     than 2^8 (probabilities stay <= 256, fine in fp16): a 32-row block normally needs
+//     two consumer barriers; raising the reference rescales O, the sums and that
+//     block's P in every warp. O += P . V: warp w owns value dims 64w .. 64w+63.
+// Rows are stored unpadded with their 16-byte chunks XOR-swizzled, which keeps the
+// producers' copies and the consumers' ldmatrix reads free of bank conflicts.
+// fp32 logits, sums and output; P enters P . V as fp16; exponentials on ex2.approx.
+// Every wait is bounded; a consumer that gives up sets a flag that all consumer warps
+// read at their next barrier, so none is left waiting.
 #pragma once
 
 #include "device_common.cuh"
@@ -34,31 +38,45 @@ namespace attn {
 constexpr int H = 16;
 constexpr int DQK = 576;
 constexpr int DV = 512;
-constexpr int ROW_BYTES = DQK * 2;           // 1152
-constexpr int BR = 32;                       // rows per block
-constexpr int STAGES = 4;
-constexpr int CWARPS = 8;                    // consumer warps
-constexpr int THREADS = (CWARPS + 1) * 32;   // + one producer warp
-constexpr int ROW_PITCH = ROW_BYTES + 16;    // 1168 B: staggers ldmatrix rows over banks
-constexpr int STAGE_BYTES = BR * ROW_PITCH;
-constexpr int P_PITCH = (BR + 8) * 2;        // fp16 probabilities, 80 B per head
-constexpr int OFF_STAGE = 0;
-constexpr int OFF_Q = OFF_STAGE + STAGES * STAGE_BYTES;
-constexpr int OFF_P = OFF_Q + H * ROW_PITCH;
-constexpr int OFF_SX = OFF_P + H * P_PITCH;            // S partials of the upper K half
-constexpr int OFF_RED_MAX = OFF_SX + 4 * 32 * 16;
-constexpr int OFF_RED_SUM = OFF_RED_MAX + 4 * H * 4;
-constexpr int OFF_ROWOK = OFF_RED_SUM + 4 * H * 4;
-constexpr int OFF_FLAG = OFF_ROWOK + STAGES * BR * 4;
-constexpr int OFF_BAR = (OFF_FLAG + 16 + 7) / 8 * 8;
-constexpr int N_BARS = 2 * STAGES + 2;                 // full, empty, q_full, q_empty
-constexpr int OFF_IDX = (OFF_BAR + N_BARS * 8 + 15) / 16 * 16;  // two top-k rows (int32)
-constexpr int MAX_TOPK = 4096;                          // top-k rows staged in shared memory
-__host__ __device__ constexpr int smem_bytes(int k) { return OFF_IDX + 2 * ((k + 3) / 4 * 4) * 4; }
-constexpr int CONSUMER_BAR = 1;                        // named barrier id of warps 0-7
+constexpr int ROW = DQK * 2;                  // 1152 bytes per latent row
+constexpr int CH = ROW / 16;                  // 72 sixteen-byte chunks per row
+constexpr int BR = 32;                        // rows per unit
+constexpr int NS = 5;                         // ring slots
+constexpr int CWARPS = 8;                     // consumer warps
+constexpr int PWARPS = 4;                     // producer warps
+constexpr int CTHREADS = CWARPS * 32;
+constexpr int PTHREADS = PWARPS * 32;
+constexpr int THREADS = CTHREADS + PTHREADS;
+constexpr int CONSUMER_BAR = 1;               // named barriers
+constexpr int PRODUCER_BAR = 2;
+constexpr float HEADROOM = 8.f;               // log2 units a block may exceed the reference
+constexpr int SLOT = BR * ROW;
+constexpr int P_PITCH = (BR + 8) * 2;         // fp16 probabilities, 80 B per head
+constexpr int IDX_BUFS = 2;                   // producers' top-k rows: this token, the next
+constexpr int OFF_RING = 0;
+constexpr int OFF_P = OFF_RING + NS * SLOT;
+constexpr int OFF_SX = OFF_P + H * P_PITCH;   // S partials of the upper K half
+constexpr int OFF_REF = OFF_SX + 4 * 32 * 16; // per row tile: reference used for its P
+constexpr int OFF_RED_SUM = OFF_REF + 4 * H * 4;
+constexpr int OFF_FLAGS = OFF_RED_SUM + 4 * H * 4;   // raised[2], abort, pad
+constexpr int OFF_MASK = OFF_FLAGS + 16;             // row-validity bits per slot
+constexpr int OFF_BAR = OFF_MASK + 32;               // full[NS], empty[NS]
+constexpr int OFF_IDX = OFF_BAR + 2 * NS * 8;
+constexpr int MAX_TOPK = 2048;
+__host__ __device__ constexpr int smem_bytes(int k) {
+    return OFF_IDX + IDX_BUFS * ((k + 3) / 4 * 4) * 4;
+}
 static_assert(DV == CWARPS * 64, "each consumer warp owns 64 value dims");
-static_assert(BR == 32, "one producer lane per row");
-static_assert((OFF_Q % 16) == 0 && (ROW_PITCH % 16) == 0, "bulk copies need 16-byte alignment");
+static_assert(CH % 8 == 0 && BR * CH == PTHREADS * 18, "producer chunk split");
+static_assert(smem_bytes(MAX_TOPK) <= 227 * 1024, "shared memory budget");
+
+// 16-byte chunk swizzle: eight consecutive rows put one chunk in eight different bank
+// groups (ldmatrix), and rows 2m, 2m+1 put an aligned group of four chunks in
+// complementary halves (a quarter warp's cp.async).
+__device__ __forceinline__ int swz(int row) { return ((row & 1) << 2) | ((row >> 1) & 3); }
+__device__ __forceinline__ uint32_t chunk_addr(uint32_t slot, int row, int chunk) {
+    return slot + row * ROW + ((chunk ^ swz(row)) << 4);
+}
 
 }  // namespace attn
 
@@ -89,209 +107,234 @@ __device__ __forceinline__ TokenRows token_rows(const AttnParams& p, int idx) {
     return r;
 }
 
+// Position in a CTA's flat unit sequence: token number n (the CTA's n-th token), unit u
+// (0 = Q, 1.. = row blocks).
+struct UnitCursor {
+    int n, idx, u;
+    TokenRows tr;
+    bool valid;
+    __device__ __forceinline__ void start(const AttnParams& p) {
+        n = 0;
+        idx = blockIdx.x;
+        u = 0;
+        valid = idx < p.n_q;
+        if (valid) tr = token_rows(p, idx);
+    }
+    __device__ __forceinline__ void advance(const AttnParams& p) {
+        if (!valid) return;
+        if (++u > tr.nblk) {
+            u = 0;
+            ++n;
+            idx += gridDim.x;
+            valid = idx < p.n_q;
+            if (valid) tr = token_rows(p, idx);
+        }
+    }
+};
+
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnParams p) {
     using namespace attn;
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
-    float* red_max = reinterpret_cast<float*>(smem + OFF_RED_MAX);
-    float* red_sum = reinterpret_cast<float*>(smem + OFF_RED_SUM);
-    int* rowok = reinterpret_cast<int*>(smem + OFF_ROWOK);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_FLAG);
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int kpad = (p.k + 3) / 4 * 4;
+    volatile int* flags = reinterpret_cast<volatile int*>(smem + OFF_FLAGS);  // raised[2], abort
+    volatile uint32_t* rowmask = reinterpret_cast<volatile uint32_t*>(smem + OFF_MASK);
     const uint32_t bar0 = sbase + OFF_BAR;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-    const uint32_t qfull_bar = bar0 + 8u * (2 * STAGES);
-    const uint32_t qempty_bar = bar0 + 8u * (2 * STAGES + 1);
+    auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
 
-    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     if (tid == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(full_bar(s), PTHREADS + PWARPS);   // noinc copy arrivals + mask writers
             mbar_init(empty_bar(s), CWARPS);
         }
-        mbar_init(qfull_bar, 1);
-        mbar_init(qempty_bar, CWARPS);
-        *abort_flag = 0;
+        flags[0] = flags[1] = flags[2] = 0;
         fence_mbar_init();
     }
     __syncthreads();
 
     bool abort = false;
-    if (warp == CWARPS) {
-        // ------------------------------------------------------------ producer
-        int it = 0, ntok = 0;
-        int issued[STAGES] = {};
-        bool q_issued = false;
-        const int kpad = (p.k + 3) / 4 * 4;
-        int* sidx = reinterpret_cast<int*>(smem + OFF_IDX);
-        // Stage the selected entries of a token's top-k row in buffer `buf`.
-        auto prefetch_idx = [&](int idx, int buf) {
-            if (idx < p.n_q) {
-                const TokenRows nx = token_rows(p, idx);
-                const int32_t* src = p.topk + (size_t)nx.i * p.k;
-                const uint32_t dst = sbase + OFF_IDX + buf * kpad * 4;
-                for (int g = lane; g < nx.nsel; g += 32)
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst + 4 * g),
-                                 "l"(src + g)
-                                 : "memory");
-            }
-            cp_async_commit();
+    if (warp >= CWARPS) {
+        // ================================================================ producers
+        const int ptid = tid - CTHREADS, pw = warp - CWARPS;
+        auto stage_idx = [&](int n) {             // top-k row of the CTA's token number n
+            const int idx = blockIdx.x + n * gridDim.x;
+            if (idx >= p.n_q) return;
+            const TokenRows nx = token_rows(p, idx);
+            const int32_t* src = p.topk + (size_t)nx.i * p.k;
+            const uint32_t dst = sbase + OFF_IDX + (n % IDX_BUFS) * kpad * 4;
+            for (int e = ptid; e < nx.nsel; e += PTHREADS)
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst + 4 * e),
+                             "l"(src + e)
+                             : "memory");
         };
-        prefetch_idx(blockIdx.x, 0);
-        for (int idx = blockIdx.x; idx < p.n_q && !abort; idx += gridDim.x, ++ntok) {
-            const TokenRows tr = token_rows(p, idx);
-            cp_async_wait<0>();                   // this token's top-k row is in shared memory
-            __syncwarp();
-            const int* tk = sidx + (ntok & 1) * kpad;
-            prefetch_idx(idx + gridDim.x, (ntok + 1) & 1);   // lands while this token streams
-            if (!__all_sync(0xffffffffu, mbar_wait(qempty_bar, (ntok & 1) ^ 1, p.status, abort))) {
-                abort = true;                      // warp-uniform from here on
-                break;
-            }
-            if (lane == 0) mbar_arrive_expect_tx(qfull_bar, H * ROW_BYTES);
-            __syncwarp();
-            if (lane < H)
-                bulk_load(sbase + OFF_Q + lane * ROW_PITCH, p.q + ((size_t)tr.i * H + lane) * DQK,
-                          ROW_BYTES, qfull_bar);
-            q_issued = true;
-            for (int blk = 0; blk < tr.nblk; ++blk, ++it) {
-                const int s = it % STAGES;
-                // Resolve this lane's row before waiting for the stage to free up.
-                const int gr = blk * BR + lane;
-                const __half* src = p.kv_raw + (size_t)tr.t * DQK;   // harmless stand-in
-                int ok = 0;
-                if (gr < tr.nsel) {
-                    const int j = tk[gr];
-                    if (j >= 0 && j < tr.nv) {
-                        src = p.kv_cmp + (size_t)j * DQK;
-                        ok = 1;
-                    } else {
-                        record_status(p.status, kStatusBounds);
-                    }
-                } else if (gr < tr.nrows) {
-                    src = p.kv_raw + (size_t)(tr.s_lo + gr - tr.nsel) * DQK;
-                    ok = 1;
-                }
-                if (!__all_sync(0xffffffffu,
-                                mbar_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1, p.status, abort))) {
-                    abort = true;
-                    break;
-                }
-                rowok[s * BR + lane] = ok;
-                __syncwarp();
-                if (lane == 0) mbar_arrive_expect_tx(full_bar(s), BR * ROW_BYTES);
-                __syncwarp();
-                bulk_load(sbase + OFF_STAGE + s * STAGE_BYTES + lane * ROW_PITCH, src, ROW_BYTES,
-                          full_bar(s));
-                ++issued[s];
-            }
-        }
-        // Every copy started here must land before the CTA exits.
+        stage_idx(0);
+        cp_async_commit();
         cp_async_wait<0>();
-        bool drain_abort = false;
-        if (q_issued) mbar_wait(qfull_bar, (ntok - 1) & 1, p.status, drain_abort);
-        for (int s = 0; s < STAGES; ++s) {
-            drain_abort = false;
-            if (issued[s]) mbar_wait(full_bar(s), (issued[s] - 1) & 1, p.status, drain_abort);
+        named_barrier(PRODUCER_BAR, PTHREADS);
+        UnitCursor cu;
+        cu.start(p);
+        for (int uc = 0; cu.valid; ++uc, cu.advance(p)) {
+            const int s = uc % NS;
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(empty_bar(s), ((uc / NS) & 1) ^ 1, p.status, abort)))
+                break;
+            const uint32_t dst = sbase + OFF_RING + s * SLOT;
+            if (cu.u == 0) {
+                // Q of the token, and the next token's top-k row one token ahead.
+                stage_idx(cu.n + 1);
+                const __half* qt = p.q + (size_t)cu.tr.i * H * DQK;
+#pragma unroll
+                for (int m = 0; m < H * CH / PTHREADS; ++m) {
+                    const int e = ptid + m * PTHREADS, r = e / CH, ch = e % CH;
+                    cp_async_16(chunk_addr(dst, r, ch), qt + r * DQK + ch * 8, true);
+                }
+                cp_async_commit();
+                cp_async_arrive_noinc(full_bar(s));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(full_bar(s));
+                // This token's top-k row (staged one token earlier) must be in shared
+                // memory, for every producer thread, before its row units are resolved.
+                cp_async_wait<1>();
+                named_barrier(PRODUCER_BAR, PTHREADS);
+                continue;
+            }
+            const int* tk = reinterpret_cast<const int*>(smem + OFF_IDX) + (cu.n % IDX_BUFS) * kpad;
+            const int r = 8 * pw + (lane >> 2);   // this lane's row of the unit
+            const int gr = (cu.u - 1) * BR + r;
+            const __half* row = p.kv_raw + (size_t)cu.tr.t * DQK;   // valid stand-in
+            bool ok = false;
+            if (gr < cu.tr.nsel) {
+                const int j = tk[gr];
+                if (j >= 0 && j < cu.tr.nv) {
+                    row = p.kv_cmp + (size_t)j * DQK;
+                    ok = true;
+                } else if ((lane & 3) == 0) {
+                    record_status(p.status, kStatusBounds);
+                }
+            } else if (gr < cu.tr.nrows) {
+                row = p.kv_raw + (size_t)(cu.tr.s_lo + gr - cu.tr.nsel) * DQK;
+                ok = true;
+            }
+#pragma unroll
+            for (int m = 0; m < 18; ++m) {
+                const int ch = (lane & 3) + 4 * m;
+                cp_async_16(chunk_addr(dst, r, ch), row + ch * 8, ok);   // zero-filled if masked
+            }
+            cp_async_arrive_noinc(full_bar(s));
+            const uint32_t bits = __ballot_sync(0xffffffffu, ok && (lane & 3) == 0);
+            if (lane == 0) {
+                uint32_t m8 = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) m8 |= ((bits >> (4 * i)) & 1u) << i;
+                reinterpret_cast<volatile uint8_t*>(rowmask + s)[pw] = (uint8_t)m8;
+                mbar_arrive(full_bar(s));         // release: the mask byte is visible with the slot
+            }
         }
+        cp_async_wait<0>();
     } else {
-        // ------------------------------------------------------------ consumers
-        const int g = lane / 4, c = lane % 4;     // mma fragment coordinates
-        const int nt = warp & 3, kh = warp >> 2;  // S: n-tile (8 rows) and K half
-        int it = 0, ntok = 0;
-        for (int idx = blockIdx.x; idx < p.n_q; idx += gridDim.x, ++ntok) {
-            const TokenRows tr = token_rows(p, idx);
-            if (!mbar_wait(qfull_bar, ntok & 1, p.status, abort)) *abort_flag = 1;
-            uint32_t qf[18][4];                   // this warp's K half of Q as A fragments
-            {
-                const int r = (lane & 7) + ((lane >> 3) & 1) * 8, kc = (lane >> 4) * 8;
+        // ================================================================ consumers
+        float* ref_tile = reinterpret_cast<float*>(smem + OFF_REF);
+        float* red_sum = reinterpret_cast<float*>(smem + OFF_RED_SUM);
+        const int g = lane / 4, c = lane % 4;    // mma fragment coordinates
+        const int nt = warp & 3, kh = warp >> 2; // S: row tile and K half of this warp
+        const int r0 = 8 * nt + 2 * c;           // S columns of this lane: block rows r0, r0+1
+        uint32_t qf[18][4];
+        float o[8][4];
+        float m_g = -INFINITY, m_g8 = -INFINITY; // reference max, heads g and g+8 (log2 units)
+        float l_g = 0.f, l_g8 = 0.f;             // partial sums (K-half-0 warps only)
+        UnitCursor cu;
+        cu.start(p);
+        int rr = 0;                               // row units consumed
+        for (int q = 0; cu.valid; ++q, cu.advance(p)) {
+            const int s = q % NS;
+            const uint32_t slot = sbase + OFF_RING + s * SLOT;
+            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (q / NS) & 1, p.status, abort)))
+                flags[2] = 1;
+            if (cu.u == 0) {
+                const int r = (lane & 7) + ((lane >> 3) & 1) * 8, hi = lane >> 4;
 #pragma unroll
                 for (int kk = 0; kk < 18; ++kk)
-                    ldsm_x4(sbase + OFF_Q + r * ROW_PITCH + ((18 * kh + kk) * 16 + kc) * 2,
-                            qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+                    ldsm_x4(chunk_addr(slot, r, 36 * kh + 2 * kk + hi), qf[kk][0], qf[kk][1],
+                            qf[kk][2], qf[kk][3]);
+#pragma unroll
+                for (int n = 0; n < 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+                m_g = m_g8 = -INFINITY;
+                l_g = l_g8 = 0.f;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar(s));
+                continue;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(qempty_bar);
 
-            float o[8][4];
+            // ---- S partial over this warp's K half, four accumulator chains
+            float acc[4][4] = {};
+            {
+                const int rr8 = 8 * nt + (lane & 7);
 #pragma unroll
-            for (int n = 0; n < 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-            float m_g = -INFINITY, m_g8 = -INFINITY;   // running max, heads g and g+8 (log2 units)
-            float l_g = 0.f, l_g8 = 0.f;               // partial sums (K-half-0 warps only)
-
-            for (int blk = 0; blk < tr.nblk; ++blk, ++it) {
-                const int s = it % STAGES;
-                if (!mbar_wait(full_bar(s), (it / STAGES) & 1, p.status, abort)) *abort_flag = 1;
-                const uint32_t stage = sbase + OFF_STAGE + s * STAGE_BYTES;
-
-                // ---- S partial over this warp's K half, two accumulator chains
-                float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-                {
-                    const uint32_t rowaddr = stage + (8 * nt + (lane & 7)) * ROW_PITCH +
-                                             (lane >> 3) * 16 + kh * (ROW_BYTES / 2);
+                for (int k2 = 0; k2 < 9; ++k2) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(chunk_addr(slot, rr8, 36 * kh + 4 * k2 + (lane >> 3)), b0, b1, b2, b3);
+                    mma_16816(acc[(k2 & 1) * 2], qf[2 * k2], b0, b1);
+                    mma_16816(acc[(k2 & 1) * 2 + 1], qf[2 * k2 + 1], b2, b3);
+                }
+            }
+            float sv[4];
 #pragma unroll
-                    for (int k2 = 0; k2 < 9; ++k2) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4(rowaddr + k2 * 64, b0, b1, b2, b3);
-                        if (k2 & 1) {
-                            mma_16816(a1, qf[2 * k2], b0, b1);
-                            mma_16816(a1, qf[2 * k2 + 1], b2, b3);
-                        } else {
-                            mma_16816(a0, qf[2 * k2], b0, b1);
-                            mma_16816(a0, qf[2 * k2 + 1], b2, b3);
-                        }
-                    }
-                }
-                float sv[4] = {a0[0] + a1[0], a0[1] + a1[1], a0[2] + a1[2], a0[3] + a1[3]};
-                float4* sx = reinterpret_cast<float4*>(smem + OFF_SX) + nt * 32 + lane;
-                if (kh == 1) *sx = make_float4(sv[0], sv[1], sv[2], sv[3]);
-                named_barrier(CONSUMER_BAR, CWARPS * 32);
-                if (*abort_flag) break;            // every consumer warp sees the same flag here
+            for (int e = 0; e < 4; ++e) sv[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
+            float4* sx = reinterpret_cast<float4*>(smem + OFF_SX) + nt * 32 + lane;
+            if (kh == 1) *sx = make_float4(sv[0], sv[1], sv[2], sv[3]);
+            named_barrier(CONSUMER_BAR, CTHREADS);    // A: S halves meet
+            if (flags[2]) break;                       // every consumer warp sees the same flag
 
-                const int r0 = 8 * nt + 2 * c;
-                if (kh == 0) {
-                    const float4 up = *sx;
-                    const bool ok0 = rowok[s * BR + r0] != 0, ok1 = rowok[s * BR + r0 + 1] != 0;
-                    sv[0] = ok0 ? (sv[0] + up.x) * p.scale_log2 : -INFINITY;
-                    sv[1] = ok1 ? (sv[1] + up.y) * p.scale_log2 : -INFINITY;
-                    sv[2] = ok0 ? (sv[2] + up.z) * p.scale_log2 : -INFINITY;
-                    sv[3] = ok1 ? (sv[3] + up.w) * p.scale_log2 : -INFINITY;
-                    float mx_g = fmaxf(sv[0], sv[1]), mx_g8 = fmaxf(sv[2], sv[3]);
+            float ref_g = m_g, ref_g8 = m_g8;
+            if (kh == 0) {
+                const float4 up = *sx;
+                const uint32_t mask = rowmask[s];
+                const bool ok0 = (mask >> r0) & 1u, ok1 = (mask >> (r0 + 1)) & 1u;
+                sv[0] = ok0 ? (sv[0] + up.x) * p.scale_log2 : -INFINITY;
+                sv[1] = ok1 ? (sv[1] + up.y) * p.scale_log2 : -INFINITY;
+                sv[2] = ok0 ? (sv[2] + up.z) * p.scale_log2 : -INFINITY;
+                sv[3] = ok1 ? (sv[3] + up.w) * p.scale_log2 : -INFINITY;
+                float mx_g = fmaxf(sv[0], sv[1]), mx_g8 = fmaxf(sv[2], sv[3]);
 #pragma unroll
-                    for (int off = 1; off <= 2; off <<= 1) {
-                        mx_g = fmaxf(mx_g, __shfl_xor_sync(0xffffffffu, mx_g, off));
-                        mx_g8 = fmaxf(mx_g8, __shfl_xor_sync(0xffffffffu, mx_g8, off));
-                    }
-                    if (c == 0) {
-                        red_max[nt * H + g] = mx_g;
-                        red_max[nt * H + g + 8] = mx_g8;
-                    }
+                for (int off = 1; off <= 2; off <<= 1) {
+                    mx_g = fmaxf(mx_g, __shfl_xor_sync(0xffffffffu, mx_g, off));
+                    mx_g8 = fmaxf(mx_g8, __shfl_xor_sync(0xffffffffu, mx_g8, off));
                 }
-                named_barrier(CONSUMER_BAR, CWARPS * 32);
-
-                // ---- online softmax (every warp derives the same running max)
-                float bm_g = fmaxf(fmaxf(red_max[g], red_max[H + g]),
-                                   fmaxf(red_max[2 * H + g], red_max[3 * H + g]));
-                float bm_g8 = fmaxf(fmaxf(red_max[g + 8], red_max[H + g + 8]),
-                                    fmaxf(red_max[2 * H + g + 8], red_max[3 * H + g + 8]));
-                const float mn_g = fmaxf(m_g, bm_g), mn_g8 = fmaxf(m_g8, bm_g8);
-                const float ref_g = mn_g == -INFINITY ? 0.f : mn_g;
-                const float ref_g8 = mn_g8 == -INFINITY ? 0.f : mn_g8;
-                const float alpha_g = fast_exp2(m_g - ref_g), alpha_g8 = fast_exp2(m_g8 - ref_g8);
-                m_g = mn_g;
-                m_g8 = mn_g8;
-                if (kh == 0) {
-                    const float p0 = fast_exp2(sv[0] - ref_g), p1 = fast_exp2(sv[1] - ref_g);
-                    const float p2 = fast_exp2(sv[2] - ref_g8), p3 = fast_exp2(sv[3] - ref_g8);
-                    l_g = l_g * alpha_g + p0 + p1;
-                    l_g8 = l_g8 * alpha_g8 + p2 + p3;
-                    uint8_t* pb = smem + OFF_P;
-                    *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + r0 * 2) = pack_half2(p0, p1);
-                    *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + r0 * 2) = pack_half2(p2, p3);
+                // Keep the running reference unless this tile exceeds it by the headroom.
+                if (mx_g > m_g + HEADROOM) ref_g = mx_g;
+                if (mx_g8 > m_g8 + HEADROOM) ref_g8 = mx_g8;
+                const float rg = ref_g == -INFINITY ? 0.f : ref_g;
+                const float rg8 = ref_g8 == -INFINITY ? 0.f : ref_g8;
+                sv[0] = fast_exp2(sv[0] - rg);
+                sv[1] = fast_exp2(sv[1] - rg);
+                sv[2] = fast_exp2(sv[2] - rg8);
+                sv[3] = fast_exp2(sv[3] - rg8);
+                uint8_t* pb = smem + OFF_P;
+                *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + r0 * 2) = pack_half2(sv[0], sv[1]);
+                *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + r0 * 2) = pack_half2(sv[2], sv[3]);
+                if (c == 0) {
+                    ref_tile[nt * H + g] = ref_g;
+                    ref_tile[nt * H + g + 8] = ref_g8;
                 }
-                named_barrier(CONSUMER_BAR, CWARPS * 32);
+                if (ref_g != m_g || ref_g8 != m_g8) flags[rr & 1] = 1;
+            }
+            named_barrier(CONSUMER_BAR, CTHREADS);    // B: P and the tiles' references visible
+            const bool raise = flags[rr & 1] != 0;    // the same in every consumer thread
+            if (tid == 0) flags[(rr + 1) & 1] = 0;    // next row unit's flag; its writers follow A
 
-                // ---- O = alpha * O + P . V over value dims 64w .. 64w+63
+            if (raise) {                              // rare: raise the reference, rescale
+                const float M_g = fmaxf(fmaxf(ref_tile[g], ref_tile[H + g]),
+                                        fmaxf(ref_tile[2 * H + g], ref_tile[3 * H + g]));
+                const float M_g8 = fmaxf(fmaxf(ref_tile[g + 8], ref_tile[H + g + 8]),
+                                         fmaxf(ref_tile[2 * H + g + 8], ref_tile[3 * H + g + 8]));
+                const float Mg = M_g == -INFINITY ? 0.f : M_g, Mg8 = M_g8 == -INFINITY ? 0.f : M_g8;
+                const float alpha_g = fast_exp2(m_g - Mg), alpha_g8 = fast_exp2(m_g8 - Mg8);
 #pragma unroll
                 for (int n = 0; n < 8; ++n) {
                     o[n][0] *= alpha_g;
@@ -299,53 +342,79 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                     o[n][2] *= alpha_g8;
                     o[n][3] *= alpha_g8;
                 }
-                {
-                    const int ar = (lane & 7) + ((lane >> 3) & 1) * 8, hi = (lane >> 4) * 8;
+                if (kh == 0) {
+                    const float rg = ref_g == -INFINITY ? 0.f : ref_g;
+                    const float rg8 = ref_g8 == -INFINITY ? 0.f : ref_g8;
+                    const float beta_g = fast_exp2(rg - Mg), beta_g8 = fast_exp2(rg8 - Mg8);
+                    sv[0] *= beta_g;
+                    sv[1] *= beta_g;
+                    sv[2] *= beta_g8;
+                    sv[3] *= beta_g8;
+                    l_g *= alpha_g;
+                    l_g8 *= alpha_g8;
+                    uint8_t* pb = smem + OFF_P;
+                    *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + r0 * 2) = pack_half2(sv[0], sv[1]);
+                    *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + r0 * 2) =
+                        pack_half2(sv[2], sv[3]);
+                }
+                m_g = M_g;
+                m_g8 = M_g8;
+                named_barrier(CONSUMER_BAR, CTHREADS);   // rescaled P visible
+            }
+            if (kh == 0) {
+                l_g += sv[0] + sv[1];
+                l_g8 += sv[2] + sv[3];
+            }
+            ++rr;
+
+            // ---- O += P . V over value dims 64w .. 64w+63
+            {
+                const int ar = (lane & 7) + ((lane >> 3) & 1) * 8, hi = lane >> 4;
 #pragma unroll
-                    for (int ks = 0; ks < BR / 16; ++ks) {
-                        uint32_t a[4];
-                        ldsm_x4(sbase + OFF_P + ar * P_PITCH + (ks * 16 + hi) * 2, a[0], a[1], a[2], a[3]);
-                        const uint32_t vrow = stage + (ks * 16 + ar) * ROW_PITCH + (64 * warp + hi) * 2;
+                for (int ks = 0; ks < BR / 16; ++ks) {
+                    uint32_t a[4];
+                    ldsm_x4(sbase + OFF_P + ar * P_PITCH + (ks * 16 + hi * 8) * 2, a[0], a[1], a[2], a[3]);
+                    const int vr = ks * 16 + ar;
 #pragma unroll
-                        for (int np = 0; np < 4; ++np) {
-                            uint32_t b0, b1, b2, b3;
-                            ldsm_x4_trans(vrow + np * 32, b0, b1, b2, b3);
-                            mma_16816(o[2 * np], a, b0, b1);
-                            mma_16816(o[2 * np + 1], a, b2, b3);
-                        }
+                    for (int np = 0; np < 4; ++np) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4_trans(chunk_addr(slot, vr, 8 * warp + 2 * np + hi), b0, b1, b2, b3);
+                        mma_16816(o[2 * np], a, b0, b1);
+                        mma_16816(o[2 * np + 1], a, b2, b3);
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));
             }
-            if (*abort_flag) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty_bar(s));
 
-            // ---- normalise and store
-            if (kh == 0) {
+            if (cu.u == cu.tr.nblk) {
+                // ---- last block of the token: normalise and store
+                if (kh == 0) {
 #pragma unroll
-                for (int off = 1; off <= 2; off <<= 1) {
-                    l_g += __shfl_xor_sync(0xffffffffu, l_g, off);
-                    l_g8 += __shfl_xor_sync(0xffffffffu, l_g8, off);
+                    for (int off = 1; off <= 2; off <<= 1) {
+                        l_g += __shfl_xor_sync(0xffffffffu, l_g, off);
+                        l_g8 += __shfl_xor_sync(0xffffffffu, l_g8, off);
+                    }
+                    if (c == 0) {
+                        red_sum[nt * H + g] = l_g;
+                        red_sum[nt * H + g + 8] = l_g8;
+                    }
                 }
-                if (c == 0) {
-                    red_sum[nt * H + g] = l_g;
-                    red_sum[nt * H + g + 8] = l_g8;
-                }
-            }
-            named_barrier(CONSUMER_BAR, CWARPS * 32);
-            const float L_g = red_sum[g] + red_sum[H + g] + red_sum[2 * H + g] + red_sum[3 * H + g];
-            const float L_g8 = red_sum[g + 8] + red_sum[H + g + 8] + red_sum[2 * H + g + 8] +
-                               red_sum[3 * H + g + 8];
-            named_barrier(CONSUMER_BAR, CWARPS * 32);   // red_sum is rewritten by the next token
-            const float inv_g = L_g > 0.f ? 1.f / L_g : 0.f;
-            const float inv_g8 = L_g8 > 0.f ? 1.f / L_g8 : 0.f;
-            float* ot = p.out + (size_t)tr.i * H * DV;
+                named_barrier(CONSUMER_BAR, CTHREADS);
+                const float L_g = red_sum[g] + red_sum[H + g] + red_sum[2 * H + g] + red_sum[3 * H + g];
+                const float L_g8 = red_sum[g + 8] + red_sum[H + g + 8] + red_sum[2 * H + g + 8] +
+                                   red_sum[3 * H + g + 8];
+                const float inv_g = L_g > 0.f ? 1.f / L_g : 0.f;
+                const float inv_g8 = L_g8 > 0.f ? 1.f / L_g8 : 0.f;
+                float* ot = p.out + (size_t)cu.tr.i * H * DV;
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const int d = 64 * warp + 8 * n + 2 * c;
-                *reinterpret_cast<float2*>(ot + g * DV + d) = make_float2(o[n][0] * inv_g, o[n][1] * inv_g);
-                *reinterpret_cast<float2*>(ot + (g + 8) * DV + d) =
-                    make_float2(o[n][2] * inv_g8, o[n][3] * inv_g8);
+                for (int n = 0; n < 8; ++n) {
+                    const int d = 64 * warp + 8 * n + 2 * c;
+                    *reinterpret_cast<float2*>(ot + g * DV + d) =
+                        make_float2(o[n][0] * inv_g, o[n][1] * inv_g);
+                    *reinterpret_cast<float2*>(ot + (g + 8) * DV + d) =
+                        make_float2(o[n][2] * inv_g8, o[n][3] * inv_g8);
+                }
             }
         }
     }

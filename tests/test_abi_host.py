@@ -49,6 +49,7 @@ def _cfg(**kw):
     (dict(n_idx_heads=48), D.ERR_UNSUPPORTED),
     (dict(n_idx_heads=2), D.ERR_UNSUPPORTED),
     (dict(top_k=-1), D.ERR_INVALID_ARG),
+    (dict(top_k=2049), D.ERR_UNSUPPORTED),
     (dict(n_swa=0), D.ERR_INVALID_ARG),
     (dict(band=0), D.ERR_INVALID_ARG),
     (dict(max_tokens=0), D.ERR_INVALID_ARG),
