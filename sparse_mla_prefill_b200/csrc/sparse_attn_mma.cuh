@@ -18,11 +18,12 @@
 //     its 8 rows are valid. Producers never take part in the consumers' barriers.
 //   * Warps 0-7 consume, with the 16 heads as the M of mma.sync.m16n8k16. Warp w owns
 //     row tile nt = w%4 (8 rows) and K half kh = w/4 (288 dims) of S = Q . R^T, Q held
-//     in registers; the two K halves meet in shared memory. Softmax runs against a
-//     running reference max that is raised only when a block's max exceeds it by more
-//     than 2^8 (probabilities stay <= 256, fine in fp16): a 32-row block normally needs
-//     two consumer barriers; raising the reference rescales O, the sums and that
-//     block's P in every warp. O += P . V: warp w owns value dims 64w .. 64w+63.
+//     in registers; the two K halves meet in shared memory. A round takes two
+//     consecutive row units of a token (64 rows: two row tiles per warp) when it can.
+//     Softmax runs against a running reference max that is raised only when a round's
+//     max exceeds it by more than 2^8 (probabilities stay <= 256, fine in fp16): a round
+//     normally needs two consumer barriers; raising the reference rescales O, the sums
+//     and that round's P in every warp. O += P . V: warp w owns value dims 64w .. 64w+63.
 // Rows are stored unpadded with their 16-byte chunks XOR-swizzled, which keeps the
 // producers' copies and the consumers' ldmatrix reads free of bank conflicts.
 // fp32 logits, sums and output; P enters P . V as fp16; exponentials on ex2.approx.
@@ -51,12 +52,12 @@ constexpr int CONSUMER_BAR = 1;               // named barriers
 constexpr int PRODUCER_BAR = 2;
 constexpr float HEADROOM = 8.f;               // log2 units a block may exceed the reference
 constexpr int SLOT = BR * ROW;
-constexpr int P_PITCH = (BR + 8) * 2;         // fp16 probabilities, 80 B per head
+constexpr int P_PITCH = (2 * BR + 8) * 2;     // fp16 probabilities of two units, 144 B per head
 constexpr int IDX_BUFS = 2;                   // producers' top-k rows: this token, the next
 constexpr int OFF_RING = 0;
 constexpr int OFF_P = OFF_RING + NS * SLOT;
-constexpr int OFF_SX = OFF_P + H * P_PITCH;   // S partials of the upper K half
-constexpr int OFF_REF = OFF_SX + 4 * 32 * 16; // per row tile: reference used for its P
+constexpr int OFF_SX = OFF_P + H * P_PITCH;   // S partials of the upper K half, two units
+constexpr int OFF_REF = OFF_SX + 2 * 4 * 32 * 16;  // per row tile: reference used for its P
 constexpr int OFF_RED_SUM = OFF_REF + 4 * H * 4;
 constexpr int OFF_FLAGS = OFF_RED_SUM + 4 * H * 4;   // raised[2], abort, pad
 constexpr int OFF_MASK = OFF_FLAGS + 16;             // row-validity bits per slot
@@ -239,85 +240,122 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         cp_async_wait<0>();
     } else {
         // ================================================================ consumers
+        // A round consumes the Q unit of a token, or one or two consecutive row units of
+        // the same token (64 rows): two row tiles per warp between the same two barriers.
         float* ref_tile = reinterpret_cast<float*>(smem + OFF_REF);
         float* red_sum = reinterpret_cast<float*>(smem + OFF_RED_SUM);
         const int g = lane / 4, c = lane % 4;    // mma fragment coordinates
         const int nt = warp & 3, kh = warp >> 2; // S: row tile and K half of this warp
-        const int r0 = 8 * nt + 2 * c;           // S columns of this lane: block rows r0, r0+1
+        const int r0 = 8 * nt + 2 * c;           // S columns of this lane: unit rows r0, r0+1
+        const int rr8 = 8 * nt + (lane & 7);     // S: this lane's ldmatrix row
+        const int ar = (lane & 7) + ((lane >> 3) & 1) * 8, hi = lane >> 4;
         uint32_t qf[18][4];
         float o[8][4];
         float m_g = -INFINITY, m_g8 = -INFINITY; // reference max, heads g and g+8 (log2 units)
         float l_g = 0.f, l_g8 = 0.f;             // partial sums (K-half-0 warps only)
+        auto wait_full = [&](int q) {
+            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(q % NS), (q / NS) & 1, p.status, abort)))
+                flags[2] = 1;
+        };
         UnitCursor cu;
         cu.start(p);
-        int rr = 0;                               // row units consumed
-        for (int q = 0; cu.valid; ++q, cu.advance(p)) {
-            const int s = q % NS;
-            const uint32_t slot = sbase + OFF_RING + s * SLOT;
-            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (q / NS) & 1, p.status, abort)))
-                flags[2] = 1;
+        int rr = 0;                               // row rounds
+        int q = 0;                                // next unit of the ring
+        while (cu.valid) {
+            const uint32_t slot_a = sbase + OFF_RING + (q % NS) * SLOT;
             if (cu.u == 0) {
-                const int r = (lane & 7) + ((lane >> 3) & 1) * 8, hi = lane >> 4;
+                wait_full(q);
 #pragma unroll
                 for (int kk = 0; kk < 18; ++kk)
-                    ldsm_x4(chunk_addr(slot, r, 36 * kh + 2 * kk + hi), qf[kk][0], qf[kk][1],
+                    ldsm_x4(chunk_addr(slot_a, ar, 36 * kh + 2 * kk + hi), qf[kk][0], qf[kk][1],
                             qf[kk][2], qf[kk][3]);
 #pragma unroll
                 for (int n = 0; n < 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
                 m_g = m_g8 = -INFINITY;
                 l_g = l_g8 = 0.f;
                 __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));
+                if (lane == 0) mbar_arrive(empty_bar(q % NS));
+                ++q;
+                cu.advance(p);
                 continue;
             }
+            const bool two = cu.u < cu.tr.nblk;   // a second row unit of this token follows
+            const bool last = cu.u + (two ? 1 : 0) == cu.tr.nblk;
+            const uint32_t slot_b = sbase + OFF_RING + ((q + 1) % NS) * SLOT;
+            wait_full(q);
+            if (two) wait_full(q + 1);
 
-            // ---- S partial over this warp's K half, four accumulator chains
-            float acc[4][4] = {};
-            {
-                const int rr8 = 8 * nt + (lane & 7);
+            // ---- S partials over this warp's K half: unit A and unit B interleaved
+            float aa[2][4] = {}, ab[2][4] = {};
 #pragma unroll
-                for (int k2 = 0; k2 < 9; ++k2) {
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(chunk_addr(slot, rr8, 36 * kh + 4 * k2 + (lane >> 3)), b0, b1, b2, b3);
-                    mma_16816(acc[(k2 & 1) * 2], qf[2 * k2], b0, b1);
-                    mma_16816(acc[(k2 & 1) * 2 + 1], qf[2 * k2 + 1], b2, b3);
+            for (int k2 = 0; k2 < 9; ++k2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(chunk_addr(slot_a, rr8, 36 * kh + 4 * k2 + (lane >> 3)), b0, b1, b2, b3);
+                mma_16816(aa[0], qf[2 * k2], b0, b1);
+                mma_16816(aa[1], qf[2 * k2 + 1], b2, b3);
+                if (two) {
+                    ldsm_x4(chunk_addr(slot_b, rr8, 36 * kh + 4 * k2 + (lane >> 3)), b0, b1, b2, b3);
+                    mma_16816(ab[0], qf[2 * k2], b0, b1);
+                    mma_16816(ab[1], qf[2 * k2 + 1], b2, b3);
                 }
             }
-            float sv[4];
+            float sa[4], sb[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) sv[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
+            for (int e = 0; e < 4; ++e) {
+                sa[e] = aa[0][e] + aa[1][e];
+                sb[e] = ab[0][e] + ab[1][e];
+            }
             float4* sx = reinterpret_cast<float4*>(smem + OFF_SX) + nt * 32 + lane;
-            if (kh == 1) *sx = make_float4(sv[0], sv[1], sv[2], sv[3]);
+            if (kh == 1) {
+                sx[0] = make_float4(sa[0], sa[1], sa[2], sa[3]);
+                if (two) sx[128] = make_float4(sb[0], sb[1], sb[2], sb[3]);
+            }
             named_barrier(CONSUMER_BAR, CTHREADS);    // A: S halves meet
             if (flags[2]) break;                       // every consumer warp sees the same flag
 
             float ref_g = m_g, ref_g8 = m_g8;
             if (kh == 0) {
-                const float4 up = *sx;
-                const uint32_t mask = rowmask[s];
-                const bool ok0 = (mask >> r0) & 1u, ok1 = (mask >> (r0 + 1)) & 1u;
-                sv[0] = ok0 ? (sv[0] + up.x) * p.scale_log2 : -INFINITY;
-                sv[1] = ok1 ? (sv[1] + up.y) * p.scale_log2 : -INFINITY;
-                sv[2] = ok0 ? (sv[2] + up.z) * p.scale_log2 : -INFINITY;
-                sv[3] = ok1 ? (sv[3] + up.w) * p.scale_log2 : -INFINITY;
-                float mx_g = fmaxf(sv[0], sv[1]), mx_g8 = fmaxf(sv[2], sv[3]);
+                const float4 ua = sx[0];
+                const uint32_t ma = rowmask[q % NS];
+                const bool a0 = (ma >> r0) & 1u, a1 = (ma >> (r0 + 1)) & 1u;
+                sa[0] = a0 ? (sa[0] + ua.x) * p.scale_log2 : -INFINITY;
+                sa[1] = a1 ? (sa[1] + ua.y) * p.scale_log2 : -INFINITY;
+                sa[2] = a0 ? (sa[2] + ua.z) * p.scale_log2 : -INFINITY;
+                sa[3] = a1 ? (sa[3] + ua.w) * p.scale_log2 : -INFINITY;
+                if (two) {
+                    const float4 ub = sx[128];
+                    const uint32_t mb = rowmask[(q + 1) % NS];
+                    const bool b0 = (mb >> r0) & 1u, b1 = (mb >> (r0 + 1)) & 1u;
+                    sb[0] = b0 ? (sb[0] + ub.x) * p.scale_log2 : -INFINITY;
+                    sb[1] = b1 ? (sb[1] + ub.y) * p.scale_log2 : -INFINITY;
+                    sb[2] = b0 ? (sb[2] + ub.z) * p.scale_log2 : -INFINITY;
+                    sb[3] = b1 ? (sb[3] + ub.w) * p.scale_log2 : -INFINITY;
+                } else {
+                    sb[0] = sb[1] = sb[2] = sb[3] = -INFINITY;
+                }
+                float mx_g = fmaxf(fmaxf(sa[0], sa[1]), fmaxf(sb[0], sb[1]));
+                float mx_g8 = fmaxf(fmaxf(sa[2], sa[3]), fmaxf(sb[2], sb[3]));
 #pragma unroll
                 for (int off = 1; off <= 2; off <<= 1) {
                     mx_g = fmaxf(mx_g, __shfl_xor_sync(0xffffffffu, mx_g, off));
                     mx_g8 = fmaxf(mx_g8, __shfl_xor_sync(0xffffffffu, mx_g8, off));
                 }
-                // Keep the running reference unless this tile exceeds it by the headroom.
+                // Keep the running reference unless these tiles exceed it by the headroom.
                 if (mx_g > m_g + HEADROOM) ref_g = mx_g;
                 if (mx_g8 > m_g8 + HEADROOM) ref_g8 = mx_g8;
                 const float rg = ref_g == -INFINITY ? 0.f : ref_g;
                 const float rg8 = ref_g8 == -INFINITY ? 0.f : ref_g8;
-                sv[0] = fast_exp2(sv[0] - rg);
-                sv[1] = fast_exp2(sv[1] - rg);
-                sv[2] = fast_exp2(sv[2] - rg8);
-                sv[3] = fast_exp2(sv[3] - rg8);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    sa[e] = fast_exp2(sa[e] - (e < 2 ? rg : rg8));
+                    sb[e] = fast_exp2(sb[e] - (e < 2 ? rg : rg8));
+                }
                 uint8_t* pb = smem + OFF_P;
-                *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + r0 * 2) = pack_half2(sv[0], sv[1]);
-                *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + r0 * 2) = pack_half2(sv[2], sv[3]);
+                *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + r0 * 2) = pack_half2(sa[0], sa[1]);
+                *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + r0 * 2) = pack_half2(sa[2], sa[3]);
+                *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + (BR + r0) * 2) = pack_half2(sb[0], sb[1]);
+                *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + (BR + r0) * 2) =
+                    pack_half2(sb[2], sb[3]);
                 if (c == 0) {
                     ref_tile[nt * H + g] = ref_g;
                     ref_tile[nt * H + g + 8] = ref_g8;
@@ -326,7 +364,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
             }
             named_barrier(CONSUMER_BAR, CTHREADS);    // B: P and the tiles' references visible
             const bool raise = flags[rr & 1] != 0;    // the same in every consumer thread
-            if (tid == 0) flags[(rr + 1) & 1] = 0;    // next row unit's flag; its writers follow A
+            if (tid == 0) flags[(rr + 1) & 1] = 0;    // next round's flag; its writers follow A
 
             if (raise) {                              // rare: raise the reference, rescale
                 const float M_g = fmaxf(fmaxf(ref_tile[g], ref_tile[H + g]),
@@ -346,48 +384,55 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                     const float rg = ref_g == -INFINITY ? 0.f : ref_g;
                     const float rg8 = ref_g8 == -INFINITY ? 0.f : ref_g8;
                     const float beta_g = fast_exp2(rg - Mg), beta_g8 = fast_exp2(rg8 - Mg8);
-                    sv[0] *= beta_g;
-                    sv[1] *= beta_g;
-                    sv[2] *= beta_g8;
-                    sv[3] *= beta_g8;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        sa[e] *= e < 2 ? beta_g : beta_g8;
+                        sb[e] *= e < 2 ? beta_g : beta_g8;
+                    }
                     l_g *= alpha_g;
                     l_g8 *= alpha_g8;
                     uint8_t* pb = smem + OFF_P;
-                    *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + r0 * 2) = pack_half2(sv[0], sv[1]);
+                    *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + r0 * 2) = pack_half2(sa[0], sa[1]);
                     *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + r0 * 2) =
-                        pack_half2(sv[2], sv[3]);
+                        pack_half2(sa[2], sa[3]);
+                    *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + (BR + r0) * 2) =
+                        pack_half2(sb[0], sb[1]);
+                    *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + (BR + r0) * 2) =
+                        pack_half2(sb[2], sb[3]);
                 }
                 m_g = M_g;
                 m_g8 = M_g8;
                 named_barrier(CONSUMER_BAR, CTHREADS);   // rescaled P visible
             }
             if (kh == 0) {
-                l_g += sv[0] + sv[1];
-                l_g8 += sv[2] + sv[3];
+                l_g += (sa[0] + sa[1]) + (sb[0] + sb[1]);
+                l_g8 += (sa[2] + sa[3]) + (sb[2] + sb[3]);
             }
             ++rr;
 
-            // ---- O += P . V over value dims 64w .. 64w+63
-            {
-                const int ar = (lane & 7) + ((lane >> 3) & 1) * 8, hi = lane >> 4;
+            // ---- O += P . V over value dims 64w .. 64w+63, 32 or 64 rows
 #pragma unroll
-                for (int ks = 0; ks < BR / 16; ++ks) {
-                    uint32_t a[4];
-                    ldsm_x4(sbase + OFF_P + ar * P_PITCH + (ks * 16 + hi * 8) * 2, a[0], a[1], a[2], a[3]);
-                    const int vr = ks * 16 + ar;
+            for (int ks = 0; ks < 4; ++ks) {
+                if (ks >= 2 && !two) break;
+                uint32_t a[4];
+                ldsm_x4(sbase + OFF_P + ar * P_PITCH + (ks * 16 + hi * 8) * 2, a[0], a[1], a[2], a[3]);
+                const uint32_t vslot = ks < 2 ? slot_a : slot_b;
+                const int vr = (ks & 1) * 16 + ar;
 #pragma unroll
-                    for (int np = 0; np < 4; ++np) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4_trans(chunk_addr(slot, vr, 8 * warp + 2 * np + hi), b0, b1, b2, b3);
-                        mma_16816(o[2 * np], a, b0, b1);
-                        mma_16816(o[2 * np + 1], a, b2, b3);
-                    }
+                for (int np = 0; np < 4; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_trans(chunk_addr(vslot, vr, 8 * warp + 2 * np + hi), b0, b1, b2, b3);
+                    mma_16816(o[2 * np], a, b0, b1);
+                    mma_16816(o[2 * np + 1], a, b2, b3);
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(empty_bar(s));
+            if (lane == 0) {
+                mbar_arrive(empty_bar(q % NS));
+                if (two) mbar_arrive(empty_bar((q + 1) % NS));
+            }
 
-            if (cu.u == cu.tr.nblk) {
+            if (last) {
                 // ---- last block of the token: normalise and store
                 if (kh == 0) {
 #pragma unroll
@@ -416,6 +461,9 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                         make_float2(o[n][2] * inv_g8, o[n][3] * inv_g8);
                 }
             }
+            q += two ? 2 : 1;
+            cu.advance(p);
+            if (two) cu.advance(p);
         }
     }
     __syncthreads();
