@@ -238,6 +238,12 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    attn::smem_bytes(attn::MAX_TOPK));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention)");
+        cudaFuncAttributes fa;
+        const cudaError_t ea = cudaFuncGetAttributes(&fa, sparse_attn_mma_kernel);
+        if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncGetAttributes(attention)");
+        if (fa.numRegs != attn::LAUNCH_REGS)   // the warp roles' register split assumes it
+            return fail(DS4SP_ERR_UNSUPPORTED, "attention kernel built with %d registers, not %d",
+                        fa.numRegs, attn::LAUNCH_REGS);
         h->smem_set[kAttn] = true;
     }
     AttnParams p;

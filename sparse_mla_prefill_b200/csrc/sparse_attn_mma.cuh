@@ -50,6 +50,15 @@ constexpr int PTHREADS = PWARPS * 32;
 constexpr int THREADS = CTHREADS + PTHREADS;
 constexpr int CONSUMER_BAR = 1;               // named barriers
 constexpr int PRODUCER_BAR = 2;
+// Registers per thread: the kernel is built for LAUNCH_REGS (one CTA of THREADS per
+// SM); producers hand part of theirs to the consumers with setmaxnreg. The host checks
+// the built count before the first launch: a split above the launch's total would
+// leave the consumers' setmaxnreg.inc waiting.
+constexpr int LAUNCH_REGS = 168;
+constexpr int CONSUMER_REGS = 224;
+constexpr int PRODUCER_REGS = 56;
+static_assert(CWARPS * 32 * CONSUMER_REGS + PWARPS * 32 * PRODUCER_REGS <= THREADS * LAUNCH_REGS,
+              "register split must fit the launch's registers");
 constexpr float HEADROOM = 8.f;               // log2 units a block may exceed the reference
 constexpr int SLOT = BR * ROW;
 constexpr int P_PITCH = (2 * BR + 8) * 2;     // fp16 probabilities of two units, 144 B per head
@@ -162,6 +171,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
     bool abort = false;
     if (warp >= CWARPS) {
         // ================================================================ producers
+        regs_decrease<PRODUCER_REGS>();
         const int ptid = tid - CTHREADS, pw = warp - CWARPS;
         auto stage_idx = [&](int n) {             // top-k row of the CTA's token number n
             const int idx = blockIdx.x + n * gridDim.x;
@@ -240,6 +250,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         cp_async_wait<0>();
     } else {
         // ================================================================ consumers
+        regs_increase<CONSUMER_REGS>();
         // A round consumes the Q unit of a token, or one or two consecutive row units of
         // the same token (64 rows): two row tiles per warp between the same two barriers.
         float* ref_tile = reinterpret_cast<float*>(smem + OFF_REF);
