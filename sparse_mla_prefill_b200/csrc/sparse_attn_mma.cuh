@@ -8,27 +8,33 @@
 // heads". The per-token visibility (n_vis = (t+1)/4, window bounds) is computed
 // here from t; no mask is stored.
 //
-// Persistent CTAs (one per SM) walk their tokens heaviest first as a flat sequence of
-// units: per token, one unit holding its Q (16 rows), then its rows in blocks of 32.
-// Units stream through a 5-slot shared-memory ring with one mbarrier pair per slot.
+// Persistent CTAs (one per SM) take every gridDim-th token, heaviest first. A token
+// is a sequence of units: one unit holding its Q (16 rows), then its rows in blocks of
+// 32. Two consumer groups work on different tokens at once (group g takes the CTA's
+// tokens g, g+2, ...), so one group's softmax and barriers overlap the other group's
+// tensor-core work. The two groups' unit sequences are merged, one unit of each in
+// turn, into one stream through a 5-slot shared-memory ring with an mbarrier pair
+// per slot; producers and both groups walk the same merged order.
 //   * Warps 8-11 produce. They stage each token's top-k row in shared memory one
-//     token ahead, resolve and check every row, and copy it in 16-byte chunks with
-//     cp.async; cp.async.mbarrier.arrive.noinc lets the slot's barrier count the copies
-//     without the producer waiting for them. Each producer warp also publishes which of
-//     its 8 rows are valid. Producers never take part in the consumers' barriers.
-//   * Warps 0-7 consume, with the 16 heads as the M of mma.sync.m16n8k16. Warp w owns
-//     row tile nt = w%4 (8 rows) and K half kh = w/4 (288 dims) of S = Q . R^T, Q held
-//     in registers; the two K halves meet in shared memory. A round takes two
-//     consecutive row units of a token (64 rows: two row tiles per warp) when it can.
-//     Softmax runs against a running reference max that is raised only when a round's
-//     max exceeds it by more than 2^8 (probabilities stay <= 256, fine in fp16): a round
-//     normally needs two consumer barriers; raising the reference rescales O, the sums
-//     and that round's P in every warp. O += P . V: warp w owns value dims 64w .. 64w+63.
+//     token ahead per group, resolve and check every row, and copy it in 16-byte chunks
+//     with cp.async; cp.async.mbarrier.arrive.noinc lets the slot's barrier count the
+//     copies without the producer waiting for them. Each producer warp also publishes
+//     which of its 8 rows are valid. Producers never take part in the consumers'
+//     barriers, and setmaxnreg moves most of their registers to the consumers.
+//   * Warps 4g .. 4g+3 form consumer group g, with the 16 heads as the M of
+//     mma.sync.m16n8k16. Group warp w (kh = w/2, rh = w%2) computes the partial
+//     S = Q . R^T of rows 16rh .. 16rh+15 over K half kh (288 dims), Q's half held in
+//     registers; the halves meet in shared memory and warp w completes and
+//     normalises the 8-row tile 2rh+kh. Softmax runs against a running reference max
+//     that is raised only when a tile's max exceeds it by more than 2^8 (probabilities
+//     stay <= 256, fine in fp16): a unit normally needs two group barriers; raising the
+//     reference rescales O, the sums and that unit's P. O += P . V: group warp w owns
+//     value dims 128w .. 128w+127.
 // Rows are stored unpadded with their 16-byte chunks XOR-swizzled, which keeps the
 // producers' copies and the consumers' ldmatrix reads free of bank conflicts.
 // fp32 logits, sums and output; P enters P . V as fp16; exponentials on ex2.approx.
-// Every wait is bounded; a consumer that gives up sets a flag that all consumer warps
-// read at their next barrier, so none is left waiting.
+// Every wait is bounded; a consumer that gives up sets its group's flag, which the
+// group's warps read after their next barrier, so none is left waiting.
 #pragma once
 
 #include "device_common.cuh"
@@ -43,13 +49,16 @@ constexpr int ROW = DQK * 2;                  // 1152 bytes per latent row
 constexpr int CH = ROW / 16;                  // 72 sixteen-byte chunks per row
 constexpr int BR = 32;                        // rows per unit
 constexpr int NS = 5;                         // ring slots
-constexpr int CWARPS = 8;                     // consumer warps
+constexpr int GROUPS = 2;                     // consumer groups, each on its own token
+constexpr int GWARPS = 4;                     // warps per consumer group
+constexpr int CWARPS = GROUPS * GWARPS;       // consumer warps
 constexpr int PWARPS = 4;                     // producer warps
+constexpr int GTHREADS = GWARPS * 32;
 constexpr int CTHREADS = CWARPS * 32;
 constexpr int PTHREADS = PWARPS * 32;
 constexpr int THREADS = CTHREADS + PTHREADS;
-constexpr int CONSUMER_BAR = 1;               // named barriers
-constexpr int PRODUCER_BAR = 2;
+constexpr int PRODUCER_BAR = 1;               // named barriers; group g uses GROUP_BAR + g
+constexpr int GROUP_BAR = 2;
 // Registers per thread: the kernel is built for LAUNCH_REGS (one CTA of THREADS per
 // SM); producers hand part of theirs to the consumers with setmaxnreg. The host checks
 // the built count before the first launch: a split above the launch's total would
@@ -59,25 +68,31 @@ constexpr int CONSUMER_REGS = 224;
 constexpr int PRODUCER_REGS = 56;
 static_assert(CWARPS * 32 * CONSUMER_REGS + PWARPS * 32 * PRODUCER_REGS <= THREADS * LAUNCH_REGS,
               "register split must fit the launch's registers");
-constexpr float HEADROOM = 8.f;               // log2 units a block may exceed the reference
+constexpr float HEADROOM = 8.f;               // log2 units a tile may exceed the reference
 constexpr int SLOT = BR * ROW;
-constexpr int P_PITCH = (2 * BR + 8) * 2;     // fp16 probabilities of two units, 144 B per head
-constexpr int IDX_BUFS = 2;                   // producers' top-k rows: this token, the next
+constexpr int P_PITCH = (BR + 8) * 2;         // fp16 probabilities of one unit, 80 B per head
+constexpr int IDX_BUFS = 2;                   // per group: top-k rows of this token, the next
+// Per-group areas.
+constexpr int P_BYTES = H * P_PITCH;
+constexpr int X_BYTES = 4 * 32 * 16;          // S partials passed between the K halves
+constexpr int REF_BYTES = 4 * H * 4;          // per S tile: reference used for its P
+constexpr int RED_BYTES = GWARPS * H * 4;     // per warp: softmax sums of a finished token
+constexpr int FLAG_BYTES = 16;                // raised[2], abort, pad
+constexpr int G_BYTES = P_BYTES + X_BYTES + REF_BYTES + RED_BYTES + FLAG_BYTES;
+constexpr int G_P = 0, G_X = P_BYTES, G_REF = G_X + X_BYTES, G_RED = G_REF + REF_BYTES,
+              G_FLAGS = G_RED + RED_BYTES;
 constexpr int OFF_RING = 0;
-constexpr int OFF_P = OFF_RING + NS * SLOT;
-constexpr int OFF_SX = OFF_P + H * P_PITCH;   // S partials of the upper K half, two units
-constexpr int OFF_REF = OFF_SX + 2 * 4 * 32 * 16;  // per row tile: reference used for its P
-constexpr int OFF_RED_SUM = OFF_REF + 4 * H * 4;
-constexpr int OFF_FLAGS = OFF_RED_SUM + 4 * H * 4;   // raised[2], abort, pad
-constexpr int OFF_MASK = OFF_FLAGS + 16;             // row-validity bits per slot
-constexpr int OFF_BAR = OFF_MASK + 32;               // full[NS], empty[NS]
+constexpr int OFF_GROUP = OFF_RING + NS * SLOT;
+constexpr int OFF_MASK = OFF_GROUP + GROUPS * G_BYTES;   // row-validity bits per slot
+constexpr int OFF_BAR = OFF_MASK + 32;                   // full[NS], empty[NS]
 constexpr int OFF_IDX = OFF_BAR + 2 * NS * 8;
 constexpr int MAX_TOPK = 2048;
 __host__ __device__ constexpr int smem_bytes(int k) {
-    return OFF_IDX + IDX_BUFS * ((k + 3) / 4 * 4) * 4;
+    return OFF_IDX + GROUPS * IDX_BUFS * ((k + 3) / 4 * 4) * 4;
 }
-static_assert(DV == CWARPS * 64, "each consumer warp owns 64 value dims");
+static_assert(DV == GWARPS * 128, "each group warp owns 128 value dims");
 static_assert(CH % 8 == 0 && BR * CH == PTHREADS * 18, "producer chunk split");
+static_assert(G_BYTES % 16 == 0 && OFF_GROUP % 16 == 0, "16-byte aligned group areas");
 static_assert(smem_bytes(MAX_TOPK) <= 227 * 1024, "shared memory budget");
 
 // 16-byte chunk swizzle: eight consecutive rows put one chunk in eight different bank
@@ -117,27 +132,50 @@ __device__ __forceinline__ TokenRows token_rows(const AttnParams& p, int idx) {
     return r;
 }
 
-// Position in a CTA's flat unit sequence: token number n (the CTA's n-th token), unit u
-// (0 = Q, 1.. = row blocks).
-struct UnitCursor {
-    int n, idx, u;
+// One consumer group's position: its m-th token (the CTA's token number g + 2m),
+// unit u of it (0 = Q, 1.. = row blocks).
+struct GroupCursor {
+    int m, idx, u;
     TokenRows tr;
     bool valid;
-    __device__ __forceinline__ void start(const AttnParams& p) {
-        n = 0;
-        idx = blockIdx.x;
+    __device__ __forceinline__ void start(const AttnParams& p, int g) {
+        m = 0;
+        idx = blockIdx.x + g * gridDim.x;
         u = 0;
         valid = idx < p.n_q;
         if (valid) tr = token_rows(p, idx);
     }
     __device__ __forceinline__ void advance(const AttnParams& p) {
-        if (!valid) return;
         if (++u > tr.nblk) {
             u = 0;
-            ++n;
-            idx += gridDim.x;
+            ++m;
+            idx += attn::GROUPS * gridDim.x;
             valid = idx < p.n_q;
             if (valid) tr = token_rows(p, idx);
+        }
+    }
+};
+
+// The ring's unit order: one unit of each group in turn while both have units left,
+// then the remaining group's units. `turn` is the group of the current unit. (Two named
+// cursors rather than an array indexed by `turn`, which would live in local memory.)
+struct MergedCursor {
+    GroupCursor c0, c1;
+    int turn;
+    __device__ __forceinline__ void start(const AttnParams& p) {
+        c0.start(p, 0);
+        c1.start(p, 1);
+        turn = c0.valid ? 0 : 1;
+    }
+    __device__ __forceinline__ const GroupCursor& group(int g) const { return g ? c1 : c0; }
+    __device__ __forceinline__ bool valid() const { return turn ? c1.valid : c0.valid; }
+    __device__ __forceinline__ void advance(const AttnParams& p) {
+        if (turn) {
+            c1.advance(p);
+            if (c0.valid) turn = 0;
+        } else {
+            c0.advance(p);
+            if (c1.valid) turn = 1;
         }
     }
 };
@@ -152,7 +190,6 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int kpad = (p.k + 3) / 4 * 4;
-    volatile int* flags = reinterpret_cast<volatile int*>(smem + OFF_FLAGS);  // raised[2], abort
     volatile uint32_t* rowmask = reinterpret_cast<volatile uint32_t*>(smem + OFF_MASK);
     const uint32_t bar0 = sbase + OFF_BAR;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -161,9 +198,12 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(full_bar(s), PTHREADS + PWARPS);   // noinc copy arrivals + mask writers
-            mbar_init(empty_bar(s), CWARPS);
+            mbar_init(empty_bar(s), GWARPS);             // the owning group's warps
         }
-        flags[0] = flags[1] = flags[2] = 0;
+        for (int g = 0; g < GROUPS; ++g) {
+            volatile int* f = reinterpret_cast<volatile int*>(smem + OFF_GROUP + g * G_BYTES + G_FLAGS);
+            f[0] = f[1] = f[2] = 0;
+        }
         fence_mbar_init();
     }
     __syncthreads();
@@ -173,32 +213,35 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         // ================================================================ producers
         regs_decrease<PRODUCER_REGS>();
         const int ptid = tid - CTHREADS, pw = warp - CWARPS;
-        auto stage_idx = [&](int n) {             // top-k row of the CTA's token number n
-            const int idx = blockIdx.x + n * gridDim.x;
+        auto idx_buf = [&](int g, int m) { return OFF_IDX + (g * IDX_BUFS + (m & 1)) * kpad * 4; };
+        auto stage_idx = [&](int g, int m) {      // top-k row of group g's m-th token
+            const int idx = blockIdx.x + (g + GROUPS * m) * gridDim.x;
             if (idx >= p.n_q) return;
             const TokenRows nx = token_rows(p, idx);
             const int32_t* src = p.topk + (size_t)nx.i * p.k;
-            const uint32_t dst = sbase + OFF_IDX + (n % IDX_BUFS) * kpad * 4;
+            const uint32_t dst = sbase + idx_buf(g, m);
             for (int e = ptid; e < nx.nsel; e += PTHREADS)
                 asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst + 4 * e),
                              "l"(src + e)
                              : "memory");
         };
-        stage_idx(0);
+        stage_idx(0, 0);
+        stage_idx(1, 0);
         cp_async_commit();
         cp_async_wait<0>();
         named_barrier(PRODUCER_BAR, PTHREADS);
-        UnitCursor cu;
-        cu.start(p);
-        for (int uc = 0; cu.valid; ++uc, cu.advance(p)) {
+        MergedCursor mc;
+        mc.start(p);
+        for (int uc = 0; mc.valid(); ++uc, mc.advance(p)) {
             const int s = uc % NS;
             if (!__all_sync(0xffffffffu,
                             mbar_wait(empty_bar(s), ((uc / NS) & 1) ^ 1, p.status, abort)))
                 break;
             const uint32_t dst = sbase + OFF_RING + s * SLOT;
+            const GroupCursor cu = mc.group(mc.turn);
             if (cu.u == 0) {
-                // Q of the token, and the next token's top-k row one token ahead.
-                stage_idx(cu.n + 1);
+                // Q of the token, and the group's next top-k row one token ahead.
+                stage_idx(mc.turn, cu.m + 1);
                 const __half* qt = p.q + (size_t)cu.tr.i * H * DQK;
 #pragma unroll
                 for (int m = 0; m < H * CH / PTHREADS; ++m) {
@@ -209,13 +252,14 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                 cp_async_arrive_noinc(full_bar(s));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(full_bar(s));
-                // This token's top-k row (staged one token earlier) must be in shared
-                // memory, for every producer thread, before its row units are resolved.
+                // This token's top-k row (staged at the group's previous Q unit, an earlier
+                // commit group) must be in shared memory, for every producer thread,
+                // before its row units are resolved.
                 cp_async_wait<1>();
                 named_barrier(PRODUCER_BAR, PTHREADS);
                 continue;
             }
-            const int* tk = reinterpret_cast<const int*>(smem + OFF_IDX) + (cu.n % IDX_BUFS) * kpad;
+            const int* tk = reinterpret_cast<const int*>(smem + idx_buf(mc.turn, cu.m));
             const int r = 8 * pw + (lane >> 2);   // this lane's row of the unit
             const int gr = (cu.u - 1) * BR + r;
             const __half* row = p.kv_raw + (size_t)cu.tr.t * DQK;   // valid stand-in
@@ -251,230 +295,191 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
     } else {
         // ================================================================ consumers
         regs_increase<CONSUMER_REGS>();
-        // A round consumes the Q unit of a token, or one or two consecutive row units of
-        // the same token (64 rows): two row tiles per warp between the same two barriers.
-        float* ref_tile = reinterpret_cast<float*>(smem + OFF_REF);
-        float* red_sum = reinterpret_cast<float*>(smem + OFF_RED_SUM);
+        const int grp = warp / GWARPS, gw = warp % GWARPS;
+        const int gbar = GROUP_BAR + grp;
+        uint8_t* garea = smem + OFF_GROUP + grp * G_BYTES;
+        const uint32_t pbase = sbase + OFF_GROUP + grp * G_BYTES + G_P;
+        float4* xbuf = reinterpret_cast<float4*>(garea + G_X);
+        float* ref_tile = reinterpret_cast<float*>(garea + G_REF);
+        float* red_sum = reinterpret_cast<float*>(garea + G_RED);
+        volatile int* flags = reinterpret_cast<volatile int*>(garea + G_FLAGS);  // raised[2], abort
         const int g = lane / 4, c = lane % 4;    // mma fragment coordinates
-        const int nt = warp & 3, kh = warp >> 2; // S: row tile and K half of this warp
-        const int r0 = 8 * nt + 2 * c;           // S columns of this lane: unit rows r0, r0+1
-        const int rr8 = 8 * nt + (lane & 7);     // S: this lane's ldmatrix row
+        const int kh = gw >> 1, rh = gw & 1;     // S: K half, row half (rows 16rh .. 16rh+15)
+        const int own = 2 * rh + kh;             // the 8-row S tile this warp completes
+        const int give = 2 * rh + (kh ^ 1);      // the partner's tile
+        const int r0 = 8 * own + 2 * c;          // S columns of this lane: unit rows r0, r0+1
+        const int rlo = 16 * rh + (lane & 7);    // S: this lane's ldmatrix row, first tile
         const int ar = (lane & 7) + ((lane >> 3) & 1) * 8, hi = lane >> 4;
         uint32_t qf[18][4];
-        float o[8][4];
+        float o[16][4];
         float m_g = -INFINITY, m_g8 = -INFINITY; // reference max, heads g and g+8 (log2 units)
-        float l_g = 0.f, l_g8 = 0.f;             // partial sums (K-half-0 warps only)
+        float l_g = 0.f, l_g8 = 0.f;             // this warp's share of the softmax sums
         auto wait_full = [&](int q) {
             if (!__all_sync(0xffffffffu, mbar_wait(full_bar(q % NS), (q / NS) & 1, p.status, abort)))
                 flags[2] = 1;
         };
-        UnitCursor cu;
-        cu.start(p);
-        int rr = 0;                               // row rounds
-        int q = 0;                                // next unit of the ring
-        while (cu.valid) {
-            const uint32_t slot_a = sbase + OFF_RING + (q % NS) * SLOT;
+        MergedCursor mc;
+        mc.start(p);
+        int rr = 0;                               // this group's row units
+        for (int q = 0; mc.valid(); ++q, mc.advance(p)) {
+            if (mc.turn != grp) continue;         // the other group's unit
+            const GroupCursor cu = mc.group(grp);
+            const uint32_t slot = sbase + OFF_RING + (q % NS) * SLOT;
+            wait_full(q);
             if (cu.u == 0) {
-                wait_full(q);
 #pragma unroll
                 for (int kk = 0; kk < 18; ++kk)
-                    ldsm_x4(chunk_addr(slot_a, ar, 36 * kh + 2 * kk + hi), qf[kk][0], qf[kk][1],
+                    ldsm_x4(chunk_addr(slot, ar, 36 * kh + 2 * kk + hi), qf[kk][0], qf[kk][1],
                             qf[kk][2], qf[kk][3]);
 #pragma unroll
-                for (int n = 0; n < 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+                for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
                 m_g = m_g8 = -INFINITY;
                 l_g = l_g8 = 0.f;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty_bar(q % NS));
-                ++q;
-                cu.advance(p);
                 continue;
             }
-            const bool two = cu.u < cu.tr.nblk;   // a second row unit of this token follows
-            const bool last = cu.u + (two ? 1 : 0) == cu.tr.nblk;
-            const uint32_t slot_b = sbase + OFF_RING + ((q + 1) % NS) * SLOT;
-            wait_full(q);
-            if (two) wait_full(q + 1);
 
-            // ---- S partials over this warp's K half: unit A and unit B interleaved
+            // ---- S partials over this warp's K half, both 8-row tiles of its row half
             float aa[2][4] = {}, ab[2][4] = {};
 #pragma unroll
             for (int k2 = 0; k2 < 9; ++k2) {
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4(chunk_addr(slot_a, rr8, 36 * kh + 4 * k2 + (lane >> 3)), b0, b1, b2, b3);
+                ldsm_x4(chunk_addr(slot, rlo, 36 * kh + 4 * k2 + (lane >> 3)), b0, b1, b2, b3);
                 mma_16816(aa[0], qf[2 * k2], b0, b1);
                 mma_16816(aa[1], qf[2 * k2 + 1], b2, b3);
-                if (two) {
-                    ldsm_x4(chunk_addr(slot_b, rr8, 36 * kh + 4 * k2 + (lane >> 3)), b0, b1, b2, b3);
-                    mma_16816(ab[0], qf[2 * k2], b0, b1);
-                    mma_16816(ab[1], qf[2 * k2 + 1], b2, b3);
-                }
+                ldsm_x4(chunk_addr(slot, rlo + 8, 36 * kh + 4 * k2 + (lane >> 3)), b0, b1, b2, b3);
+                mma_16816(ab[0], qf[2 * k2], b0, b1);
+                mma_16816(ab[1], qf[2 * k2 + 1], b2, b3);
             }
-            float sa[4], sb[4];
+            float s4[4], sg[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                sa[e] = aa[0][e] + aa[1][e];
-                sb[e] = ab[0][e] + ab[1][e];
+                const float lo = aa[0][e] + aa[1][e], up = ab[0][e] + ab[1][e];
+                s4[e] = kh == 0 ? lo : up;        // partial of the own tile
+                sg[e] = kh == 0 ? up : lo;        // partial of the partner's tile
             }
-            float4* sx = reinterpret_cast<float4*>(smem + OFF_SX) + nt * 32 + lane;
-            if (kh == 1) {
-                sx[0] = make_float4(sa[0], sa[1], sa[2], sa[3]);
-                if (two) sx[128] = make_float4(sb[0], sb[1], sb[2], sb[3]);
-            }
-            named_barrier(CONSUMER_BAR, CTHREADS);    // A: S halves meet
-            if (flags[2]) break;                       // every consumer warp sees the same flag
+            xbuf[give * 32 + lane] = make_float4(sg[0], sg[1], sg[2], sg[3]);
+            named_barrier(gbar, GTHREADS);        // A: S halves meet
+            if (flags[2]) break;                  // every warp of the group sees the same flag
 
-            float ref_g = m_g, ref_g8 = m_g8;
-            if (kh == 0) {
-                const float4 ua = sx[0];
-                const uint32_t ma = rowmask[q % NS];
-                const bool a0 = (ma >> r0) & 1u, a1 = (ma >> (r0 + 1)) & 1u;
-                sa[0] = a0 ? (sa[0] + ua.x) * p.scale_log2 : -INFINITY;
-                sa[1] = a1 ? (sa[1] + ua.y) * p.scale_log2 : -INFINITY;
-                sa[2] = a0 ? (sa[2] + ua.z) * p.scale_log2 : -INFINITY;
-                sa[3] = a1 ? (sa[3] + ua.w) * p.scale_log2 : -INFINITY;
-                if (two) {
-                    const float4 ub = sx[128];
-                    const uint32_t mb = rowmask[(q + 1) % NS];
-                    const bool b0 = (mb >> r0) & 1u, b1 = (mb >> (r0 + 1)) & 1u;
-                    sb[0] = b0 ? (sb[0] + ub.x) * p.scale_log2 : -INFINITY;
-                    sb[1] = b1 ? (sb[1] + ub.y) * p.scale_log2 : -INFINITY;
-                    sb[2] = b0 ? (sb[2] + ub.z) * p.scale_log2 : -INFINITY;
-                    sb[3] = b1 ? (sb[3] + ub.w) * p.scale_log2 : -INFINITY;
-                } else {
-                    sb[0] = sb[1] = sb[2] = sb[3] = -INFINITY;
-                }
-                float mx_g = fmaxf(fmaxf(sa[0], sa[1]), fmaxf(sb[0], sb[1]));
-                float mx_g8 = fmaxf(fmaxf(sa[2], sa[3]), fmaxf(sb[2], sb[3]));
+            {
+                const float4 u = xbuf[own * 32 + lane];
+                const uint32_t mk = rowmask[q % NS];
+                const bool v0 = (mk >> r0) & 1u, v1 = (mk >> (r0 + 1)) & 1u;
+                s4[0] = v0 ? (s4[0] + u.x) * p.scale_log2 : -INFINITY;
+                s4[1] = v1 ? (s4[1] + u.y) * p.scale_log2 : -INFINITY;
+                s4[2] = v0 ? (s4[2] + u.z) * p.scale_log2 : -INFINITY;
+                s4[3] = v1 ? (s4[3] + u.w) * p.scale_log2 : -INFINITY;
+            }
+            float mx_g = fmaxf(s4[0], s4[1]), mx_g8 = fmaxf(s4[2], s4[3]);
 #pragma unroll
-                for (int off = 1; off <= 2; off <<= 1) {
-                    mx_g = fmaxf(mx_g, __shfl_xor_sync(0xffffffffu, mx_g, off));
-                    mx_g8 = fmaxf(mx_g8, __shfl_xor_sync(0xffffffffu, mx_g8, off));
-                }
-                // Keep the running reference unless these tiles exceed it by the headroom.
-                if (mx_g > m_g + HEADROOM) ref_g = mx_g;
-                if (mx_g8 > m_g8 + HEADROOM) ref_g8 = mx_g8;
+            for (int off = 1; off <= 2; off <<= 1) {
+                mx_g = fmaxf(mx_g, __shfl_xor_sync(0xffffffffu, mx_g, off));
+                mx_g8 = fmaxf(mx_g8, __shfl_xor_sync(0xffffffffu, mx_g8, off));
+            }
+            // Keep the running reference unless this tile exceeds it by the headroom.
+            float ref_g = m_g, ref_g8 = m_g8;
+            if (mx_g > m_g + HEADROOM) ref_g = mx_g;
+            if (mx_g8 > m_g8 + HEADROOM) ref_g8 = mx_g8;
+            {
                 const float rg = ref_g == -INFINITY ? 0.f : ref_g;
                 const float rg8 = ref_g8 == -INFINITY ? 0.f : ref_g8;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    sa[e] = fast_exp2(sa[e] - (e < 2 ? rg : rg8));
-                    sb[e] = fast_exp2(sb[e] - (e < 2 ? rg : rg8));
-                }
-                uint8_t* pb = smem + OFF_P;
-                *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + r0 * 2) = pack_half2(sa[0], sa[1]);
-                *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + r0 * 2) = pack_half2(sa[2], sa[3]);
-                *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + (BR + r0) * 2) = pack_half2(sb[0], sb[1]);
-                *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + (BR + r0) * 2) =
-                    pack_half2(sb[2], sb[3]);
-                if (c == 0) {
-                    ref_tile[nt * H + g] = ref_g;
-                    ref_tile[nt * H + g + 8] = ref_g8;
-                }
-                if (ref_g != m_g || ref_g8 != m_g8) flags[rr & 1] = 1;
+                for (int e = 0; e < 4; ++e) s4[e] = fast_exp2(s4[e] - (e < 2 ? rg : rg8));
             }
-            named_barrier(CONSUMER_BAR, CTHREADS);    // B: P and the tiles' references visible
-            const bool raise = flags[rr & 1] != 0;    // the same in every consumer thread
-            if (tid == 0) flags[(rr + 1) & 1] = 0;    // next round's flag; its writers follow A
+            uint8_t* pb = garea + G_P + r0 * 2;
+            *reinterpret_cast<uint32_t*>(pb + g * P_PITCH) = pack_half2(s4[0], s4[1]);
+            *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH) = pack_half2(s4[2], s4[3]);
+            if (c == 0) {
+                ref_tile[own * H + g] = ref_g;
+                ref_tile[own * H + g + 8] = ref_g8;
+            }
+            if (ref_g != m_g || ref_g8 != m_g8) flags[rr & 1] = 1;
+            named_barrier(gbar, GTHREADS);        // B: P and the tiles' references visible
+            const bool raise = flags[rr & 1] != 0;   // the same in every warp of the group
+            if (gw == 0 && lane == 0) flags[(rr + 1) & 1] = 0;   // next unit's; writers follow A
 
-            if (raise) {                              // rare: raise the reference, rescale
-                const float M_g = fmaxf(fmaxf(ref_tile[g], ref_tile[H + g]),
-                                        fmaxf(ref_tile[2 * H + g], ref_tile[3 * H + g]));
-                const float M_g8 = fmaxf(fmaxf(ref_tile[g + 8], ref_tile[H + g + 8]),
-                                         fmaxf(ref_tile[2 * H + g + 8], ref_tile[3 * H + g + 8]));
+            if (raise) {                          // rare: raise the reference, rescale
+                float M_g = -INFINITY, M_g8 = -INFINITY;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    M_g = fmaxf(M_g, ref_tile[t * H + g]);
+                    M_g8 = fmaxf(M_g8, ref_tile[t * H + g + 8]);
+                }
                 const float Mg = M_g == -INFINITY ? 0.f : M_g, Mg8 = M_g8 == -INFINITY ? 0.f : M_g8;
                 const float alpha_g = fast_exp2(m_g - Mg), alpha_g8 = fast_exp2(m_g8 - Mg8);
 #pragma unroll
-                for (int n = 0; n < 8; ++n) {
+                for (int n = 0; n < 16; ++n) {
                     o[n][0] *= alpha_g;
                     o[n][1] *= alpha_g;
                     o[n][2] *= alpha_g8;
                     o[n][3] *= alpha_g8;
                 }
-                if (kh == 0) {
-                    const float rg = ref_g == -INFINITY ? 0.f : ref_g;
-                    const float rg8 = ref_g8 == -INFINITY ? 0.f : ref_g8;
-                    const float beta_g = fast_exp2(rg - Mg), beta_g8 = fast_exp2(rg8 - Mg8);
+                l_g *= alpha_g;
+                l_g8 *= alpha_g8;
+                const float rg = ref_g == -INFINITY ? 0.f : ref_g;
+                const float rg8 = ref_g8 == -INFINITY ? 0.f : ref_g8;
+                const float beta_g = fast_exp2(rg - Mg), beta_g8 = fast_exp2(rg8 - Mg8);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        sa[e] *= e < 2 ? beta_g : beta_g8;
-                        sb[e] *= e < 2 ? beta_g : beta_g8;
-                    }
-                    l_g *= alpha_g;
-                    l_g8 *= alpha_g8;
-                    uint8_t* pb = smem + OFF_P;
-                    *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + r0 * 2) = pack_half2(sa[0], sa[1]);
-                    *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + r0 * 2) =
-                        pack_half2(sa[2], sa[3]);
-                    *reinterpret_cast<uint32_t*>(pb + g * P_PITCH + (BR + r0) * 2) =
-                        pack_half2(sb[0], sb[1]);
-                    *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH + (BR + r0) * 2) =
-                        pack_half2(sb[2], sb[3]);
-                }
+                for (int e = 0; e < 4; ++e) s4[e] *= e < 2 ? beta_g : beta_g8;
+                *reinterpret_cast<uint32_t*>(pb + g * P_PITCH) = pack_half2(s4[0], s4[1]);
+                *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH) = pack_half2(s4[2], s4[3]);
                 m_g = M_g;
                 m_g8 = M_g8;
-                named_barrier(CONSUMER_BAR, CTHREADS);   // rescaled P visible
+                named_barrier(gbar, GTHREADS);    // rescaled P visible
             }
-            if (kh == 0) {
-                l_g += (sa[0] + sa[1]) + (sb[0] + sb[1]);
-                l_g8 += (sa[2] + sa[3]) + (sb[2] + sb[3]);
-            }
+            l_g += s4[0] + s4[1];
+            l_g8 += s4[2] + s4[3];
             ++rr;
 
-            // ---- O += P . V over value dims 64w .. 64w+63, 32 or 64 rows
+            // ---- O += P . V over value dims 128gw .. 128gw+127, 32 rows
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                if (ks >= 2 && !two) break;
+            for (int ks = 0; ks < 2; ++ks) {
                 uint32_t a[4];
-                ldsm_x4(sbase + OFF_P + ar * P_PITCH + (ks * 16 + hi * 8) * 2, a[0], a[1], a[2], a[3]);
-                const uint32_t vslot = ks < 2 ? slot_a : slot_b;
-                const int vr = (ks & 1) * 16 + ar;
+                ldsm_x4(pbase + ar * P_PITCH + (ks * 16 + hi * 8) * 2, a[0], a[1], a[2], a[3]);
+                const int vr = ks * 16 + ar;
 #pragma unroll
-                for (int np = 0; np < 4; ++np) {
+                for (int np = 0; np < 8; ++np) {
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4_trans(chunk_addr(vslot, vr, 8 * warp + 2 * np + hi), b0, b1, b2, b3);
+                    ldsm_x4_trans(chunk_addr(slot, vr, 16 * gw + 2 * np + hi), b0, b1, b2, b3);
                     mma_16816(o[2 * np], a, b0, b1);
                     mma_16816(o[2 * np + 1], a, b2, b3);
                 }
             }
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(empty_bar(q % NS));
-                if (two) mbar_arrive(empty_bar((q + 1) % NS));
-            }
+            if (lane == 0) mbar_arrive(empty_bar(q % NS));
 
-            if (last) {
-                // ---- last block of the token: normalise and store
-                if (kh == 0) {
+            if (cu.u == cu.tr.nblk) {
+                // ---- last unit of the token: normalise and store
 #pragma unroll
-                    for (int off = 1; off <= 2; off <<= 1) {
-                        l_g += __shfl_xor_sync(0xffffffffu, l_g, off);
-                        l_g8 += __shfl_xor_sync(0xffffffffu, l_g8, off);
-                    }
-                    if (c == 0) {
-                        red_sum[nt * H + g] = l_g;
-                        red_sum[nt * H + g + 8] = l_g8;
-                    }
+                for (int off = 1; off <= 2; off <<= 1) {
+                    l_g += __shfl_xor_sync(0xffffffffu, l_g, off);
+                    l_g8 += __shfl_xor_sync(0xffffffffu, l_g8, off);
                 }
-                named_barrier(CONSUMER_BAR, CTHREADS);
-                const float L_g = red_sum[g] + red_sum[H + g] + red_sum[2 * H + g] + red_sum[3 * H + g];
-                const float L_g8 = red_sum[g + 8] + red_sum[H + g + 8] + red_sum[2 * H + g + 8] +
-                                   red_sum[3 * H + g + 8];
+                if (c == 0) {
+                    red_sum[gw * H + g] = l_g;
+                    red_sum[gw * H + g + 8] = l_g8;
+                }
+                named_barrier(gbar, GTHREADS);
+                float L_g = 0.f, L_g8 = 0.f;
+#pragma unroll
+                for (int w = 0; w < GWARPS; ++w) {
+                    L_g += red_sum[w * H + g];
+                    L_g8 += red_sum[w * H + g + 8];
+                }
                 const float inv_g = L_g > 0.f ? 1.f / L_g : 0.f;
                 const float inv_g8 = L_g8 > 0.f ? 1.f / L_g8 : 0.f;
                 float* ot = p.out + (size_t)cu.tr.i * H * DV;
 #pragma unroll
-                for (int n = 0; n < 8; ++n) {
-                    const int d = 64 * warp + 8 * n + 2 * c;
+                for (int n = 0; n < 16; ++n) {
+                    const int d = 128 * gw + 8 * n + 2 * c;
                     *reinterpret_cast<float2*>(ot + g * DV + d) =
                         make_float2(o[n][0] * inv_g, o[n][1] * inv_g);
                     *reinterpret_cast<float2*>(ot + (g + 8) * DV + d) =
                         make_float2(o[n][2] * inv_g8, o[n][3] * inv_g8);
                 }
             }
-            q += two ? 2 : 1;
-            cu.advance(p);
-            if (two) cu.advance(p);
         }
     }
     __syncthreads();
