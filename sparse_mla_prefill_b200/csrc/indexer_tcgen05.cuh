@@ -14,7 +14,8 @@
 // Work unit: one block of 256/H_i tokens and a range of its 128-row j-tiles. CTAs are
 // persistent (one per SM) and take units in snake order over a heaviest-first list.
 // Warp roles (352 threads): warp 10 loads q_idx blocks into two B buffers, up to two
-// units ahead; warp 0 streams k_idx tiles as 16 KB K sub-tiles into a 4-deep ring;
+// units ahead; warp 0 streams whole k_idx tiles (one 64-dim TMA box per K sub-tile)
+// into a ring of two (D_i = 128) or four (D_i = 64) stages;
 // warp 1 owns TMEM and issues the MMAs; warps 2-9 run the epilogue (ReLU, head
 // weights, sum, store), two
 // warps per TMEM lane quarter, each on half of the columns. Two TMEM accumulators
@@ -34,20 +35,21 @@ struct IndexerTile {
     static constexpr int BN = 256;              // (token, head) columns per tile (UMMA N)
     static constexpr int TB = BN / H_I;         // tokens per tile
     static constexpr int KSUB = D_I / 64;       // 128-byte K sub-tiles (64 fp16 each)
-    static constexpr int A_SUB = BM * 128;      // bytes of one A sub-tile (one ring stage)
+    static constexpr int A_SUB = BM * 128;      // bytes of one 64-dim A sub-tile
+    static constexpr int A_STAGE = A_SUB * KSUB;  // one ring stage: a whole k_idx tile
     static constexpr int B_SUB = BN * 128;      // bytes of one B sub-tile
     static constexpr int B_BYTES = B_SUB * KSUB;
-    static constexpr int A_STAGES = 4;
+    static constexpr int A_STAGES = KSUB == 2 ? 2 : 4;
     static constexpr int EPI_WARPS = 8;
     static constexpr int B_WARP = 2 + EPI_WARPS;                      // q_idx loader
     static constexpr int THREADS = (3 + EPI_WARPS) * 32;
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int OFF_B = 0;                                   // two B buffers
     static constexpr int OFF_A = 2 * B_BYTES;
-    static constexpr int OFF_W = OFF_A + A_STAGES * A_SUB;            // two w buffers
+    static constexpr int OFF_W = OFF_A + A_STAGES * A_STAGE;          // two w buffers
     static constexpr int OFF_BAR = OFF_W + 2 * BN * 4;
-    // afull[4], aempty[4], bfull[2], bempty[2], tfull[2], tempty[2], done
-    static constexpr int N_BARS = 2 * A_STAGES + 4 + 4 + 1;
+    // afull[A_STAGES], aempty[A_STAGES], bfull[2], bempty[2], tempty[2], done
+    static constexpr int N_BARS = 2 * A_STAGES + 2 + 2 + 2 + 1;
     static constexpr int OFF_TMEM_PTR = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;       // + alignment slack
     static constexpr uint32_t IDESC = umma_idesc_f16_f32(BM, BN);
@@ -126,9 +128,8 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     auto aempty = [&](int s) { return bar0 + 8u * (C::A_STAGES + s); };
     auto bfull = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + i); };
     auto bempty = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + 2 + i); };
-    auto tfull = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + 4 + i); };
-    auto tempty = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + 6 + i); };
-    const uint32_t done_bar = bar0 + 8u * (2 * C::A_STAGES + 8);
+    auto tempty = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + 4 + i); };
+    const uint32_t done_bar = bar0 + 8u * (2 * C::A_STAGES + 6);
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_PTR);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -140,7 +141,6 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int i = 0; i < 2; ++i) {
             mbar_init(bfull(i), 1);
             mbar_init(bempty(i), 1);
-            mbar_init(tfull(i), 1);
             mbar_init(tempty(i), C::EPI_WARPS);   // one arrive per epilogue warp
         }
         mbar_init(done_bar, 1);
@@ -161,7 +161,7 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (warp == C::B_WARP || warp == 0) {
         // ------------------------------------------------------------ TMA producers
         // The last warp loads the q_idx blocks (B) and runs up to two units ahead; warp 0
-        // streams the k_idx sub-tiles (A). Each waits only on the ring it fills.
+        // streams the k_idx tiles (A). Each waits only on the ring it fills.
         if (warp == C::B_WARP && lane == 0) {
             int bi = 0;
             int b_issued[2] = {0, 0};
@@ -191,16 +191,16 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const int u = snake_unit(r, b, G);
                 if (u >= n_units) break;
                 const IndexerUnit w = indexer_unit<C::TB>(p, u);
-                for (int it = 0; it < w.n_tiles && !abort; ++it) {
-                    for (int ks = 0; ks < C::KSUB; ++ks, ++a_it) {
-                        const int s = a_it % C::A_STAGES;
-                        if (!mbar_wait(aempty(s), ((a_it / C::A_STAGES) & 1) ^ 1, p.status, abort))
-                            break;
-                        mbar_arrive_expect_tx(afull(s), C::A_SUB);
-                        tma_load_2d(base + C::OFF_A + s * C::A_SUB, &tmap_k, afull(s), ks * 64,
-                                    w.jt(it) * C::BM);
-                        ++a_issued[s];
-                    }
+                for (int it = 0; it < w.n_tiles; ++it, ++a_it) {
+                    const int s = a_it % C::A_STAGES;
+                    if (!mbar_wait(aempty(s), ((a_it / C::A_STAGES) & 1) ^ 1, p.status, abort))
+                        break;
+                    mbar_arrive_expect_tx(afull(s), C::A_STAGE);
+#pragma unroll
+                    for (int ks = 0; ks < C::KSUB; ++ks)
+                        tma_load_2d(base + C::OFF_A + s * C::A_STAGE + ks * C::A_SUB, &tmap_k, afull(s),
+                                    ks * 64, w.jt(it) * C::BM);
+                    ++a_issued[s];
                 }
             }
             for (int s = 0; s < C::A_STAGES; ++s) {
@@ -212,7 +212,11 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int bi = 0, a_it = 0, tc = 0;
+            // Descriptors differ only in their start-address field (address >> 4 in the low
+            // 14 bits), so each stage's is built once and offset per K step.
+            const uint64_t a_desc0 = umma_desc_sw128(base + C::OFF_A);
+            const uint64_t b_desc0 = umma_desc_sw128(base + C::OFF_B);
+            int bi = 0, tc = 0;
             for (int r = 0; !abort; ++r) {
                 const int u = snake_unit(r, b, G);
                 if (u >= n_units) break;
@@ -220,24 +224,24 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 if (w.n_tiles == 0) continue;
                 const int bb = bi & 1;
                 if (!mbar_wait(bfull(bb), (bi >> 1) & 1, p.status, abort)) break;
-                const uint32_t bsm = base + C::OFF_B + bb * C::B_BYTES;
-                for (int it = 0; it < w.n_tiles && !abort; ++it, ++tc) {
-                    const int buf = tc & 1;
+                const uint64_t b_desc = b_desc0 + (uint64_t)((bb * C::B_BYTES) >> 4);
+                for (int it = 0; it < w.n_tiles; ++it, ++tc) {
+                    const int buf = tc & 1, s = tc % C::A_STAGES;
                     if (!mbar_wait(tempty(buf), ((tc >> 1) & 1) ^ 1, p.status, abort)) break;
+                    if (!mbar_wait(afull(s), (tc / C::A_STAGES) & 1, p.status, abort)) break;
+                    tc_fence_after();
                     const uint32_t d = tmem_base + buf * C::BN;
-                    for (int ks = 0; ks < C::KSUB; ++ks, ++a_it) {
-                        const int s = a_it % C::A_STAGES;
-                        if (!mbar_wait(afull(s), (a_it / C::A_STAGES) & 1, p.status, abort)) break;
-                        tc_fence_after();
-                        const uint32_t asm_ = base + C::OFF_A + s * C::A_SUB;
+                    const uint64_t a_desc = a_desc0 + (uint64_t)((s * C::A_STAGE) >> 4);
+#pragma unroll
+                    for (int ks = 0; ks < C::KSUB; ++ks)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)   // k16 steps: 32 bytes into the 128-byte row
-                            umma_f16(d, umma_desc_sw128(asm_ + kk * 32),
-                                     umma_desc_sw128(bsm + ks * C::B_SUB + kk * 32), C::IDESC,
+                            umma_f16(d, a_desc + (uint64_t)((ks * C::A_SUB + kk * 32) >> 4),
+                                     b_desc + (uint64_t)((ks * C::B_SUB + kk * 32) >> 4), C::IDESC,
                                      ks > 0 || kk > 0);
-                        umma_commit(aempty(s));          // A sub-tile free once these finish
-                    }
-                    umma_commit(tfull(buf));             // accumulator ready for the epilogue
+                    // One commit: frees the A stage and tells the epilogue that the
+                    // accumulator of this tile is complete.
+                    umma_commit(aempty(s));
                 }
                 umma_commit(bempty(bb));                 // B buffer free once the unit's MMAs finish
                 ++bi;
@@ -254,26 +258,37 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int quarter = warp & 3;                // TMEM lanes 32*quarter .. +31
         const int half = e / 4;                      // columns 128*half .. +127
         const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + half * 128;
+        // Head weight of column e*32+lane for unit u, read from global memory one unit
+        // ahead so that its latency hides behind the previous unit's tiles.
+        const int col = e * 32 + lane;
+        auto unit_weight = [&](int u) {
+            if (u >= n_units) return 0.f;
+            const IndexerUnit w = indexer_unit<C::TB>(p, u);
+            const int tl = col / H_I;
+            return (w.tok0 + tl < w.tok_end) ? p.w[(size_t)(w.tok0 - p.t0 + tl) * H_I + (col % H_I)]
+                                             : 0.f;
+        };
         int bi = 0, tc = 0;
+        float w_next = unit_weight(snake_unit(0, b, G));
         for (int r = 0;; ++r) {
             const int u = snake_unit(r, b, G);
             if (u >= n_units) break;
             const IndexerUnit w = indexer_unit<C::TB>(p, u);
+            const float w_this = w_next;
+            w_next = unit_weight(snake_unit(r + 1, b, G));
             if (w.n_tiles == 0) continue;
             // Head weights of the unit's tokens, in column order (col = token*H_i + h).
             float* swb = sw + (bi & 1) * C::BN;
-            {
-                const int col = e * 32 + lane, tl = col / H_I;
-                swb[col] = (w.tok0 + tl < w.tok_end)
-                               ? p.w[(size_t)(w.tok0 - p.t0 + tl) * H_I + (col % H_I)] : 0.f;
-            }
+            swb[col] = w_this;
             named_barrier(1, C::EPI_WARPS * 32);
             const float* wh = swb + half * 128;
             // After a wait gives up this warp keeps walking the units (waits then return at
             // once) so that it still meets every named barrier of the epilogue warps.
             for (int it = 0; it < w.n_tiles; ++it, ++tc) {
                 const int buf = tc & 1;
-                const bool ready = mbar_wait(tfull(buf), (tc >> 1) & 1, p.status, abort);
+                // The tile's A-stage barrier completes when its MMAs do.
+                const bool ready = mbar_wait(aempty(tc % C::A_STAGES), (tc / C::A_STAGES) & 1,
+                                             p.status, abort);
                 if (!__all_sync(0xffffffffu, ready)) continue;   // warp-uniform skip
                 tc_fence_after();
                 const int j = w.jt(it) * C::BM + quarter * 32 + lane;
