@@ -301,26 +301,35 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(tempty(buf));
-                float ax = 0.f, ay = 0.f;                // running sum (even, odd heads)
+                // Per token: NP independent packed accumulators keep the FMA chains short.
+                constexpr int TPW = 128 / H_I;           // tokens in this warp's 128 columns
+                constexpr int NP = H_I >= 16 ? 4 : H_I / 4;
+                const int t_first = w.tok0 + half * TPW;
 #pragma unroll
-                for (int c = 0; c < 128; c += 4) {
-                    const float4 wv = *reinterpret_cast<const float4*>(wh + c);
-                    ffma2(ax, ay, wv.x, wv.y, fmaxf(__uint_as_float(v[c / 32][c % 32]), 0.f),
-                          fmaxf(__uint_as_float(v[c / 32][c % 32 + 1]), 0.f));
-                    if ((c + 2) % H_I == 0) {
-                        const int t = w.tok0 + (half * 128 + c) / H_I;
-                        if (t < w.tok_end && j < n_vis(t, p.ratio))
-                            p.scores[(size_t)(t - p.t0) * p.ld + j] = ax + ay;
-                        ax = ay = 0.f;
+                for (int tk = 0; tk < TPW; ++tk) {
+                    float acc[2 * NP];
+#pragma unroll
+                    for (int i = 0; i < 2 * NP; ++i) acc[i] = 0.f;
+#pragma unroll
+                    for (int c = tk * H_I; c < (tk + 1) * H_I; c += 4) {
+                        const float4 wv = *reinterpret_cast<const float4*>(wh + c);
+                        const int pr = (c / 4) % NP;
+                        ffma2(acc[2 * pr], acc[2 * pr + 1], wv.x, wv.y,
+                              fmaxf(__uint_as_float(v[c / 32][c % 32]), 0.f),
+                              fmaxf(__uint_as_float(v[c / 32][c % 32 + 1]), 0.f));
+                        ffma2(acc[2 * pr], acc[2 * pr + 1], wv.z, wv.w,
+                              fmaxf(__uint_as_float(v[c / 32][c % 32 + 2]), 0.f),
+                              fmaxf(__uint_as_float(v[c / 32][c % 32 + 3]), 0.f));
                     }
-                    ffma2(ax, ay, wv.z, wv.w, fmaxf(__uint_as_float(v[c / 32][c % 32 + 2]), 0.f),
-                          fmaxf(__uint_as_float(v[c / 32][c % 32 + 3]), 0.f));
-                    if ((c + 4) % H_I == 0) {
-                        const int t = w.tok0 + (half * 128 + c + 2) / H_I;
-                        if (t < w.tok_end && j < n_vis(t, p.ratio))
-                            p.scores[(size_t)(t - p.t0) * p.ld + j] = ax + ay;
-                        ax = ay = 0.f;
+#pragma unroll
+                    for (int i = 2; i < 2 * NP; i += 2) {
+                        acc[0] += acc[i];
+                        acc[1] += acc[i + 1];
                     }
+                    const int t = t_first + tk;
+                    // j < n_vis(t) = floor((t+1)/ratio)  <=>  ratio*(j+1) <= t+1
+                    if (t < w.tok_end && p.ratio * (j + 1) <= t + 1)
+                        p.scores[(size_t)(t - p.t0) * p.ld + j] = acc[0] + acc[1];
                 }
             }
             ++bi;
