@@ -180,13 +180,13 @@ ds4sp_status launch_indexer(ds4sp_handle* h, const void* q_idx, const void* k_id
     p.ld = ld;
     p.ratio = ratio;
     p.n_tb = (n_q + C::TB - 1) / C::TB;
-    // Split the j-tiles of each token block until there are about four units per SM,
-    // keeping at least four tiles per unit; CTAs are persistent, one per SM.
-    const int n_jt_max = (n_rows + C::BM - 1) / C::BM;
-    int nsplit = 1;
-    while (p.n_tb * nsplit < 4 * h->sm_count && n_jt_max / (2 * nsplit) >= 4) nsplit *= 2;
-    p.nsplit = nsplit;
-    const int grid = std::min(p.n_tb * nsplit, h->sm_count);
+    // Persistent CTAs, one per SM, each taking an equal share of the launch's tiles
+    // (token block x 128-row j-tile); no CTA without a tile.
+    long long tiles = 0;
+    for (int tb = 0; tb < p.n_tb; ++tb)
+        tiles += (nvis(t0 + std::min((tb + 1) * C::TB, n_q) - 1, ratio) + C::BM - 1) / C::BM;
+    if (tiles == 0) return DS4SP_OK;
+    const int grid = (int)std::min<long long>(tiles, h->sm_count);
     return launch(h, kIndexer, stream, [&] {
         indexer_tcgen05_kernel<D_I, H_I><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tq, p);
     });

@@ -11,8 +11,9 @@
 // and the head sum for a token runs along that lane's columns, inside one thread:
 // no cross-lane reduction. K = D_i in steps of 16.
 //
-// Work unit: one block of 256/H_i tokens and a range of its 128-row j-tiles. CTAs are
-// persistent (one per SM) and take units in snake order over a heaviest-first list.
+// Work: the (block of 256/H_i tokens, 128-row j-tile) pairs a launch needs, in block
+// order. Persistent CTAs (one per SM) each take an equal contiguous share (within one
+// tile) and process it as one unit per token block it touches.
 // Warp roles (352 threads): warp 10 loads q_idx blocks into two B buffers, up to two
 // units ahead; warp 0 streams whole k_idx tiles (one 64-dim TMA box per K sub-tile)
 // into a ring of two (D_i = 128) or four (D_i = 64) stages;
@@ -64,38 +65,51 @@ struct IndexerParams {
     uint32_t* status;      // device status word
     int t0, n_q, ld, ratio;
     int n_tb;              // token blocks of TB tokens
-    int nsplit;            // j-tile ranges per token block
 };
 
+// j-tiles (128 compressed rows each) that token block tb needs: those below n_vis of its
+// last token.
+template <int TB>
+__device__ __forceinline__ int block_tiles(const IndexerParams& p, int tb) {
+    const int t_last = p.t0 + min((tb + 1) * TB, p.n_q) - 1;
+    return (n_vis(t_last, p.ratio) + 127) / 128;
+}
+
+// A unit: j-tiles jt_begin .. jt_begin+n_tiles-1 of one token block.
 struct IndexerUnit {
-    int tok0, tok_end, jt_begin, n_tiles, rot;
-    // j-tile of the unit's it-th tile. Each CTA starts at its own offset so that the SMs do
-    // not all fetch the same k_idx tile from L2 at the same moment.
-    __device__ __forceinline__ int jt(int it) const {
-        const int k = it + rot;
-        return jt_begin + (k >= n_tiles ? k - n_tiles : k);
+    int tok0, tok_end, jt_begin, n_tiles;
+    __device__ __forceinline__ int jt(int it) const { return jt_begin + it; }
+};
+
+// A CTA's share of the launch: `left` consecutive tiles of the list of all (token block,
+// j-tile) pairs in block order, starting at tile jt of block tb. Shares differ by at most
+// one tile; the walk cuts a share into one unit per token block it touches.
+struct IndexerWalk {
+    int tb, jt, left;
+    template <int TB>
+    __device__ __forceinline__ bool next(const IndexerParams& p, IndexerUnit& w) {
+        if (left <= 0) return false;
+        int n = block_tiles<TB>(p, tb);
+        while (n - jt <= 0 && tb + 1 < p.n_tb) {
+            ++tb;
+            jt = 0;
+            n = block_tiles<TB>(p, tb);
+        }
+        if (n - jt <= 0) {
+            left = 0;
+            return false;
+        }
+        const int take = min(n - jt, left);
+        w.tok0 = p.t0 + tb * TB;
+        w.tok_end = min(w.tok0 + TB, p.t0 + p.n_q);
+        w.jt_begin = jt;
+        w.n_tiles = take;
+        left -= take;
+        ++tb;
+        jt = 0;
+        return true;
     }
 };
-
-template <int TB>
-__device__ __forceinline__ IndexerUnit indexer_unit(const IndexerParams& p, int u) {
-    IndexerUnit w;
-    const int tb = p.n_tb - 1 - u / p.nsplit;                 // heaviest token blocks first
-    const int split = u % p.nsplit;
-    w.tok0 = p.t0 + tb * TB;
-    w.tok_end = min(w.tok0 + TB, p.t0 + p.n_q);
-    const int n_jt = (n_vis(w.tok_end - 1, p.ratio) + 127) / 128;
-    const int chunk = (n_jt + p.nsplit - 1) / p.nsplit;
-    w.jt_begin = split * chunk;
-    w.n_tiles = max(0, min(n_jt, w.jt_begin + chunk) - w.jt_begin);
-    w.rot = w.n_tiles > 0 ? (int)(blockIdx.x % (unsigned)w.n_tiles) : 0;
-    return w;
-}
-
-// Unit taken by CTA b in round r: snake order pairs heavy units with light ones.
-__device__ __forceinline__ int snake_unit(int r, int b, int G) {
-    return r * G + ((r & 1) ? (G - 1 - b) : b);
-}
 
 // acc.xy += a.xy * b.xy as one packed fp32x2 FMA (round-to-nearest per lane).
 __device__ __forceinline__ void ffma2(float& acc_x, float& acc_y, float a_x, float a_y, float b_x,
@@ -115,7 +129,6 @@ __global__ void __launch_bounds__(IndexerTile<D_I, H_I>::THREADS, 1)
 indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_q, IndexerParams p) {
     using C = IndexerTile<D_I, H_I>;
-    const int n_units = p.n_tb * p.nsplit;
     const int G = gridDim.x, b = blockIdx.x;
 
     extern __shared__ uint8_t smem_raw[];
@@ -133,6 +146,38 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_PTR);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    __shared__ int s_walk[3];
+    if (warp == 2) {
+        // This CTA's share: tiles [b*T/G, (b+1)*T/G) of the T tiles of the launch. Each
+        // lane sums the tiles of a contiguous run of token blocks; a warp scan gives the
+        // run's first tile; the lane whose run holds the share's first tile finds it.
+        const int per = (p.n_tb + 31) / 32;
+        const int b0 = min(p.n_tb, lane * per), b1 = min(p.n_tb, b0 + per);
+        int sum = 0;
+        for (int tb = b0; tb < b1; ++tb) sum += block_tiles<C::TB>(p, tb);
+        int incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31), excl = incl - sum;
+        const int first = (int)((long long)b * total / G);
+        const int last = (int)((long long)(b + 1) * total / G);
+        if (lane == 0) {
+            s_walk[0] = 0;
+            s_walk[1] = 0;
+            s_walk[2] = 0;
+        }
+        __syncwarp();
+        if (first >= excl && first < incl) {
+            int acc = excl, tb = b0;
+            while (tb + 1 < b1 && acc + block_tiles<C::TB>(p, tb) <= first) acc += block_tiles<C::TB>(p, tb++);
+            s_walk[0] = tb;
+            s_walk[1] = first - acc;
+            s_walk[2] = last - first;
+        }
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::A_STAGES; ++s) {
             mbar_init(afull(s), 1);
@@ -156,6 +201,7 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_ptr;
+    const IndexerWalk walk0{s_walk[0], s_walk[1], s_walk[2]};
 
     bool abort = false;
     if (warp == C::B_WARP || warp == 0) {
@@ -165,11 +211,9 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (warp == C::B_WARP && lane == 0) {
             int bi = 0;
             int b_issued[2] = {0, 0};
-            for (int r = 0; !abort; ++r) {
-                const int u = snake_unit(r, b, G);
-                if (u >= n_units) break;
-                const IndexerUnit w = indexer_unit<C::TB>(p, u);
-                if (w.n_tiles == 0) continue;
+            IndexerWalk wk = walk0;
+            IndexerUnit w;
+            while (!abort && wk.next<C::TB>(p, w)) {
                 const int bb = bi & 1;
                 if (!mbar_wait(bempty(bb), ((bi >> 1) & 1) ^ 1, p.status, abort)) break;
                 mbar_arrive_expect_tx(bfull(bb), C::B_BYTES);
@@ -187,10 +231,9 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         } else if (warp == 0 && lane == 0) {
             int a_it = 0;
             int a_issued[C::A_STAGES] = {};
-            for (int r = 0; !abort; ++r) {
-                const int u = snake_unit(r, b, G);
-                if (u >= n_units) break;
-                const IndexerUnit w = indexer_unit<C::TB>(p, u);
+            IndexerWalk wk = walk0;
+            IndexerUnit w;
+            while (!abort && wk.next<C::TB>(p, w)) {
                 for (int it = 0; it < w.n_tiles; ++it, ++a_it) {
                     const int s = a_it % C::A_STAGES;
                     if (!mbar_wait(aempty(s), ((a_it / C::A_STAGES) & 1) ^ 1, p.status, abort))
@@ -217,11 +260,9 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const uint64_t a_desc0 = umma_desc_sw128(base + C::OFF_A);
             const uint64_t b_desc0 = umma_desc_sw128(base + C::OFF_B);
             int bi = 0, tc = 0;
-            for (int r = 0; !abort; ++r) {
-                const int u = snake_unit(r, b, G);
-                if (u >= n_units) break;
-                const IndexerUnit w = indexer_unit<C::TB>(p, u);
-                if (w.n_tiles == 0) continue;
+            IndexerWalk wk = walk0;
+            IndexerUnit w;
+            while (!abort && wk.next<C::TB>(p, w)) {
                 const int bb = bi & 1;
                 if (!mbar_wait(bfull(bb), (bi >> 1) & 1, p.status, abort)) break;
                 const uint64_t b_desc = b_desc0 + (uint64_t)((bb * C::B_BYTES) >> 4);
@@ -258,25 +299,24 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int quarter = warp & 3;                // TMEM lanes 32*quarter .. +31
         const int half = e / 4;                      // columns 128*half .. +127
         const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + half * 128;
-        // Head weight of column e*32+lane for unit u, read from global memory one unit
+        // Head weight of column e*32+lane for a unit, read from global memory one unit
         // ahead so that its latency hides behind the previous unit's tiles.
         const int col = e * 32 + lane;
-        auto unit_weight = [&](int u) {
-            if (u >= n_units) return 0.f;
-            const IndexerUnit w = indexer_unit<C::TB>(p, u);
+        auto unit_weight = [&](const IndexerUnit& w) {
             const int tl = col / H_I;
             return (w.tok0 + tl < w.tok_end) ? p.w[(size_t)(w.tok0 - p.t0 + tl) * H_I + (col % H_I)]
                                              : 0.f;
         };
         int bi = 0, tc = 0;
-        float w_next = unit_weight(snake_unit(0, b, G));
-        for (int r = 0;; ++r) {
-            const int u = snake_unit(r, b, G);
-            if (u >= n_units) break;
-            const IndexerUnit w = indexer_unit<C::TB>(p, u);
+        IndexerWalk wk = walk0;
+        IndexerUnit w, w_nx;
+        bool have = wk.next<C::TB>(p, w_nx);
+        float w_next = have ? unit_weight(w_nx) : 0.f;
+        while (have) {
+            w = w_nx;
             const float w_this = w_next;
-            w_next = unit_weight(snake_unit(r + 1, b, G));
-            if (w.n_tiles == 0) continue;
+            have = wk.next<C::TB>(p, w_nx);
+            w_next = have ? unit_weight(w_nx) : 0.f;
             // Head weights of the unit's tokens, in column order (col = token*H_i + h).
             float* swb = sw + (bi & 1) * C::BN;
             swb[col] = w_this;
