@@ -180,13 +180,28 @@ ds4sp_status launch_indexer(ds4sp_handle* h, const void* q_idx, const void* k_id
     p.ld = ld;
     p.ratio = ratio;
     p.n_tb = (n_q + C::TB - 1) / C::TB;
-    // Persistent CTAs, one per SM, each taking an equal share of the launch's tiles
-    // (token block x 128-row j-tile); no CTA without a tile.
+    // Persistent CTAs, one per SM, each taking an equal contiguous share of the launch's
+    // tiles (token block x 128-row j-tile, in block order); no CTA without a tile.
+    auto block_tiles = [&](int tb) {
+        return (nvis(t0 + std::min((tb + 1) * C::TB, n_q) - 1, ratio) + C::BM - 1) / C::BM;
+    };
     long long tiles = 0;
-    for (int tb = 0; tb < p.n_tb; ++tb)
-        tiles += (nvis(t0 + std::min((tb + 1) * C::TB, n_q) - 1, ratio) + C::BM - 1) / C::BM;
+    for (int tb = 0; tb < p.n_tb; ++tb) tiles += block_tiles(tb);
     if (tiles == 0) return DS4SP_OK;
-    const int grid = (int)std::min<long long>(tiles, h->sm_count);
+    if (tiles > (1 << 30) || p.n_tb > 65535)
+        return fail(DS4SP_ERR_UNSUPPORTED, "indexer launch of %lld tiles", tiles);
+    const int grid = (int)std::min<long long>(tiles, std::min(h->sm_count, kIndexerMaxGrid));
+    p.total = (int)tiles;
+    {
+        int tb = 0;
+        long long before = 0;                     // tiles of blocks < tb
+        for (int b = 0; b < grid; ++b) {
+            const long long first = (long long)b * tiles / grid;
+            while (before + block_tiles(tb) <= first) before += block_tiles(tb++);
+            p.start_tb[b] = (uint16_t)tb;
+            p.start_jt[b] = (uint16_t)(first - before);
+        }
+    }
     return launch(h, kIndexer, stream, [&] {
         indexer_tcgen05_kernel<D_I, H_I><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tq, p);
     });

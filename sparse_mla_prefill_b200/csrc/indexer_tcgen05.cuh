@@ -59,12 +59,17 @@ struct IndexerTile {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
+constexpr int kIndexerMaxGrid = 160;
+
 struct IndexerParams {
     const float* w;        // [n_q, H_i] fp32, row 0 = token t0
     float* scores;         // [n_q, ld] fp32 scratch
     uint32_t* status;      // device status word
     int t0, n_q, ld, ratio;
     int n_tb;              // token blocks of TB tokens
+    int total;             // (token block, j-tile) pairs of the launch
+    // First tile of CTA b's share: token block start_tb[b], j-tile start_jt[b].
+    uint16_t start_tb[kIndexerMaxGrid], start_jt[kIndexerMaxGrid];
 };
 
 // j-tiles (128 compressed rows each) that token block tb needs: those below n_vis of its
@@ -146,38 +151,6 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_PTR);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    __shared__ int s_walk[3];
-    if (warp == 2) {
-        // This CTA's share: tiles [b*T/G, (b+1)*T/G) of the T tiles of the launch. Each
-        // lane sums the tiles of a contiguous run of token blocks; a warp scan gives the
-        // run's first tile; the lane whose run holds the share's first tile finds it.
-        const int per = (p.n_tb + 31) / 32;
-        const int b0 = min(p.n_tb, lane * per), b1 = min(p.n_tb, b0 + per);
-        int sum = 0;
-        for (int tb = b0; tb < b1; ++tb) sum += block_tiles<C::TB>(p, tb);
-        int incl = sum;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += o;
-        }
-        const int total = __shfl_sync(0xffffffffu, incl, 31), excl = incl - sum;
-        const int first = (int)((long long)b * total / G);
-        const int last = (int)((long long)(b + 1) * total / G);
-        if (lane == 0) {
-            s_walk[0] = 0;
-            s_walk[1] = 0;
-            s_walk[2] = 0;
-        }
-        __syncwarp();
-        if (first >= excl && first < incl) {
-            int acc = excl, tb = b0;
-            while (tb + 1 < b1 && acc + block_tiles<C::TB>(p, tb) <= first) acc += block_tiles<C::TB>(p, tb++);
-            s_walk[0] = tb;
-            s_walk[1] = first - acc;
-            s_walk[2] = last - first;
-        }
-    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::A_STAGES; ++s) {
             mbar_init(afull(s), 1);
@@ -201,7 +174,10 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_ptr;
-    const IndexerWalk walk0{s_walk[0], s_walk[1], s_walk[2]};
+    // This CTA's share: tiles [b*T/G, (b+1)*T/G) of the launch's T tiles; the host found
+    // where it starts.
+    const IndexerWalk walk0{p.start_tb[b], p.start_jt[b],
+                            (int)((long long)(b + 1) * p.total / G - (long long)b * p.total / G)};
 
     bool abort = false;
     if (warp == C::B_WARP || warp == 0) {
