@@ -121,6 +121,42 @@ ds4sp_status ds4sp_prefill_band(ds4sp_handle* h, int b, int n_tokens, const void
                                 const void* kv_cmp, const void* k_idx, int32_t* topk,
                                 float* out, void* ws, size_t ws_bytes, void* stream);
 
+/* Whole-sequence tensors of one prefill, by role (all row-major, layouts as for
+ * ds4sp_prefill_band). As inputs of ds4sp_prefill_host they live in host memory (pinned
+ * memory lets the copies run asynchronously; pageable memory works but serialises the
+ * copies); as its device buffers they live on the handle's device. topk may be NULL
+ * in the host set (indices are then not copied back); with top_k = 0 it is unused. */
+typedef struct ds4sp_io {
+    const void* q;        /* [n_tokens, 16, 576] fp16 */
+    const void* q_idx;    /* [n_tokens, H_i, D_i] fp16 */
+    const float* w;       /* [n_tokens, H_i] fp32 */
+    const void* kv_raw;   /* [n_tokens, 576] fp16 */
+    const void* kv_cmp;   /* [n_tokens/4, 576] fp16 */
+    const void* k_idx;    /* [n_tokens/4, D_i] fp16 */
+    int32_t* topk;        /* [n_tokens, top_k] int32 (output) */
+    float* out;           /* [n_tokens, 16, 512] fp32 (output) */
+} ds4sp_io;
+
+/* A whole n_tokens prefill from host memory to host memory: every band in order, as
+ * ds4sp_prefill_band does, with the transfers overlapped. Band b's rows of q, q_idx and
+ * w, and the KV, compressed-KV and index-key rows it is the first band to need, are
+ * copied in on a copy stream of the handle; band b computes on `stream` once they have
+ * arrived; band b's rows of out (and topk) go back on a second copy stream of the
+ * handle, so copies in, compute and copies out of neighbouring bands run at the same
+ * time. The pages commit bands in order ("perf(ds4): extend sparse prefill scheduling
+ * to 10K", Summary); this entry point is the host side of that loop.
+ *   host  inputs and outputs in host memory; dev  device buffers of the same shapes
+ *   (all of them required, including topk when top_k > 0), overwritten by the call;
+ *   ws    device scratch of ws_bytes >= ds4sp_workspace_bytes(h, t0, band) for every
+ *   band (the largest is the last band's).
+ * Resets the handle's band order to 0 and leaves it at the band after the last. All
+ * work is ordered after work already queued on `stream`, and the call returns without
+ * waiting: host->out (and host->topk) hold the result once `stream` has completed. The
+ * host buffers must stay valid and unchanged until then. Errors as for
+ * ds4sp_prefill_band; a failed copy returns DS4SP_ERR_CUDA. */
+ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* host,
+                                const ds4sp_io* dev, void* ws, size_t ws_bytes, void* stream);
+
 /* Set the band the next ds4sp_prefill_band call must name (resume or restart). */
 ds4sp_status ds4sp_reset(ds4sp_handle* h, int next_band);
 

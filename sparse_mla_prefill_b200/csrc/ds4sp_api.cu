@@ -62,6 +62,10 @@ struct ds4sp_handle {
     std::vector<TimedLaunch> timed;
     std::vector<cudaEvent_t> event_pool;
     bool smem_set[3] = {false, false, false};
+    // ds4sp_prefill_host: copy streams (in, out) and per-band events, made on first use.
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
+    std::vector<cudaEvent_t> band_in, band_done;
+    cudaEvent_t host_start = nullptr, host_end = nullptr;
 };
 
 namespace {
@@ -408,6 +412,16 @@ ds4sp_status ds4sp_destroy(ds4sp_handle* h) {
         cudaEventDestroy(tl.stop);
     }
     for (auto e : h->event_pool) cudaEventDestroy(e);
+    if (h->copy_in && cudaStreamSynchronize(h->copy_in) != cudaSuccess)
+        s = fail(DS4SP_ERR_CUDA, "pending copies failed before destroy");
+    if (h->copy_out && cudaStreamSynchronize(h->copy_out) != cudaSuccess)
+        s = fail(DS4SP_ERR_CUDA, "pending copies failed before destroy");
+    for (auto e : h->band_in) cudaEventDestroy(e);
+    for (auto e : h->band_done) cudaEventDestroy(e);
+    if (h->host_start) cudaEventDestroy(h->host_start);
+    if (h->host_end) cudaEventDestroy(h->host_end);
+    if (h->copy_in) cudaStreamDestroy(h->copy_in);
+    if (h->copy_out) cudaStreamDestroy(h->copy_out);
     if (h->last) cudaEventDestroy(h->last);
     if (h->d_status) cudaFree(h->d_status);
     delete h;
@@ -478,6 +492,114 @@ ds4sp_status ds4sp_prefill_band(ds4sp_handle* h, int b, int n_tokens, const void
     DS4SP_TRY(sparse_attn_impl(h, qh, kv_raw, kv_cmp, tk, t0, n_q, ot, s));
     h->next_band = b + 1;
     return DS4SP_OK;
+}
+
+ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* host,
+                                const ds4sp_io* dev, void* ws, size_t ws_bytes, void* stream) {
+    DS4SP_TRY(check_handle(h));
+    if (!host || !dev) return fail(DS4SP_ERR_INVALID_ARG, "host or dev is null");
+    const ds4sp_config& c = h->cfg;
+    if (n_tokens < 1 || n_tokens > c.max_tokens)
+        return fail(DS4SP_ERR_INVALID_ARG, "n_tokens %d outside [1, %d]", n_tokens, c.max_tokens);
+    const bool sel = c.top_k > 0;
+    const int n_c = nvis(n_tokens - 1, c.ratio);   // compressed rows the last token sees
+    for (const ds4sp_io* io : {host, dev}) {
+        const char* side = io == host ? "host" : "dev";
+        if (!io->q || !io->q_idx || !io->w || !io->kv_raw || !io->out)
+            return fail(DS4SP_ERR_INVALID_ARG, "%s: null q, q_idx, w, kv_raw or out", side);
+        if (n_c > 0 && sel && (!io->kv_cmp || !io->k_idx))
+            return fail(DS4SP_ERR_INVALID_ARG, "%s: null kv_cmp or k_idx", side);
+    }
+    if (sel && !dev->topk) return fail(DS4SP_ERR_INVALID_ARG, "dev: null topk");
+    const int n_bands = (n_tokens + c.band - 1) / c.band;
+    const size_t need = ds4sp_workspace_bytes(h, (n_bands - 1) * c.band,
+                                              n_tokens - (n_bands - 1) * c.band);
+    if (sel && ws_bytes < need)
+        return fail(DS4SP_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+
+    cudaError_t e = cudaSuccess;
+    if (!h->copy_in) e = cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !h->copy_out)
+        e = cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !h->host_start)
+        e = cudaEventCreateWithFlags(&h->host_start, cudaEventDisableTiming);
+    if (e == cudaSuccess && !h->host_end)
+        e = cudaEventCreateWithFlags(&h->host_end, cudaEventDisableTiming);
+    while (e == cudaSuccess && (int)h->band_in.size() < n_bands) {
+        cudaEvent_t a = nullptr, b = nullptr;
+        e = cudaEventCreateWithFlags(&a, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&b, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            if (a) cudaEventDestroy(a);
+            break;
+        }
+        h->band_in.push_back(a);
+        h->band_done.push_back(b);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: streams/events");
+
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // Copies start after whatever the caller queued on `stream` before this call.
+    e = cudaEventRecord(h->host_start, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_in, h->host_start, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: ordering");
+
+    const size_t q_row = (size_t)c.n_heads * c.d_qk * 2, qi_row = (size_t)c.n_idx_heads * c.d_idx * 2;
+    const size_t w_row = (size_t)c.n_idx_heads * 4, kv_row = (size_t)c.d_qk * 2;
+    const size_t ki_row = (size_t)c.d_idx * 2, o_row = (size_t)c.n_heads * c.d_v * 4;
+    const size_t tk_row = (size_t)c.top_k * 4;
+    auto h2d = [&](const void* dst, const void* src, size_t off, size_t bytes) {
+        if (bytes == 0) return cudaSuccess;
+        return cudaMemcpyAsync(static_cast<char*>(const_cast<void*>(dst)) + off,
+                               static_cast<const char*>(src) + off, bytes,
+                               cudaMemcpyHostToDevice, h->copy_in);
+    };
+    auto d2h = [&](void* dst, const void* src, size_t off, size_t bytes) {
+        if (bytes == 0) return cudaSuccess;
+        return cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off,
+                               bytes, cudaMemcpyDeviceToHost, h->copy_out);
+    };
+    // Inputs: per band, its token rows and the KV rows it is the first to need.
+    int raw_done = 0, cmp_done = 0;
+    for (int b = 0; b < n_bands && e == cudaSuccess; ++b) {
+        const int t0 = b * c.band, t1 = std::min(n_tokens, t0 + c.band), n = t1 - t0;
+        e = h2d(dev->q, host->q, t0 * q_row, n * q_row);
+        if (e == cudaSuccess && sel) e = h2d(dev->q_idx, host->q_idx, t0 * qi_row, n * qi_row);
+        if (e == cudaSuccess && sel) e = h2d(dev->w, host->w, t0 * w_row, n * w_row);
+        if (e == cudaSuccess) e = h2d(dev->kv_raw, host->kv_raw, raw_done * kv_row, (t1 - raw_done) * kv_row);
+        raw_done = t1;
+        const int cmp_need = sel ? nvis(t1 - 1, c.ratio) : 0;
+        if (e == cudaSuccess && cmp_need > cmp_done) {
+            e = h2d(dev->kv_cmp, host->kv_cmp, cmp_done * kv_row, (cmp_need - cmp_done) * kv_row);
+            if (e == cudaSuccess)
+                e = h2d(dev->k_idx, host->k_idx, cmp_done * ki_row, (cmp_need - cmp_done) * ki_row);
+            cmp_done = cmp_need;
+        }
+        if (e == cudaSuccess) e = cudaEventRecord(h->band_in[b], h->copy_in);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: copies in");
+
+    // Compute, band by band, each after its inputs; outputs copied back band by band.
+    h->next_band = 0;
+    for (int b = 0; b < n_bands; ++b) {
+        const int t0 = b * c.band, n = std::min(n_tokens, t0 + c.band) - t0;
+        e = cudaStreamWaitEvent(s, h->band_in[b], 0);
+        if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: wait for inputs");
+        DS4SP_TRY(ds4sp_prefill_band(h, b, n_tokens, dev->q, dev->q_idx, dev->w, dev->kv_raw,
+                                     dev->kv_cmp, dev->k_idx, dev->topk, dev->out, ws, ws_bytes,
+                                     stream));
+        e = cudaEventRecord(h->band_done[b], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->band_done[b], 0);
+        if (e == cudaSuccess) e = d2h(host->out, dev->out, t0 * o_row, n * o_row);
+        if (e == cudaSuccess && sel && host->topk)
+            e = d2h(host->topk, dev->topk, t0 * tk_row, n * tk_row);
+        if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: copies out");
+    }
+    // `stream` completes only after the last copy out.
+    e = cudaEventRecord(h->host_end, h->copy_out);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, h->host_end, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: ordering");
+    return record_last(h, s);
 }
 
 ds4sp_status ds4sp_reset(ds4sp_handle* h, int next_band) {

@@ -34,6 +34,12 @@ class ds4sp_config(ctypes.Structure):
                 ("max_tokens", ctypes.c_int), ("softmax_scale", ctypes.c_float)]
 
 
+class ds4sp_io(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("q_idx", ctypes.c_void_p), ("w", ctypes.c_void_p),
+                ("kv_raw", ctypes.c_void_p), ("kv_cmp", ctypes.c_void_p), ("k_idx", ctypes.c_void_p),
+                ("topk", ctypes.c_void_p), ("out", ctypes.c_void_p)]
+
+
 _lib: Optional[ctypes.CDLL] = None
 _vp, _i32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
@@ -44,6 +50,8 @@ _SIGS = {
     "ds4sp_indexer_topk": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _sz, _vp]),
     "ds4sp_sparse_attn": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp]),
     "ds4sp_prefill_band": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                  _vp, _sz, _vp]),
+    "ds4sp_prefill_host": (_i32, [_vp, _i32, ctypes.POINTER(ds4sp_io), ctypes.POINTER(ds4sp_io),
                                   _vp, _sz, _vp]),
     "ds4sp_reset": (_i32, [_vp, _i32]),
     "ds4sp_next_band": (_i32, [_vp]),
@@ -261,14 +269,42 @@ def prefill(h: Handle, inputs: Dict[str, torch.Tensor], n_tokens: int,
                            stream)
 
 
+def _io(t: Dict[str, torch.Tensor], topk: Optional[torch.Tensor], out: torch.Tensor,
+        pinned: bool) -> ds4sp_io:
+    def ptr(name, x, dtype):
+        if x is None:
+            return None
+        if pinned and x.is_cuda:
+            raise ValueError(f"{name}: expected a host tensor")
+        if not pinned and not x.is_cuda:
+            raise ValueError(f"{name}: expected a device tensor")
+        if x.dtype != dtype or not x.is_contiguous():
+            raise ValueError(f"{name}: expected a contiguous {dtype} tensor")
+        return x.data_ptr()
+    f16, f32, i32 = torch.float16, torch.float32, torch.int32
+    return ds4sp_io(ptr("q", t["q"], f16), ptr("q_idx", t["q_idx"], f16), ptr("w", t["w"], f32),
+                    ptr("kv_raw", t["kv_raw"], f16), ptr("kv_cmp", t.get("kv_cmp"), f16),
+                    ptr("k_idx", t.get("k_idx"), f16), ptr("topk", topk, i32), ptr("out", out, f32))
+
+
+def ds4sp_prefill_host(h: Handle, n_tokens: int, host: Dict[str, torch.Tensor],
+                       host_topk: Optional[torch.Tensor], host_out: torch.Tensor,
+                       dev: Dict[str, torch.Tensor], dev_topk: Optional[torch.Tensor],
+                       dev_out: torch.Tensor, ws: Optional[torch.Tensor], stream=None) -> None:
+    lib = load_library()
+    hio, dio = _io(host, host_topk, host_out, True), _io(dev, dev_topk, dev_out, False)
+    _check(lib.ds4sp_prefill_host(h.ptr, n_tokens, ctypes.byref(hio), ctypes.byref(dio),
+                                  _ptr(ws, "ws"),
+                                  ws.numel() * ws.element_size() if ws is not None else 0,
+                                  _stream(stream)), "ds4sp_prefill_host")
+
+
 def prefill_host(h: Handle, host: Dict[str, torch.Tensor], dev: Dict[str, torch.Tensor],
                  n_tokens: int, topk: torch.Tensor, out: torch.Tensor, ws: torch.Tensor,
-                 out_host: torch.Tensor, stream=None) -> None:
-    """Prefill from host (pinned) inputs into a host output: copies each input to its
-    device buffer, runs every band, copies ``out`` back. Asynchronous on the stream."""
+                 out_host: torch.Tensor, stream=None, topk_host: Optional[torch.Tensor] = None) -> None:
+    """Prefill from host (pinned) inputs into a host output through ds4sp_prefill_host:
+    per band, inputs copied in, computed, output copied back, the three overlapped across
+    bands. ``dev``, ``topk`` and ``out`` are the device buffers. Asynchronous on the
+    stream."""
     s = torch.cuda.current_stream() if stream is None else stream
-    with torch.cuda.stream(s):
-        for k in ("q", "q_idx", "w", "kv_raw", "kv_cmp", "k_idx"):
-            dev[k].copy_(host[k], non_blocking=True)
-        prefill(h, dev, n_tokens, topk, out, ws, s)
-        out_host.copy_(out, non_blocking=True)
+    ds4sp_prefill_host(h, n_tokens, host, topk_host, out_host, dev, topk, out, ws, s)

@@ -72,6 +72,9 @@ def test_null_handle_paths(lib):
     assert lib.ds4sp_create(None, None) == D.ERR_INVALID_ARG
     for fn in ("ds4sp_profile_enable", "ds4sp_debug_fail_launches"):
         assert getattr(lib, fn)(None, 1) == D.ERR_INVALID_ARG
+    io = D.ds4sp_io()
+    assert lib.ds4sp_prefill_host(None, 16, ctypes.byref(io), ctypes.byref(io), None, 0,
+                                  None) == D.ERR_INVALID_ARG
 
 
 def test_status_strings(lib):
