@@ -155,6 +155,12 @@ __device__ __forceinline__ void named_barrier(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Ask L2 to fetch [src, src+bytes) from global memory (no destination, no completion
+// signal). bytes is a multiple of 16 and src 16-byte aligned.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Per-warpgroup register budget changes (all four warps of a warpgroup execute them).
 template <int N>
 __device__ __forceinline__ void regs_increase() {

@@ -250,7 +250,8 @@ ds4sp_status launch_topk(ds4sp_handle* h, const float* scores, int ld, int t0, i
 }
 
 ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, const void* kv_cmp,
-                         const int32_t* topk, int t0, int n_q, float* out, cudaStream_t stream) {
+                         const int32_t* topk, int t0, int n_q, float* out, cudaStream_t stream,
+                         const void* prefetch = nullptr, size_t prefetch_bytes = 0) {
     const int smem = attn::smem_bytes(h->cfg.top_k);
     if (!h->smem_set[kAttn]) {
         const cudaError_t e = cudaFuncSetAttribute(sparse_attn_mma_kernel,
@@ -278,6 +279,10 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
     p.n_swa = h->cfg.n_swa;
     p.ratio = h->cfg.ratio;
     p.scale_log2 = scale_of(h->cfg) * 1.4426950408889634f;
+    // The region must start 16-byte aligned; its length is cut to a multiple of 16.
+    const bool pf = prefetch && aligned16(prefetch) && prefetch_bytes >= 16;
+    p.prefetch = pf ? static_cast<const char*>(prefetch) : nullptr;
+    p.prefetch_bytes = pf ? (long long)(prefetch_bytes / 16 * 16) : 0;
     return launch(h, kAttn, stream, [&] {
         // persistent: one CTA per SM, each walking its share of the tokens
         const int grid = std::min(n_q, h->sm_count);
@@ -348,7 +353,8 @@ ds4sp_status indexer_topk_impl(ds4sp_handle* h, const void* q_idx, const void* k
 
 ds4sp_status sparse_attn_impl(ds4sp_handle* h, const void* q, const void* kv_raw,
                               const void* kv_cmp, const int32_t* topk, int t0, int n_q,
-                              float* out, cudaStream_t stream) {
+                              float* out, cudaStream_t stream, const void* prefetch = nullptr,
+                              size_t prefetch_bytes = 0) {
     DS4SP_TRY(check_range(h, t0, n_q));
     if (n_q == 0) return DS4SP_OK;
     DS4SP_TRY(check_ptr(q, "q"));
@@ -358,7 +364,8 @@ ds4sp_status sparse_attn_impl(ds4sp_handle* h, const void* q, const void* kv_raw
         DS4SP_TRY(check_ptr(topk, "topk"));
         if (nvis(t0 + n_q - 1, h->cfg.ratio) > 0) DS4SP_TRY(check_ptr(kv_cmp, "kv_cmp"));
     }
-    DS4SP_TRY(launch_attn(h, q, kv_raw, kv_cmp, topk, t0, n_q, out, stream));
+    DS4SP_TRY(launch_attn(h, q, kv_raw, kv_cmp, topk, t0, n_q, out, stream, prefetch,
+                          prefetch_bytes));
     return record_last(h, stream);
 }
 
@@ -489,7 +496,16 @@ ds4sp_status ds4sp_prefill_band(ds4sp_handle* h, int b, int n_tokens, const void
                         ds4sp_workspace_bytes(h, t0, n_q));
         DS4SP_TRY(indexer_topk_impl(h, qi, k_idx, wt, t0, n_q, tk, ws, ws_bytes, s));
     }
-    DS4SP_TRY(sparse_attn_impl(h, qh, kv_raw, kv_cmp, tk, t0, n_q, ot, s));
+    // The next band's indexer queries (read first thing by its indexer) are brought into
+    // L2 at the tail of this band's attention.
+    const int t1 = t0 + n_q, n_next = std::min(c.band, n_tokens - t1);
+    const void* pf = nullptr;
+    size_t pf_bytes = 0;
+    if (c.top_k > 0 && n_next > 0) {
+        pf = static_cast<const __half*>(q_idx) + (size_t)t1 * c.n_idx_heads * c.d_idx;
+        pf_bytes = (size_t)n_next * c.n_idx_heads * c.d_idx * 2;
+    }
+    DS4SP_TRY(sparse_attn_impl(h, qh, kv_raw, kv_cmp, tk, t0, n_q, ot, s, pf, pf_bytes));
     h->next_band = b + 1;
     return DS4SP_OK;
 }

@@ -114,6 +114,11 @@ struct AttnParams {
     uint32_t* status;
     int t0, n_q, k, n_swa, ratio;
     float scale_log2;      // softmax scale * log2(e)
+    // Optional: a region the next kernel will read (the next band's indexer queries);
+    // once a CTA's producers have issued their last copy they ask L2 to fetch this CTA's
+    // slice of it, while the consumers finish. NULL or 0 bytes: nothing.
+    const char* prefetch;
+    long long prefetch_bytes;
 };
 
 struct TokenRows {
@@ -290,6 +295,16 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                 reinterpret_cast<volatile uint8_t*>(rowmask + s)[pw] = (uint8_t)m8;
                 mbar_arrive(full_bar(s));         // release: the mask byte is visible with the slot
             }
+        }
+        if (p.prefetch_bytes > 0 && !abort) {
+            // This CTA's slice of the region, in 16-byte-aligned pieces of up to 32 KB,
+            // spread over the producer warps' first lanes.
+            const long long per = (p.prefetch_bytes / gridDim.x + 15) / 16 * 16;
+            const long long lo = per * blockIdx.x;
+            const long long hi = min(p.prefetch_bytes, lo + per);
+            if (lane == 0)
+                for (long long off = lo + (long long)pw * 32768; off < hi; off += PWARPS * 32768LL)
+                    prefetch_l2(p.prefetch + off, (uint32_t)min(32768LL, hi - off));
         }
         cp_async_wait<0>();
     } else {
