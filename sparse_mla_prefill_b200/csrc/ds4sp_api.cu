@@ -195,16 +195,47 @@ ds4sp_status launch_indexer(ds4sp_handle* h, const void* q_idx, const void* k_id
     if (tiles > (1 << 30) || p.n_tb > 65535)
         return fail(DS4SP_ERR_UNSUPPORTED, "indexer launch of %lld tiles", tiles);
     const int grid = (int)std::min<long long>(tiles, std::min(h->sm_count, kIndexerMaxGrid));
-    p.total = (int)tiles;
+    if ((tiles + p.n_tb) / grid + 2 > 65535)     // a share's tile count must fit 16 bits
+        return fail(DS4SP_ERR_UNSUPPORTED, "indexer launch of %lld tiles", tiles);
     {
-        int tb = 0;
-        long long before = 0;                     // tiles of blocks < tb
-        for (int b = 0; b < grid; ++b) {
-            const long long first = (long long)b * tiles / grid;
-            while (before + block_tiles(tb) <= first) before += block_tiles(tb++);
-            p.start_tb[b] = (uint16_t)tb;
-            p.start_jt[b] = (uint16_t)(first - before);
+        // Cut the tile list into `grid` contiguous shares of about equal cost: one per
+        // tile, plus kLoadCost for the first tile of each token block (its q_idx block
+        // load). Every share gets at least one tile.
+        constexpr double kLoadCost = 1.0;
+        const double total_cost = (double)tiles + kLoadCost * p.n_tb;
+        int b = 0, tb = 0, jt = 0, nb = block_tiles(0);
+        long long left_tiles = tiles;
+        double cost = 0.0;
+        p.start_tb[0] = 0;
+        p.start_jt[0] = 0;
+        int count = 0;
+        while (left_tiles > 0) {
+            while (jt >= nb) {                    // next token block with tiles
+                ++tb;
+                jt = 0;
+                nb = block_tiles(tb);
+            }
+            cost += 1.0 + (jt == 0 ? kLoadCost : 0.0);
+            ++count;
+            ++jt;
+            --left_tiles;
+            const double target = total_cost * (b + 1) / grid;
+            // Close share b at its cost target, but leave a tile for every later share.
+            if (b + 1 < grid && (cost >= target || left_tiles == grid - 1 - b)) {
+                p.count[b] = (uint16_t)count;
+                ++b;
+                count = 0;
+                while (jt >= nb && left_tiles > 0) {
+                    ++tb;
+                    jt = 0;
+                    nb = block_tiles(tb);
+                }
+                p.start_tb[b] = (uint16_t)tb;
+                p.start_jt[b] = (uint16_t)jt;
+            }
         }
+        p.count[b] = (uint16_t)count;
+        if (b != grid - 1) return fail(DS4SP_ERR_CUDA, "indexer partition: %d of %d shares", b + 1, grid);
     }
     return launch(h, kIndexer, stream, [&] {
         indexer_tcgen05_kernel<D_I, H_I><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tq, p);

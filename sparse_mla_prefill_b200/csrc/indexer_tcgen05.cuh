@@ -12,8 +12,9 @@
 // no cross-lane reduction. K = D_i in steps of 16.
 //
 // Work: the (block of 256/H_i tokens, 128-row j-tile) pairs a launch needs, in block
-// order. Persistent CTAs (one per SM) each take an equal contiguous share (within one
-// tile) and process it as one unit per token block it touches.
+// order. Persistent CTAs (one per SM) each take a contiguous share of about equal cost
+// (a tile, plus the q_idx load of each token block it starts) and process it as one
+// unit per token block it touches.
 // Warp roles (352 threads): warp 10 loads q_idx blocks into two B buffers, up to two
 // units ahead; warp 0 streams whole k_idx tiles (one 64-dim TMA box per K sub-tile)
 // into a ring of two (D_i = 128) or four (D_i = 64) stages;
@@ -67,9 +68,9 @@ struct IndexerParams {
     uint32_t* status;      // device status word
     int t0, n_q, ld, ratio;
     int n_tb;              // token blocks of TB tokens
-    int total;             // (token block, j-tile) pairs of the launch
-    // First tile of CTA b's share: token block start_tb[b], j-tile start_jt[b].
-    uint16_t start_tb[kIndexerMaxGrid], start_jt[kIndexerMaxGrid];
+    // CTA b's share: count[b] consecutive (token block, j-tile) pairs from token block
+    // start_tb[b], j-tile start_jt[b].
+    uint16_t start_tb[kIndexerMaxGrid], start_jt[kIndexerMaxGrid], count[kIndexerMaxGrid];
 };
 
 // j-tiles (128 compressed rows each) that token block tb needs: those below n_vis of its
@@ -87,8 +88,8 @@ struct IndexerUnit {
 };
 
 // A CTA's share of the launch: `left` consecutive tiles of the list of all (token block,
-// j-tile) pairs in block order, starting at tile jt of block tb. Shares differ by at most
-// one tile; the walk cuts a share into one unit per token block it touches.
+// j-tile) pairs in block order, starting at tile jt of block tb. The walk cuts a share
+// into one unit per token block it touches.
 struct IndexerWalk {
     int tb, jt, left;
     template <int TB>
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(IndexerTile<D_I, H_I>::THREADS, 1)
 indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_q, IndexerParams p) {
     using C = IndexerTile<D_I, H_I>;
-    const int G = gridDim.x, b = blockIdx.x;
+    const int b = blockIdx.x;
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -174,10 +175,8 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_ptr;
-    // This CTA's share: tiles [b*T/G, (b+1)*T/G) of the launch's T tiles; the host found
-    // where it starts.
-    const IndexerWalk walk0{p.start_tb[b], p.start_jt[b],
-                            (int)((long long)(b + 1) * p.total / G - (long long)b * p.total / G)};
+    // This CTA's share, as the host cut it.
+    const IndexerWalk walk0{p.start_tb[b], p.start_jt[b], p.count[b]};
 
     bool abort = false;
     if (warp == C::B_WARP || warp == 0) {
