@@ -77,7 +77,9 @@ typedef struct {
 } ds4sp_config;
 
 /* Validate cfg and create a handle bound to the current CUDA device. The handle owns
- * a 4-byte device status word and some host state. *out is NULL on error. */
+ * a 4-byte device status word, the partial-result buffer of few-token attention calls
+ * (2 x SMs x 16 x 512 fp32 plus 2 x SMs x 32 fp32: about 9.7 MB on a 148-SM B200) and
+ * some host state. *out is NULL on error. */
 ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out);
 
 /* Wait for every launch this handle made (it records an event after each call), then
@@ -105,7 +107,13 @@ ds4sp_status ds4sp_indexer_topk(ds4sp_handle* h, const void* q_idx, const void* 
  *   fp16, topk [n_q, top_k] int32 as written by ds4sp_indexer_topk (entries
  *   0 .. min(k, n_vis(t))-1 hold visible rows), out [n_q, 16, 512] fp32 (output).
  * Rows are fp16; logits, softmax and accumulation are fp32; probabilities enter the
- * value product as fp16. */
+ * value product as fp16. Calls of at most 36 tokens whose tokens attend at most 64 x 32
+ * rows each, and that fit the handle's partial buffer, spread each token's rows over
+ * the GPU 32 at a time and merge the partial softmax results per token in a second
+ * kernel (each unit's O and sum rescaled to the largest reference max, added in unit
+ * order): a token's result then depends only on the token, not on the other tokens of
+ * the call. Such calls use the handle's partial buffer, so two of them must not run
+ * concurrently on one handle. */
 ds4sp_status ds4sp_sparse_attn(ds4sp_handle* h, const void* q, const void* kv_raw,
                                const void* kv_cmp, const int32_t* topk, int t0, int n_q,
                                float* out, void* stream);

@@ -66,6 +66,10 @@ struct ds4sp_handle {
     cudaStream_t copy_in = nullptr, copy_out = nullptr;
     std::vector<cudaEvent_t> band_in, band_done;
     cudaEvent_t host_start = nullptr, host_end = nullptr;
+    // Split-mode attention partials (few tokens): capacity in 32-row units.
+    int split_cap = 0;
+    float* part_o = nullptr;
+    float* part_ml = nullptr;
 };
 
 namespace {
@@ -310,14 +314,44 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
     p.n_swa = h->cfg.n_swa;
     p.ratio = h->cfg.ratio;
     p.scale_log2 = scale_of(h->cfg) * 1.4426950408889634f;
+    // Few tokens: one work item per 32-row unit, then a merge per token. The decision
+    // and each token's units depend only on the token, so a token's result is the same
+    // in every call that takes this path.
+    MergeParams mp{};
+    p.split = 0;
+    p.n_items = n_q;
+    if (n_q <= attn::SPLIT_MAX_TOKENS && h->split_cap > 0) {
+        int items = 0;
+        bool fits = true;
+        for (int i = 0; i < n_q; ++i) {
+            const int t = t0 + i, nsel = std::min(h->cfg.top_k, nvis(t, h->cfg.ratio));
+            const int nrows = nsel + (t - std::max(0, t - h->cfg.n_swa + 1) + 1);
+            const int nblk = (nrows + attn::BR - 1) / attn::BR;
+            mp.first[i] = items;
+            items += nblk;
+            fits = fits && nblk <= attn::SPLIT_MAX_UNITS;
+        }
+        mp.first[n_q] = items;
+        if (fits && items <= h->split_cap && items > n_q) {
+            p.split = 1;
+            p.n_items = items;
+            p.part_o = h->part_o;
+            p.part_ml = h->part_ml;
+            mp.part_o = h->part_o;
+            mp.part_ml = h->part_ml;
+            mp.out = out;
+            mp.n_q = n_q;
+        }
+    }
     // The region must start 16-byte aligned; its length is cut to a multiple of 16.
     const bool pf = prefetch && aligned16(prefetch) && prefetch_bytes >= 16;
     p.prefetch = pf ? static_cast<const char*>(prefetch) : nullptr;
     p.prefetch_bytes = pf ? (long long)(prefetch_bytes / 16 * 16) : 0;
     return launch(h, kAttn, stream, [&] {
-        // persistent: one CTA per SM, each walking its share of the tokens
-        const int grid = std::min(n_q, h->sm_count);
+        // persistent: one CTA per SM, each walking its share of the work items
+        const int grid = std::min(p.n_items, h->sm_count);
         sparse_attn_mma_kernel<<<grid, attn::THREADS, smem, stream>>>(p);
+        if (p.split) attn_merge_kernel<<<n_q * attn::H, 128, 0, stream>>>(mp);
     });
 }
 
@@ -431,6 +465,13 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
     if (e == cudaSuccess) e = cudaMalloc(&h->d_status, sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMemset(h->d_status, 0, sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->last, cudaEventDisableTiming);
+    // Partials of split-mode attention (calls of few tokens): two 32-row units per SM.
+    if (e == cudaSuccess) {
+        h->split_cap = 2 * h->sm_count;
+        e = cudaMalloc(&h->part_o, (size_t)h->split_cap * c.n_heads * c.d_v * sizeof(float));
+        if (e == cudaSuccess)
+            e = cudaMalloc(&h->part_ml, (size_t)h->split_cap * 2 * c.n_heads * sizeof(float));
+    }
     if (e != cudaSuccess) {
         ds4sp_destroy(h);
         return cuda_fail(e, "ds4sp_create");
@@ -462,6 +503,8 @@ ds4sp_status ds4sp_destroy(ds4sp_handle* h) {
     if (h->copy_out) cudaStreamDestroy(h->copy_out);
     if (h->last) cudaEventDestroy(h->last);
     if (h->d_status) cudaFree(h->d_status);
+    if (h->part_o) cudaFree(h->part_o);
+    if (h->part_ml) cudaFree(h->part_ml);
     delete h;
     return s;
 }

@@ -119,21 +119,47 @@ struct AttnParams {
     // slice of it, while the consumers finish. NULL or 0 bytes: nothing.
     const char* prefetch;
     long long prefetch_bytes;
+    // Split mode (few tokens): when `split` is set, a work item is one 32-row unit of a
+    // token rather than the whole token, items come in token order (the units of token
+    // 0, then token 1, ...), and each item writes its unnormalised O with its reference
+    // max and softmax sum to part_o / part_ml for attn_merge_kernel.
+    int split, n_items;
+    float* part_o;         // [n_items, 16, 512]
+    float* part_ml;        // [n_items, 2, 16]: reference max (log2 units), sum
 };
 
+// A work item: the token (i, t and its rows) and the run of its 32-row units it covers,
+// units u0 .. u0+nblk-1 (0-based) of the token's nrows rows.
 struct TokenRows {
-    int i, t, nv, nsel, s_lo, nrows, nblk;
+    int i, t, nv, nsel, s_lo, nrows, nblk, u0, item;
 };
 
-__device__ __forceinline__ TokenRows token_rows(const AttnParams& p, int idx) {
+__device__ __forceinline__ TokenRows token_rows_of(const AttnParams& p, int i) {
     TokenRows r;
-    r.i = p.n_q - 1 - idx;                        // heaviest (latest) tokens first
-    r.t = p.t0 + r.i;
+    r.i = i;
+    r.t = p.t0 + i;
     r.nv = n_vis(r.t, p.ratio);
     r.nsel = min(p.k, r.nv);
     r.s_lo = max(0, r.t - p.n_swa + 1);
     r.nrows = r.nsel + (r.t - r.s_lo + 1);
     r.nblk = (r.nrows + attn::BR - 1) / attn::BR;
+    r.u0 = 0;
+    r.item = i;
+    return r;
+}
+
+__device__ __forceinline__ TokenRows token_rows(const AttnParams& p, int idx) {
+    if (!p.split) return token_rows_of(p, p.n_q - 1 - idx);   // heaviest (latest) first
+    // Item idx is unit (idx - units of tokens before) of the token that holds it.
+    int i = 0, before = 0;
+    TokenRows r = token_rows_of(p, 0);
+    while (before + r.nblk <= idx && i + 1 < p.n_q) {
+        before += r.nblk;
+        r = token_rows_of(p, ++i);
+    }
+    r.u0 = idx - before;
+    r.nblk = 1;
+    r.item = idx;
     return r;
 }
 
@@ -147,7 +173,7 @@ struct GroupCursor {
         m = 0;
         idx = blockIdx.x + g * gridDim.x;
         u = 0;
-        valid = idx < p.n_q;
+        valid = idx < p.n_items;
         if (valid) tr = token_rows(p, idx);
     }
     __device__ __forceinline__ void advance(const AttnParams& p) {
@@ -155,7 +181,7 @@ struct GroupCursor {
             u = 0;
             ++m;
             idx += attn::GROUPS * gridDim.x;
-            valid = idx < p.n_q;
+            valid = idx < p.n_items;
             if (valid) tr = token_rows(p, idx);
         }
     }
@@ -221,7 +247,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         auto idx_buf = [&](int g, int m) { return OFF_IDX + (g * IDX_BUFS + (m & 1)) * kpad * 4; };
         auto stage_idx = [&](int g, int m) {      // top-k row of group g's m-th token
             const int idx = blockIdx.x + (g + GROUPS * m) * gridDim.x;
-            if (idx >= p.n_q) return;
+            if (idx >= p.n_items) return;
             const TokenRows nx = token_rows(p, idx);
             const int32_t* src = p.topk + (size_t)nx.i * p.k;
             const uint32_t dst = sbase + idx_buf(g, m);
@@ -266,7 +292,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
             }
             const int* tk = reinterpret_cast<const int*>(smem + idx_buf(mc.turn, cu.m));
             const int r = 8 * pw + (lane >> 2);   // this lane's row of the unit
-            const int gr = (cu.u - 1) * BR + r;
+            const int gr = (cu.tr.u0 + cu.u - 1) * BR + r;
             const __half* row = p.kv_raw + (size_t)cu.tr.t * DQK;   // valid stand-in
             bool ok = false;
             if (gr < cu.tr.nsel) {
@@ -483,6 +509,24 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                     L_g += red_sum[w * H + g];
                     L_g8 += red_sum[w * H + g + 8];
                 }
+                if (p.split) {
+                    // Unnormalised O of this unit, with the reference it is relative to.
+                    float* po = p.part_o + (size_t)cu.tr.item * H * DV;
+#pragma unroll
+                    for (int n = 0; n < 16; ++n) {
+                        const int d = 128 * gw + 8 * n + 2 * c;
+                        *reinterpret_cast<float2*>(po + g * DV + d) = make_float2(o[n][0], o[n][1]);
+                        *reinterpret_cast<float2*>(po + (g + 8) * DV + d) = make_float2(o[n][2], o[n][3]);
+                    }
+                    if (gw == 0 && c == 0) {
+                        float* ml = p.part_ml + (size_t)cu.tr.item * 2 * H;
+                        ml[g] = m_g;
+                        ml[g + 8] = m_g8;
+                        ml[H + g] = L_g;
+                        ml[H + g + 8] = L_g8;
+                    }
+                    continue;
+                }
                 const float inv_g = L_g > 0.f ? 1.f / L_g : 0.f;
                 const float inv_g8 = L_g8 > 0.f ? 1.f / L_g8 : 0.f;
                 float* ot = p.out + (size_t)cu.tr.i * H * DV;
@@ -498,6 +542,68 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         }
     }
     __syncthreads();
+}
+
+// Split mode, second step: token i's output from its units' partial results (items
+// first .. first+cnt-1): with M = the largest reference of a head, each unit's O and
+// sum are scaled by 2^(m - M) before they are added; O / sum is the token's output.
+// The units are added in order, so the result does not depend on how many tokens the
+// call held. One CTA of 128 threads per (token, head), four value dims per thread.
+namespace attn {
+constexpr int SPLIT_MAX_TOKENS = 36;          // split mode: at most this many tokens,
+constexpr int SPLIT_MAX_UNITS = 64;           // each with at most this many 32-row units
+}  // namespace attn
+
+struct MergeParams {
+    const float* part_o;
+    const float* part_ml;
+    float* out;
+    int n_q;
+    int first[attn::SPLIT_MAX_TOKENS + 1];      // token i's items: first[i] .. first[i+1]-1
+};
+
+__global__ void __launch_bounds__(128) attn_merge_kernel(const MergeParams mp) {
+    using namespace attn;
+    __shared__ float wgt[SPLIT_MAX_UNITS];      // per unit: 2^(m - M) / L for this head
+    __shared__ float red[2][4];
+    const int i = blockIdx.x / H, h = blockIdx.x % H;
+    if (i >= mp.n_q) return;
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    const int first = mp.first[i], cnt = min(mp.first[i + 1] - first, SPLIT_MAX_UNITS);
+    // Largest reference of the head over the units (threads 0 .. cnt-1 hold one each).
+    const float m = tid < cnt ? mp.part_ml[(size_t)(first + tid) * 2 * H + h] : -INFINITY;
+    float mx = m;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) red[0][warp] = mx;
+    __syncthreads();
+    const float M = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
+    const float Mr = M == -INFINITY ? 0.f : M;
+    const float a = tid < cnt ? exp2f(m - Mr) : 0.f;
+    float l = tid < cnt ? mp.part_ml[(size_t)(first + tid) * 2 * H + H + h] * a : 0.f;
+    // Sum of the scaled unit sums in unit order: gather them, then one thread adds.
+    if (tid < cnt) wgt[tid] = l;
+    __syncthreads();
+    if (tid == 0) {
+        float L = 0.f;
+        for (int s2 = 0; s2 < cnt; ++s2) L += wgt[s2];
+        red[1][0] = L > 0.f ? 1.f / L : 0.f;
+    }
+    __syncthreads();
+    if (tid < cnt) wgt[tid] = a * red[1][0];
+    __syncthreads();
+    const float* src = mp.part_o + (size_t)first * H * DV + h * DV + 4 * tid;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int s2 = 0; s2 < cnt; ++s2) {
+        const float4 v = *reinterpret_cast<const float4*>(src + (size_t)s2 * H * DV);
+        const float w = wgt[s2];
+        acc.x += v.x * w;
+        acc.y += v.y * w;
+        acc.z += v.z * w;
+        acc.w += v.w * w;
+    }
+    *reinterpret_cast<float4*>(mp.out + ((size_t)i * H + h) * DV + 4 * tid) = acc;
 }
 
 }  // namespace ds4sp
