@@ -212,6 +212,49 @@ def config_name(wl):
 
 # ------------------------------------------------------------------ our arm
 
+def verify_latency(dev, reps: int = 50):
+    """Latency of one verify step per width q: ds4sp_indexer_topk + ds4sp_sparse_attn on
+    the last q tokens of the 122,880-token verify workload (q = 1..5), device-resident
+    inputs, CUDA events around `reps` back-to-back steps."""
+    wl = workload("verify")
+    d = {k: v.to(dev) for k, v in generate(wl).items()}
+    T = wl.T
+    cfg = D.make_config(n_idx_heads=wl.H_i, d_idx=wl.D_i, top_k=wl.top_k, n_swa=wl.n_swa,
+                        max_tokens=T, band=wl.band)
+    h = D.ds4sp_create(cfg)
+    res = {}
+    try:
+        for q in range(1, 6):
+            sl = {k: (v[5 - q:].contiguous() if k in ("q", "q_idx", "w") else v) for k, v in d.items()}
+            topk = torch.empty((q, wl.top_k), dtype=torch.int32, device=dev)
+            out = torch.empty((q, 16, 512), dtype=torch.float32, device=dev)
+            ws = torch.empty(max(D.ds4sp_workspace_bytes(h, T - q, q), 256), dtype=torch.uint8,
+                             device=dev)
+
+            def call():
+                D.ds4sp_indexer_topk(h, sl["q_idx"], sl["k_idx"], sl["w"], T - q, q, topk, ws)
+                D.ds4sp_sparse_attn(h, sl["q"], sl["kv_raw"], sl["kv_cmp"], topk, T - q, q, out)
+
+            for _ in range(5):
+                call()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                call()
+            e1.record()
+            torch.cuda.synchronize()
+            res[f"q{q}"] = round(e0.elapsed_time(e1) / reps * 1e3, 1)
+        st, bits = D.ds4sp_device_status(h)
+        if st != D.OK:
+            raise RuntimeError(f"device status {bits:#x} after verify timing")
+    finally:
+        D.ds4sp_destroy(h)
+    return {"workload": "verify: 122,880-token context, the last q = 1..5 tokens, top_k 512, "
+                        "n_swa 128, indexer 64x128, seed 4",
+            "unit": "us per step (indexer + top-k + attention)", **res}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
     torch.cuda.set_device(local_rank)
@@ -284,6 +327,10 @@ def run_ours(args, rank, world, local_rank):
     if st != D.OK:
         raise RuntimeError(f"device status {bits:#x} after timing")
 
+    verify = None
+    if rank == 0 and world == 1 and not args.no_verify:
+        verify = verify_latency(dev)
+
     cpu_base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu_base = cpu_oracle_sample(wl, args.cpu_sample, {k: v.numpy() for k, v in host.items()})
@@ -320,6 +367,7 @@ def run_ours(args, rank, world, local_rank):
                          "alg_GBps": alg["topk_bytes"] * steps / (topk_ms / 1e3) / 1e9},
             },
             "gpu_launches": attn_n + idx_n + topk_n,
+            "verify": verify,
             "e2e": {"value": job_throughput(wl.T, world, e2e_steps, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "clocks": clk,
@@ -337,6 +385,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-sample", type=int, default=8192)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-verify", action="store_true",
+                    help="skip the few-token latency of the 122,880-token verify workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
