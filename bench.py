@@ -331,6 +331,29 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_verify:
         verify = verify_latency(dev)
 
+    # The same step with CUDA's exp2f for the softmax exponentials (exp_mode 1), for the
+    # fast-versus-precise comparison; not the headline.
+    variants = None
+    if rank == 0 and world == 1 and not args.no_verify:
+        cfg_p = D.make_config(n_idx_heads=wl.H_i, d_idx=wl.D_i, top_k=wl.top_k, n_swa=wl.n_swa,
+                              max_tokens=wl.T, band=wl.band, exp_mode=1)
+        hp = D.ds4sp_create(cfg_p)
+        try:
+            for _ in range(3):
+                D.prefill(hp, inputs, wl.T, topk, out, ws, stream)
+            torch.cuda.synchronize()
+            D.ds4sp_profile_enable(hp, True)
+            D.ds4sp_profile_read(hp)
+            n_var = 20
+            for _ in range(n_var):
+                D.prefill(hp, inputs, wl.T, topk, out, ws, stream)
+            torch.cuda.synchronize()
+            pv = D.ds4sp_profile_read(hp)
+            variants = {"exp2f_softmax": {"attention_ms_per_step": pv["attention"][0] / n_var,
+                                          "steps": n_var}}
+        finally:
+            D.ds4sp_destroy(hp)
+
     cpu_base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu_base = cpu_oracle_sample(wl, args.cpu_sample, {k: v.numpy() for k, v in host.items()})
@@ -368,6 +391,7 @@ def run_ours(args, rank, world, local_rank):
             },
             "gpu_launches": attn_n + idx_n + topk_n,
             "verify": verify,
+            "variants": variants,
             "e2e": {"value": job_throughput(wl.T, world, e2e_steps, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "clocks": clk,

@@ -74,6 +74,9 @@ typedef struct {
     int band;            /* tokens per band (2048) */
     int max_tokens;      /* sequence length T the KV buffers hold */
     float softmax_scale; /* <= 0 selects 1/sqrt(d_qk) */
+    int exp_mode;        /* softmax exponentials: 0 = ex2.approx (default, about 2^-22
+                            relative error), 1 = exp2f (CUDA's precise function); other
+                            values are DS4SP_ERR_INVALID_ARG */
 } ds4sp_config;
 
 /* Validate cfg and create a handle bound to the current CUDA device. The handle owns

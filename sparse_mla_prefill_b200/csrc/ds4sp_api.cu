@@ -289,16 +289,20 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
                          const void* prefetch = nullptr, size_t prefetch_bytes = 0) {
     const int smem = attn::smem_bytes(h->cfg.top_k);
     if (!h->smem_set[kAttn]) {
-        const cudaError_t e = cudaFuncSetAttribute(sparse_attn_mma_kernel,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   attn::smem_bytes(attn::MAX_TOPK));
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention)");
-        cudaFuncAttributes fa;
-        const cudaError_t ea = cudaFuncGetAttributes(&fa, sparse_attn_mma_kernel);
-        if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncGetAttributes(attention)");
-        if (fa.numRegs != attn::LAUNCH_REGS)   // the warp roles' register split assumes it
-            return fail(DS4SP_ERR_UNSUPPORTED, "attention kernel built with %d registers, not %d",
-                        fa.numRegs, attn::LAUNCH_REGS);
+        // Both instantiations (fast and precise exponentials), once per handle.
+        for (int mode = 0; mode < 2; ++mode) {
+            const void* fn = mode ? reinterpret_cast<const void*>(sparse_attn_mma_kernel<true>)
+                                  : reinterpret_cast<const void*>(sparse_attn_mma_kernel<false>);
+            const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       attn::smem_bytes(attn::MAX_TOPK));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention)");
+            cudaFuncAttributes fa;
+            const cudaError_t ea = cudaFuncGetAttributes(&fa, fn);
+            if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncGetAttributes(attention)");
+            if (fa.numRegs != attn::LAUNCH_REGS)   // the warp roles' register split assumes it
+                return fail(DS4SP_ERR_UNSUPPORTED, "attention kernel built with %d registers, not %d",
+                            fa.numRegs, attn::LAUNCH_REGS);
+        }
         h->smem_set[kAttn] = true;
     }
     AttnParams p;
@@ -350,7 +354,10 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
     return launch(h, kAttn, stream, [&] {
         // persistent: one CTA per SM, each walking its share of the work items
         const int grid = std::min(p.n_items, h->sm_count);
-        sparse_attn_mma_kernel<<<grid, attn::THREADS, smem, stream>>>(p);
+        if (h->cfg.exp_mode)
+            sparse_attn_mma_kernel<true><<<grid, attn::THREADS, smem, stream>>>(p);
+        else
+            sparse_attn_mma_kernel<false><<<grid, attn::THREADS, smem, stream>>>(p);
         if (p.split) attn_merge_kernel<<<n_q * attn::H, 128, 0, stream>>>(mp);
     });
 }
@@ -456,6 +463,8 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
         !(c.softmax_scale == c.softmax_scale))
         return fail(DS4SP_ERR_INVALID_ARG, "top_k >= 0, n_swa >= 1, band >= 1, "
                                            "1 <= max_tokens <= 2^24 and a finite scale required");
+    if (c.exp_mode != 0 && c.exp_mode != 1)
+        return fail(DS4SP_ERR_INVALID_ARG, "exp_mode %d (0 = ex2.approx, 1 = exp2f)", c.exp_mode);
     ds4sp_handle* h = new (std::nothrow) ds4sp_handle();
     if (!h) return fail(DS4SP_ERR_INVALID_ARG, "out of host memory");
     h->cfg = c;

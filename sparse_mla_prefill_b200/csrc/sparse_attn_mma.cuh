@@ -32,7 +32,8 @@
 //     value dims 128w .. 128w+127.
 // Rows are stored unpadded with their 16-byte chunks XOR-swizzled, which keeps the
 // producers' copies and the consumers' ldmatrix reads free of bank conflicts.
-// fp32 logits, sums and output; P enters P . V as fp16; exponentials on ex2.approx.
+// fp32 logits, sums and output; P enters P . V as fp16; exponentials on ex2.approx
+// (or exp2f in the precise instantiation).
 // Every wait is bounded; a consumer that gives up sets its group's flag, which the
 // group's warps read after their next barrier, so none is left waiting.
 #pragma once
@@ -215,8 +216,11 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// PRECISE selects exp2f for the softmax exponentials instead of ex2.approx.
+template <bool PRECISE>
 __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnParams p) {
     using namespace attn;
+    auto exp2_ = [](float x) { return PRECISE ? exp2f(x) : fast_exp2(x); };
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -427,7 +431,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                 const float rg = ref_g == -INFINITY ? 0.f : ref_g;
                 const float rg8 = ref_g8 == -INFINITY ? 0.f : ref_g8;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) s4[e] = fast_exp2(s4[e] - (e < 2 ? rg : rg8));
+                for (int e = 0; e < 4; ++e) s4[e] = exp2_(s4[e] - (e < 2 ? rg : rg8));
             }
             uint8_t* pb = garea + G_P + r0 * 2;
             *reinterpret_cast<uint32_t*>(pb + g * P_PITCH) = pack_half2(s4[0], s4[1]);
@@ -449,7 +453,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                     M_g8 = fmaxf(M_g8, ref_tile[t * H + g + 8]);
                 }
                 const float Mg = M_g == -INFINITY ? 0.f : M_g, Mg8 = M_g8 == -INFINITY ? 0.f : M_g8;
-                const float alpha_g = fast_exp2(m_g - Mg), alpha_g8 = fast_exp2(m_g8 - Mg8);
+                const float alpha_g = exp2_(m_g - Mg), alpha_g8 = exp2_(m_g8 - Mg8);
 #pragma unroll
                 for (int n = 0; n < 16; ++n) {
                     o[n][0] *= alpha_g;
@@ -461,7 +465,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                 l_g8 *= alpha_g8;
                 const float rg = ref_g == -INFINITY ? 0.f : ref_g;
                 const float rg8 = ref_g8 == -INFINITY ? 0.f : ref_g8;
-                const float beta_g = fast_exp2(rg - Mg), beta_g8 = fast_exp2(rg8 - Mg8);
+                const float beta_g = exp2_(rg - Mg), beta_g8 = exp2_(rg8 - Mg8);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) s4[e] *= e < 2 ? beta_g : beta_g8;
                 *reinterpret_cast<uint32_t*>(pb + g * P_PITCH) = pack_half2(s4[0], s4[1]);

@@ -31,7 +31,8 @@ class ds4sp_config(ctypes.Structure):
     _fields_ = [("n_heads", ctypes.c_int), ("d_qk", ctypes.c_int), ("d_v", ctypes.c_int),
                 ("ratio", ctypes.c_int), ("n_idx_heads", ctypes.c_int), ("d_idx", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("n_swa", ctypes.c_int), ("band", ctypes.c_int),
-                ("max_tokens", ctypes.c_int), ("softmax_scale", ctypes.c_float)]
+                ("max_tokens", ctypes.c_int), ("softmax_scale", ctypes.c_float),
+                ("exp_mode", ctypes.c_int)]
 
 
 class ds4sp_io(ctypes.Structure):
@@ -139,9 +140,9 @@ class Handle:
 
 def make_config(n_idx_heads: int, d_idx: int, top_k: int, n_swa: int, max_tokens: int,
                 band: int = 2048, softmax_scale: float = 0.0, n_heads: int = 16, d_qk: int = 576,
-                d_v: int = 512, ratio: int = 4) -> ds4sp_config:
+                d_v: int = 512, ratio: int = 4, exp_mode: int = 0) -> ds4sp_config:
     return ds4sp_config(n_heads, d_qk, d_v, ratio, n_idx_heads, d_idx, top_k, n_swa, band,
-                        max_tokens, softmax_scale)
+                        max_tokens, softmax_scale, exp_mode)
 
 
 def ds4sp_create(cfg: ds4sp_config) -> Handle:

@@ -55,6 +55,7 @@ def _cfg(**kw):
     (dict(max_tokens=0), D.ERR_INVALID_ARG),
     (dict(max_tokens=(1 << 24) + 1), D.ERR_INVALID_ARG),
     (dict(softmax_scale=float("nan")), D.ERR_INVALID_ARG),
+    (dict(exp_mode=2), D.ERR_INVALID_ARG),
 ])
 def test_create_rejects_bad_config_before_touching_the_device(lib, kw, status):
     out = ctypes.c_void_p(123)
