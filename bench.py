@@ -47,7 +47,9 @@ def attn_rows(T, k, n_swa, t0=0, t1=None):
 
 
 def algorithmic(wl):
-    """Per-step algorithmic bytes / FLOPs of each kernel (per-unit figures in the design doc)."""
+    """Per-step algorithmic bytes / FLOPs of each kernel: attention 1152 B per (token,
+    attended row) plus Q, O and index bytes per token; indexer 2*H_i*D_i FLOPs per (token,
+    visible row); top-k 4 B per (token, visible row) read plus 4*k B per token written."""
     T, k, n_swa = wl.T, wl.top_k, wl.n_swa
     rows = attn_rows(T, k, n_swa)
     sum_vis = sum(n_vis(t) for t in range(T))

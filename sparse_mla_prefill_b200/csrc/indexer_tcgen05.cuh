@@ -19,9 +19,9 @@
 // units ahead; warp 0 streams whole k_idx tiles (one 64-dim TMA box per K sub-tile)
 // into a ring of two (D_i = 128) or four (D_i = 64) stages;
 // warp 1 owns TMEM and issues the MMAs; warps 2-9 run the epilogue (ReLU, head
-// weights, sum, store), two
-// warps per TMEM lane quarter, each on half of the columns. Two TMEM accumulators
-// (2 x 256 columns) let the epilogue of tile i overlap the MMAs of tile i+1.
+// weights, sum, store), two warps per TMEM lane quarter, each on half of the columns.
+// Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i overlap the MMAs
+// of tile i+1.
 // Every wait is bounded (device_common.cuh).
 #pragma once
 
