@@ -22,6 +22,9 @@ or reordering. A reader can check each function against its definition:
   order"). Keep the min(k, n_vis(t)) largest scores among visible rows; equal
   scores go to the lower j; the kept rows are listed in ascending j, and unused
   slots hold -1.
+* Explicit-mask top-k -- same page, Qualification ("explicit-mask versus
+  analytic-mask" oracle): the same selection with the candidates read from a
+  stored mask row instead of the formula (``topk_row_masked``).
 * Attention -- same page, Summary ("keep selected raw/compressed KV transport in
   F16, and stream each selected latent row once across sixteen ... heads").
   One 576-wide latent row per position serves as key (all 576 dims) and value
@@ -151,6 +154,30 @@ def topk_row(scores: np.ndarray, k: int) -> np.ndarray:
 def topk(scores: Sequence[np.ndarray], k: int) -> np.ndarray:
     """Stack ``topk_row`` over tokens: [n_q, k] int32."""
     return np.stack([topk_row(s, k) for s in scores]) if len(scores) else np.zeros((0, k), np.int32)
+
+
+def topk_row_masked(scores: np.ndarray, visible: np.ndarray, k: int) -> np.ndarray:
+    """Top-k of one token when visibility comes from a stored mask row, not the formula.
+
+    The explicit-mask form of the selection ("perf(ds4): extend sparse prefill
+    scheduling to 10K", Qualification: "explicit-mask versus analytic-mask"):
+    the candidates are the j with visible[j] set; among them the same order as
+    ``topk_row`` applies (score descending, then j ascending), the first
+    min(k, #candidates) are kept and listed by ascending j, -1 padded to k.
+    ``scores`` must cover every visible j (visible rows past its end raise).
+    """
+    visible = np.asarray(visible, dtype=bool)
+    cand = np.flatnonzero(visible)
+    if len(cand) and cand[-1] >= len(scores):
+        raise ValueError("a visible row has no score")
+    out = np.full(k, -1, dtype=np.int32)
+    m = min(k, len(cand))
+    if m == 0:
+        return out
+    s = np.asarray(scores, dtype=np.float64)[cand]
+    order = np.lexsort((cand, -s))                      # last key is primary
+    out[:m] = np.sort(cand[order[:m]])
+    return out
 
 
 # --------------------------------------------------------------------------

@@ -153,6 +153,32 @@ def pin_topk_bruteforce(o, trials: int = 300, seed: int = 3):
                 assert sel[scores[sel] == thr].max() < rest[scores[rest] == thr].min()
 
 
+def pin_topk_masked_bruteforce(o, trials: int = 300, seed: int = 4):
+    """Explicit-mask selection: brute force over the mask's candidates, hidden rows never
+    kept, and the formula's own mask row gives the prefix selection."""
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        n = int(rng.integers(0, 70))
+        k = int(rng.integers(0, 40))
+        scores = rng.integers(-3, 6, n).astype(np.float64) * float(rng.choice([1.0, 0.5, 1e3]))
+        vis = rng.random(n + int(rng.integers(0, 4))) < rng.choice([0.2, 0.6, 1.0])
+        vis[n:] = False                            # rows past the scores are never visible
+        got = o.topk_row_masked(scores, vis, k)
+        cand = [j for j in range(n) if vis[j]]
+        want = sorted(sorted(cand, key=lambda j: (-scores[j], j))[:min(k, len(cand))])
+        assert got.dtype == np.int32 and got.shape == (k,)
+        assert got.tolist() == want + [-1] * (k - len(want)), (scores.tolist(), vis.tolist(), k)
+        assert all(vis[j] for j in got if j >= 0)
+    # The ratio-4 mask row of token t (rows 4j+3 <= t) reduces to the prefix selection.
+    scores = rng.integers(0, 4, 40).astype(np.float64)
+    for t in (0, 3, 17, 90, 170):
+        row = np.array([4 * j + 3 <= t for j in range(40)])
+        nv = int(row.sum())
+        got = o.topk_row_masked(scores, row, 8).tolist()
+        want = sorted(sorted(range(nv), key=lambda j: (-scores[j], j))[:min(8, nv)])
+        assert got == want + [-1] * (8 - len(want)), (t, got)
+
+
 # ------------------------------------------------------------------ attention
 
 def _attn_case(T=48, n_c=None, seed=21):
@@ -269,7 +295,7 @@ def pin_bands_equal_oneshot(o):
 ALL_PINS = [
     pin_visibility_mask, pin_visibility_golden,
     pin_scores_exact, pin_scores_relu_identities, pin_scores_bruteforce,
-    pin_topk_golden, pin_topk_bruteforce,
+    pin_topk_golden, pin_topk_bruteforce, pin_topk_masked_bruteforce,
     pin_attention_sdpa_causal, pin_attention_sdpa_window, pin_attention_dense_mask,
     pin_attention_bruteforce, pin_attention_closed_forms,
     pin_bands_equal_oneshot,

@@ -95,6 +95,23 @@ def _mut_dedup_window(o):
     o.attended_rows = f
 
 
+def _mut_masked_ignores_mask(o):
+    o.topk_row_masked = lambda scores, visible, k: o.topk_row(scores, k)
+
+
+def _mut_masked_ties_by_candidate_rank(o):
+    # Breaks ties by the position in the candidate list reversed (a higher j first).
+    def f(scores, visible, k):
+        cand = np.flatnonzero(np.asarray(visible, bool))
+        out = np.full(k, -1, dtype=np.int32)
+        m = min(k, len(cand))
+        if m:
+            order = np.lexsort((-cand, -np.asarray(scores, float)[cand]))
+            out[:m] = np.sort(cand[order[:m]])
+        return out
+    o.topk_row_masked = f
+
+
 MUTATIONS = [
     (_mut_visibility_first_token, [P.pin_visibility_mask, P.pin_visibility_golden]),
     (_mut_no_relu, [P.pin_scores_exact, P.pin_scores_relu_identities, P.pin_scores_bruteforce]),
@@ -102,6 +119,8 @@ MUTATIONS = [
     (_mut_unweighted_heads, [P.pin_scores_relu_identities, P.pin_scores_bruteforce]),
     (_mut_ties_to_higher_j, [P.pin_topk_golden, P.pin_topk_bruteforce]),
     (_mut_score_order_listing, [P.pin_topk_golden, P.pin_topk_bruteforce]),
+    (_mut_masked_ignores_mask, [P.pin_topk_masked_bruteforce]),
+    (_mut_masked_ties_by_candidate_rank, [P.pin_topk_masked_bruteforce]),
     (_mut_value_last_dims, [P.pin_attention_sdpa_causal, P.pin_attention_closed_forms]),
     (_mut_window_excludes_self, [P.pin_attention_sdpa_causal, P.pin_attention_sdpa_window]),
     (_mut_scale_ignored, [P.pin_attention_sdpa_causal, P.pin_attention_bruteforce]),
