@@ -333,28 +333,33 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_verify:
         verify = verify_latency(dev)
 
-    # The same step with CUDA's exp2f for the softmax exponentials (exp_mode 1), for the
-    # fast-versus-precise comparison; not the headline.
+    # The same step with CUDA's exp2f for the softmax exponentials (exp_mode 1), and with
+    # fp32-staged probabilities in P . V (pv_mode 1, fast and precise exponentials), for
+    # the fast-versus-precise and fp16-versus-fp32-staged comparisons; not the headline.
     variants = None
     if rank == 0 and world == 1 and not args.no_verify:
-        cfg_p = D.make_config(n_idx_heads=wl.H_i, d_idx=wl.D_i, top_k=wl.top_k, n_swa=wl.n_swa,
-                              max_tokens=wl.T, band=wl.band, exp_mode=1)
-        hp = D.ds4sp_create(cfg_p)
-        try:
-            for _ in range(3):
-                D.prefill(hp, inputs, wl.T, topk, out, ws, stream)
-            torch.cuda.synchronize()
-            D.ds4sp_profile_enable(hp, True)
-            D.ds4sp_profile_read(hp)
-            n_var = 20
-            for _ in range(n_var):
-                D.prefill(hp, inputs, wl.T, topk, out, ws, stream)
-            torch.cuda.synchronize()
-            pv = D.ds4sp_profile_read(hp)
-            variants = {"exp2f_softmax": {"attention_ms_per_step": pv["attention"][0] / n_var,
-                                          "steps": n_var}}
-        finally:
-            D.ds4sp_destroy(hp)
+        variants = {}
+        for name, modes in (("exp2f_softmax", dict(exp_mode=1)),
+                            ("fp32_staged_pv", dict(pv_mode=1)),
+                            ("fp32_staged_pv_exp2f", dict(pv_mode=1, exp_mode=1))):
+            cfg_v = D.make_config(n_idx_heads=wl.H_i, d_idx=wl.D_i, top_k=wl.top_k,
+                                  n_swa=wl.n_swa, max_tokens=wl.T, band=wl.band, **modes)
+            hv = D.ds4sp_create(cfg_v)
+            try:
+                for _ in range(3):
+                    D.prefill(hv, inputs, wl.T, topk, out, ws, stream)
+                torch.cuda.synchronize()
+                D.ds4sp_profile_enable(hv, True)
+                D.ds4sp_profile_read(hv)
+                n_var = 20
+                for _ in range(n_var):
+                    D.prefill(hv, inputs, wl.T, topk, out, ws, stream)
+                torch.cuda.synchronize()
+                vprof = D.ds4sp_profile_read(hv)
+                variants[name] = {"attention_ms_per_step": vprof["attention"][0] / n_var,
+                                  "steps": n_var, **modes}
+            finally:
+                D.ds4sp_destroy(hv)
 
     cpu_base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -77,6 +77,12 @@ typedef struct {
     int exp_mode;        /* softmax exponentials: 0 = ex2.approx (default, about 2^-22
                             relative error), 1 = exp2f (CUDA's precise function); other
                             values are DS4SP_ERR_INVALID_ARG */
+    int pv_mode;         /* probabilities entering P . V: 0 = one fp16 term (default),
+                            1 = fp32-staged: P = hi + lo, two fp16 terms (hi = fp16(p),
+                            lo = fp16(p - hi)), about 22 significant bits, at twice the
+                            P . V tensor work ("FP32-staged streaming MLA" of "perf(ds4):
+                            extend sparse prefill scheduling to 10K"); other values are
+                            DS4SP_ERR_INVALID_ARG */
 } ds4sp_config;
 
 /* Validate cfg and create a handle bound to the current CUDA device. The handle owns
@@ -190,6 +196,27 @@ ds4sp_status ds4sp_profile_read(ds4sp_handle* h, double ms[3], int launches[3]);
 /* Host-side fault injection for tests: the next n kernel launches of this handle are
  * not made, and the call that would make them returns DS4SP_ERR_CUDA. */
 ds4sp_status ds4sp_debug_fail_launches(ds4sp_handle* h, int n);
+
+/* Explicit-mask visibility, a debug form of the path for the "explicit-mask versus
+ * analytic-mask" oracle check ("perf(ds4): extend sparse prefill scheduling to 10K",
+ * Qualification). While a mask is set, the top-k and the attention take the visibility
+ * of compressed rows from it instead of the ratio-4 formula:
+ *   mask  device pointer, uint8 [rows, cols], row-major, caller-owned; mask[t*cols + j]
+ *         != 0 means compressed row j is visible to absolute token t. It must stay valid
+ *         until the calls that use it have completed.
+ *   top-k      the candidates of token t are the j < min(cols, n_vis(t_last)) whose byte
+ *              is set (t_last = the call's last token); fewer than k: all of them,
+ *              ascending, then -1.
+ *   attention  a top-k entry j is attended iff 0 <= j < min(cols, n_vis(t_last)) and
+ *              its byte is set; -1 entries and hidden rows are dropped silently; other
+ *              out-of-range entries set the status word's index bit.
+ * The indexer, the window of raw rows and the work partition are unchanged; the score
+ * columns j >= n_vis(t) are not computed, so a mask that shows such a row selects on an
+ * undefined score (the check then fails, which is its purpose). With the mask that the
+ * formula defines, every output is bit-identical to the analytic path.
+ * mask = NULL clears it (rows and cols are then ignored). Calls whose tokens reach past
+ * `rows` return DS4SP_ERR_INVALID_ARG before any launch. rows, cols >= 1 otherwise. */
+ds4sp_status ds4sp_debug_set_mask(ds4sp_handle* h, const uint8_t* mask, int rows, int cols);
 
 /* Steps 1-2 like ds4sp_indexer_topk, for callers that cannot allocate device memory.
  * The paper has no counterpart to this entry point; it exists for the host side only.

@@ -70,6 +70,9 @@ struct ds4sp_handle {
     int split_cap = 0;
     float* part_o = nullptr;
     float* part_ml = nullptr;
+    // ds4sp_debug_set_mask: explicit visibility mask [mask_rows, mask_cols], or NULL.
+    const uint8_t* mask = nullptr;
+    int mask_rows = 0, mask_cols = 0;
 };
 
 namespace {
@@ -262,7 +265,11 @@ ds4sp_status dispatch_indexer_h(ds4sp_handle* h, const void* q_idx, const void* 
 
 ds4sp_status launch_topk(ds4sp_handle* h, const float* scores, int ld, int t0, int n_q,
                          int32_t* topk, cudaStream_t stream) {
-    const size_t smem = (size_t)ld * 4;
+    const int k = h->cfg.top_k, ratio = h->cfg.ratio;
+    // Explicit-mask form: candidates only among the columns this call's scores cover.
+    const int mcols = h->mask ? std::min(h->mask_cols, nvis(t0 + n_q - 1, ratio)) : 0;
+    const uint8_t* vm = h->mask;
+    const long long mld = h->mask_cols;
     const bool big = ld > 4096;
     if (!h->smem_set[kTopk]) {
         cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel<256>,
@@ -275,12 +282,14 @@ ds4sp_status launch_topk(ds4sp_handle* h, const float* scores, int ld, int t0, i
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(topk)");
         h->smem_set[kTopk] = true;
     }
-    const int k = h->cfg.top_k, ratio = h->cfg.ratio;
+    const size_t smem = (size_t)ld * 4;
     return launch(h, kTopk, stream, [&] {
         if (big)
-            topk_radix_kernel<1024><<<n_q, 1024, smem, stream>>>(scores, ld, t0, n_q, k, ratio, topk);
+            topk_radix_kernel<1024><<<n_q, 1024, smem, stream>>>(scores, ld, t0, n_q, k, ratio,
+                                                                 vm, mld, mcols, topk);
         else
-            topk_radix_kernel<256><<<n_q, 256, smem, stream>>>(scores, ld, t0, n_q, k, ratio, topk);
+            topk_radix_kernel<256><<<n_q, 256, smem, stream>>>(scores, ld, t0, n_q, k, ratio,
+                                                               vm, mld, mcols, topk);
     });
 }
 
@@ -289,10 +298,13 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
                          const void* prefetch = nullptr, size_t prefetch_bytes = 0) {
     const int smem = attn::smem_bytes(h->cfg.top_k);
     if (!h->smem_set[kAttn]) {
-        // Both instantiations (fast and precise exponentials), once per handle.
-        for (int mode = 0; mode < 2; ++mode) {
-            const void* fn = mode ? reinterpret_cast<const void*>(sparse_attn_mma_kernel<true>)
-                                  : reinterpret_cast<const void*>(sparse_attn_mma_kernel<false>);
+        // Every instantiation (fast or precise exponentials x fp16 or fp32-staged P),
+        // once per handle.
+        const void* fns[4] = {reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false>),
+                              reinterpret_cast<const void*>(sparse_attn_mma_kernel<true, false>),
+                              reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, true>),
+                              reinterpret_cast<const void*>(sparse_attn_mma_kernel<true, true>)};
+        for (const void* fn : fns) {
             const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                        attn::smem_bytes(attn::MAX_TOPK));
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention)");
@@ -318,6 +330,10 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
     p.n_swa = h->cfg.n_swa;
     p.ratio = h->cfg.ratio;
     p.scale_log2 = scale_of(h->cfg) * 1.4426950408889634f;
+    // Explicit-mask form: entries only among the compressed rows this call may read.
+    p.vis_mask = h->mask;
+    p.mask_ld = h->mask_cols;
+    p.mask_cols = h->mask ? std::min(h->mask_cols, nvis(t0 + n_q - 1, h->cfg.ratio)) : 0;
     // Few tokens: one work item per 32-row unit, then a merge per token. The decision
     // and each token's units depend only on the token, so a token's result is the same
     // in every call that takes this path.
@@ -354,10 +370,13 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
     return launch(h, kAttn, stream, [&] {
         // persistent: one CTA per SM, each walking its share of the work items
         const int grid = std::min(p.n_items, h->sm_count);
-        if (h->cfg.exp_mode)
-            sparse_attn_mma_kernel<true><<<grid, attn::THREADS, smem, stream>>>(p);
-        else
-            sparse_attn_mma_kernel<false><<<grid, attn::THREADS, smem, stream>>>(p);
+        const dim3 g(grid), b(attn::THREADS);
+        switch (2 * h->cfg.pv_mode + h->cfg.exp_mode) {
+            case 0: sparse_attn_mma_kernel<false, false><<<g, b, smem, stream>>>(p); break;
+            case 1: sparse_attn_mma_kernel<true, false><<<g, b, smem, stream>>>(p); break;
+            case 2: sparse_attn_mma_kernel<false, true><<<g, b, smem, stream>>>(p); break;
+            default: sparse_attn_mma_kernel<true, true><<<g, b, smem, stream>>>(p); break;
+        }
         if (p.split) attn_merge_kernel<<<n_q * attn::H, 128, 0, stream>>>(mp);
     });
 }
@@ -371,6 +390,9 @@ ds4sp_status check_range(const ds4sp_handle* h, int t0, int n_q) {
     if (t0 < 0 || n_q < 0 || (long long)t0 + n_q > h->cfg.max_tokens)
         return fail(DS4SP_ERR_INVALID_ARG, "token range [%d, %d+%d) outside [0, %d)", t0, t0, n_q,
                     h->cfg.max_tokens);
+    if (h->mask && (long long)t0 + n_q > h->mask_rows)
+        return fail(DS4SP_ERR_INVALID_ARG, "token range [%d, %d+%d) outside the mask's %d rows",
+                    t0, t0, n_q, h->mask_rows);
     return DS4SP_OK;
 }
 
@@ -465,6 +487,8 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
                                            "1 <= max_tokens <= 2^24 and a finite scale required");
     if (c.exp_mode != 0 && c.exp_mode != 1)
         return fail(DS4SP_ERR_INVALID_ARG, "exp_mode %d (0 = ex2.approx, 1 = exp2f)", c.exp_mode);
+    if (c.pv_mode != 0 && c.pv_mode != 1)
+        return fail(DS4SP_ERR_INVALID_ARG, "pv_mode %d (0 = fp16 P, 1 = fp32-staged P)", c.pv_mode);
     ds4sp_handle* h = new (std::nothrow) ds4sp_handle();
     if (!h) return fail(DS4SP_ERR_INVALID_ARG, "out of host memory");
     h->cfg = c;
@@ -755,6 +779,20 @@ ds4sp_status ds4sp_debug_fail_launches(ds4sp_handle* h, int n) {
     DS4SP_TRY(check_handle(h));
     if (n < 0) return fail(DS4SP_ERR_INVALID_ARG, "n < 0");
     h->fail_launches = n;
+    return DS4SP_OK;
+}
+
+ds4sp_status ds4sp_debug_set_mask(ds4sp_handle* h, const uint8_t* mask, int rows, int cols) {
+    DS4SP_TRY(check_handle(h));
+    if (mask == nullptr) {
+        h->mask = nullptr;
+        h->mask_rows = h->mask_cols = 0;
+        return DS4SP_OK;
+    }
+    if (rows < 1 || cols < 1) return fail(DS4SP_ERR_INVALID_ARG, "mask of %d x %d", rows, cols);
+    h->mask = mask;
+    h->mask_rows = rows;
+    h->mask_cols = cols;
     return DS4SP_OK;
 }
 

@@ -6,7 +6,9 @@
 // sparse prefill scheduling to 10K", Summary: "keep selected raw/compressed KV
 // transport in F16, and stream each selected latent row once across sixteen ...
 // heads". The per-token visibility (n_vis = (t+1)/4, window bounds) is computed
-// here from t; no mask is stored.
+// here from t; no mask is stored. (A debug form takes the compressed rows' visibility
+// from a stored mask instead, for the page's "explicit-mask versus analytic-mask"
+// check, Qualification section: see AttnParams::vis_mask.)
 //
 // Persistent CTAs (one per SM) take every gridDim-th token, heaviest first. A token
 // is a sequence of units: one unit holding its Q (16 rows), then its rows in blocks of
@@ -32,8 +34,9 @@
 //     value dims 128w .. 128w+127.
 // Rows are stored unpadded with their 16-byte chunks XOR-swizzled, which keeps the
 // producers' copies and the consumers' ldmatrix reads free of bank conflicts.
-// fp32 logits, sums and output; P enters P . V as fp16; exponentials on ex2.approx
-// (or exp2f in the precise instantiation).
+// fp32 logits, sums and output; P enters P . V as fp16 (or, in the fp32-staged
+// instantiation, as the sum of two fp16 terms hi + lo, lo = fp16(p - hi), at twice the
+// P . V tensor work); exponentials on ex2.approx (or exp2f in the precise instantiation).
 // Every wait is bounded; a consumer that gives up sets its group's flag, which the
 // group's warps read after their next barrier, so none is left waiting.
 #pragma once
@@ -79,9 +82,9 @@ constexpr int X_BYTES = 4 * 32 * 16;          // S partials passed between the K
 constexpr int REF_BYTES = 4 * H * 4;          // per S tile: reference used for its P
 constexpr int RED_BYTES = GWARPS * H * 4;     // per warp: softmax sums of a finished token
 constexpr int FLAG_BYTES = 16;                // raised[2], abort, pad
-constexpr int G_BYTES = P_BYTES + X_BYTES + REF_BYTES + RED_BYTES + FLAG_BYTES;
-constexpr int G_P = 0, G_X = P_BYTES, G_REF = G_X + X_BYTES, G_RED = G_REF + REF_BYTES,
-              G_FLAGS = G_RED + RED_BYTES;
+constexpr int G_BYTES = 2 * P_BYTES + X_BYTES + REF_BYTES + RED_BYTES + FLAG_BYTES;
+constexpr int G_P = 0, G_PLO = P_BYTES, G_X = 2 * P_BYTES, G_REF = G_X + X_BYTES,
+              G_RED = G_REF + REF_BYTES, G_FLAGS = G_RED + RED_BYTES;
 constexpr int OFF_RING = 0;
 constexpr int OFF_GROUP = OFF_RING + NS * SLOT;
 constexpr int OFF_MASK = OFF_GROUP + GROUPS * G_BYTES;   // row-validity bits per slot
@@ -127,6 +130,13 @@ struct AttnParams {
     int split, n_items;
     float* part_o;         // [n_items, 16, 512]
     float* part_ml;        // [n_items, 2, 16]: reference max (log2 units), sum
+    // Explicit-mask form (debug): when set, a top-k entry j is attended iff
+    // 0 <= j < mask_cols and vis_mask[t * mask_ld + j] != 0, in place of j < n_vis(t);
+    // -1 entries and entries the mask hides are dropped without a status bit (the
+    // top-k of this form pads with -1 when the mask leaves fewer than k rows).
+    const uint8_t* vis_mask;
+    long long mask_ld;
+    int mask_cols;
 };
 
 // A work item: the token (i, t and its rows) and the run of its 32-row units it covers,
@@ -217,7 +227,7 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
 }
 
 // PRECISE selects exp2f for the softmax exponentials instead of ex2.approx.
-template <bool PRECISE>
+template <bool PRECISE, bool PSPLIT>
 __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnParams p) {
     using namespace attn;
     auto exp2_ = [](float x) { return PRECISE ? exp2f(x) : fast_exp2(x); };
@@ -301,10 +311,19 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
             bool ok = false;
             if (gr < cu.tr.nsel) {
                 const int j = tk[gr];
-                if (j >= 0 && j < cu.tr.nv) {
-                    row = p.kv_cmp + (size_t)j * DQK;
-                    ok = true;
-                } else if ((lane & 3) == 0) {
+                if (p.vis_mask == nullptr) {
+                    if (j >= 0 && j < cu.tr.nv) {
+                        row = p.kv_cmp + (size_t)j * DQK;
+                        ok = true;
+                    } else if ((lane & 3) == 0) {
+                        record_status(p.status, kStatusBounds);
+                    }
+                } else if (j >= 0 && j < p.mask_cols) {
+                    if (p.vis_mask[(size_t)cu.tr.t * p.mask_ld + j] != 0) {
+                        row = p.kv_cmp + (size_t)j * DQK;
+                        ok = true;
+                    }
+                } else if (j != -1 && (lane & 3) == 0) {
                     record_status(p.status, kStatusBounds);
                 }
             } else if (gr < cu.tr.nrows) {
@@ -344,6 +363,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         const int gbar = GROUP_BAR + grp;
         uint8_t* garea = smem + OFF_GROUP + grp * G_BYTES;
         const uint32_t pbase = sbase + OFF_GROUP + grp * G_BYTES + G_P;
+        const uint32_t plobase = sbase + OFF_GROUP + grp * G_BYTES + G_PLO;
         float4* xbuf = reinterpret_cast<float4*>(garea + G_X);
         float* ref_tile = reinterpret_cast<float*>(garea + G_REF);
         float* red_sum = reinterpret_cast<float*>(garea + G_RED);
@@ -436,6 +456,17 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
             uint8_t* pb = garea + G_P + r0 * 2;
             *reinterpret_cast<uint32_t*>(pb + g * P_PITCH) = pack_half2(s4[0], s4[1]);
             *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH) = pack_half2(s4[2], s4[3]);
+            // fp32-staged: the fp16 remainder lo = p - fp16(p) beside P.
+            auto store_lo = [&](const float (&v)[4]) {
+                uint8_t* pl = garea + G_PLO + r0 * 2;
+                *reinterpret_cast<uint32_t*>(pl + g * P_PITCH) =
+                    pack_half2(v[0] - __half2float(__float2half_rn(v[0])),
+                               v[1] - __half2float(__float2half_rn(v[1])));
+                *reinterpret_cast<uint32_t*>(pl + (g + 8) * P_PITCH) =
+                    pack_half2(v[2] - __half2float(__float2half_rn(v[2])),
+                               v[3] - __half2float(__float2half_rn(v[3])));
+            };
+            if constexpr (PSPLIT) store_lo(s4);
             if (c == 0) {
                 ref_tile[own * H + g] = ref_g;
                 ref_tile[own * H + g + 8] = ref_g8;
@@ -470,6 +501,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                 for (int e = 0; e < 4; ++e) s4[e] *= e < 2 ? beta_g : beta_g8;
                 *reinterpret_cast<uint32_t*>(pb + g * P_PITCH) = pack_half2(s4[0], s4[1]);
                 *reinterpret_cast<uint32_t*>(pb + (g + 8) * P_PITCH) = pack_half2(s4[2], s4[3]);
+                if constexpr (PSPLIT) store_lo(s4);
                 m_g = M_g;
                 m_g8 = M_g8;
                 named_barrier(gbar, GTHREADS);    // rescaled P visible
@@ -483,11 +515,19 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
             for (int ks = 0; ks < 2; ++ks) {
                 uint32_t a[4];
                 ldsm_x4(pbase + ar * P_PITCH + (ks * 16 + hi * 8) * 2, a[0], a[1], a[2], a[3]);
+                uint32_t al[4];
+                if constexpr (PSPLIT)
+                    ldsm_x4(plobase + ar * P_PITCH + (ks * 16 + hi * 8) * 2, al[0], al[1], al[2],
+                            al[3]);
                 const int vr = ks * 16 + ar;
 #pragma unroll
                 for (int np = 0; np < 8; ++np) {
                     uint32_t b0, b1, b2, b3;
                     ldsm_x4_trans(chunk_addr(slot, vr, 16 * gw + 2 * np + hi), b0, b1, b2, b3);
+                    if constexpr (PSPLIT) {
+                        mma_16816(o[2 * np], al, b0, b1);
+                        mma_16816(o[2 * np + 1], al, b2, b3);
+                    }
                     mma_16816(o[2 * np], a, b0, b1);
                     mma_16816(o[2 * np + 1], a, b2, b3);
                 }

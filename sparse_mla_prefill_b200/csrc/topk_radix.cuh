@@ -9,9 +9,23 @@
 // order"); the tie rule and the ascending listing are this library's reading.
 //
 // One CTA per token. fp32 scores become order-preserving 32-bit keys (+0 and -0 map
-// to the same key). Four 8-bit radix passes over the keys in shared memory find the
-// k-th largest key K and how many keys equal to K must be kept (`need`). A block
-// scan then writes, in ascending j, every key > K and the first `need` keys == K.
+// to the same key). 8-bit radix passes over the keys find the k-th largest key K and
+// how many keys equal to K must be kept (`need`). The passes cover only the bits where
+// the candidates' keys differ (a block-wide AND and OR while the keys load):
+// integer-valued indexer scores in a narrow range share their top and bottom bits, so
+// two passes usually replace four, and the first pass spreads the keys over many
+// histogram bins instead of a few. The compaction then writes, in ascending j, every
+// key > K and the first `need` keys == K.
+//
+// The keys sit in shared memory; after a block scan of per-thread counts each thread
+// compacts a contiguous run of j.
+//
+// Explicit-mask form (a debug form of the same kernel, for the "explicit-mask versus
+// analytic-mask" check of the page's Qualification section): when `vis_mask` is
+// given, the candidates are the j < mask_cols whose mask byte for token t is set,
+// instead of j < n_vis(t). Rows the mask hides get key 0, below every finite score,
+// so they are never kept; with fewer than k candidates all of them are kept and the
+// remaining slots hold -1. Scores must be finite.
 #pragma once
 
 #include "device_common.cuh"
@@ -23,6 +37,113 @@ __device__ __forceinline__ uint32_t order_key(float x) {
     if (x == 0.f) u = 0u;                        // -0 ties with +0
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+
+// Block-wide OR and AND of the candidates' keys and their count (every thread gets
+// them): bits where OR and AND agree are the same in every candidate.
+template <int THREADS>
+__device__ __forceinline__ void block_key_stats(uint32_t kor, uint32_t kand, uint32_t cand,
+                                                uint32_t* w_or, uint32_t* w_and, uint32_t* w_cnt,
+                                                uint32_t& all_or, uint32_t& all_and,
+                                                uint32_t& n_cand) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    kor = __reduce_or_sync(0xffffffffu, kor);
+    kand = __reduce_and_sync(0xffffffffu, kand);
+    cand = __reduce_add_sync(0xffffffffu, cand);
+    if (lane == 0) {
+        w_or[warp] = kor;
+        w_and[warp] = kand;
+        w_cnt[warp] = cand;
+    }
+    __syncthreads();
+    all_or = 0u;
+    all_and = 0xffffffffu;
+    n_cand = 0u;
+#pragma unroll 4
+    for (int w = 0; w < THREADS / 32; ++w) {
+        all_or |= w_or[w];
+        all_and &= w_and[w];
+        n_cand += w_cnt[w];
+    }
+}
+
+// Warp 0: in a 256-bin histogram find the digit where the count from the top first
+// reaches `remaining`, and the count of the bins above it. Lane l owns bins 8l .. 8l+7.
+__device__ __forceinline__ void radix_find_digit(const uint32_t* hist, uint32_t remaining,
+                                                 uint32_t* s_digit, uint32_t* s_above) {
+    const int lane = threadIdx.x & 31;
+    uint32_t cnt[8], lane_sum = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+        cnt[b] = hist[8 * lane + b];
+        lane_sum += cnt[b];
+    }
+    uint32_t suffix = lane_sum;                  // bins of lanes >= lane
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_down_sync(0xffffffffu, suffix, off);
+        if (lane + off < 32) suffix += o;
+    }
+    uint32_t above = suffix - lane_sum;          // bins of lanes > lane
+#pragma unroll
+    for (int b = 7; b >= 0; --b) {
+        if (above < remaining && above + cnt[b] >= remaining) {
+            *s_digit = 8u * lane + b;
+            *s_above = above;
+        }
+        above += cnt[b];
+    }
+}
+
+// Radix select of the k-th largest candidate key (thr) and of how many keys equal to
+// it to keep (need), for n_cand > k candidates whose keys have block-wide OR all_or and
+// AND all_and. The 8-bit windows run from the highest bit where the candidates differ
+// down to the lowest; bits above the first window are the common prefix, bits below
+// the last are common too. The caller runs the passes:
+//     RadixSelect rs(all_or, all_and, k);
+//     while (rs.active) {
+//         rs.clear(hist, threads);                      // barrier inside
+//         each key x with x != 0 && (x & rs.digits) == rs.prefix:
+//             atomicAdd(&hist[(x >> rs.shift) & 255], 1)
+//         rs.step(hist, &s_digit, &s_above);            // barriers inside
+//     }
+//     rs.thr, rs.need
+struct RadixSelect {
+    uint32_t all_or, digits, prefix, remaining, thr, need;
+    int shift, lo_bit;
+    bool active;
+
+    __device__ __forceinline__ RadixSelect(uint32_t or_, uint32_t and_, uint32_t k)
+        : all_or(or_), remaining(k), thr(or_), need(k) {
+        const uint32_t diff = or_ ^ and_;
+        active = diff != 0u;                     // all candidates equal: the first k
+        const int hi_bit = active ? 31 - __clz(diff) : 0;
+        lo_bit = active ? __ffs(diff) - 1 : 0;
+        digits = hi_bit < 31 ? ~((2u << hi_bit) - 1u) : 0u;
+        prefix = or_ & digits;
+        shift = max(hi_bit - 7, 0);
+    }
+    __device__ __forceinline__ void clear(uint32_t* hist, int threads) const {
+        for (int b = threadIdx.x; b < 256; b += threads) hist[b] = 0;
+        __syncthreads();
+    }
+    __device__ __forceinline__ void step(const uint32_t* hist, uint32_t* s_digit,
+                                         uint32_t* s_above) {
+        __syncthreads();                         // the histogram is complete
+        if (threadIdx.x < 32) radix_find_digit(hist, remaining, s_digit, s_above);
+        __syncthreads();
+        prefix |= *s_digit << shift;
+        digits |= 255u << shift;
+        remaining -= *s_above;
+        __syncthreads();                         // s_digit / hist reused next pass
+        if (shift <= lo_bit) {
+            active = false;
+            thr = prefix | (all_or & ((1u << shift) - 1u));
+            need = remaining;
+        } else {
+            shift = max(shift - 8, 0);
+        }
+    }
+};
 
 // Exclusive block scan of a pair of counts packed as (hi << 32 | lo).
 template <int THREADS>
@@ -45,70 +166,73 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan(unsigned long
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS)
 topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int k, int ratio,
+                  const uint8_t* __restrict__ vis_mask, long long mask_ld, int mask_cols,
                   int32_t* __restrict__ topk) {
     extern __shared__ uint32_t keys[];           // [ld]
     __shared__ uint32_t hist[256];
     __shared__ uint32_t s_digit, s_above;
+    __shared__ uint32_t w_or[THREADS / 32], w_and[THREADS / 32], w_cnt[THREADS / 32];
     __shared__ unsigned long long warp_tot[THREADS / 32];
 
     const int i = blockIdx.x;
     const int t = t0 + i;
-    const int nv = n_vis(t, ratio);
     int32_t* out = topk + (size_t)i * k;
     const int tid = threadIdx.x;
-
-    if (nv <= k) {                               // every visible row is kept
-        for (int s = tid; s < k; s += THREADS) out[s] = s < nv ? s : -1;
-        return;
-    }
     const float* row = scores + (size_t)i * ld;
-    for (int j = tid; j < nv; j += THREADS) keys[j] = order_key(row[j]);
+    int n;                                       // keys examined: j < n
+    int keep = k;                                // slots filled; the rest hold -1
+    uint32_t kor = 0u, kand = 0xffffffffu, cand = 0u;   // over this thread's candidates
 
-    uint32_t prefix = 0, mask = 0, remaining = (uint32_t)k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int b = tid; b < 256; b += THREADS) hist[b] = 0;
-        __syncthreads();
-        for (int j = tid; j < nv; j += THREADS) {
-            const uint32_t key = keys[j];
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    if (vis_mask == nullptr) {
+        n = n_vis(t, ratio);
+        if (n <= k) {                            // every visible row is kept
+            for (int s = tid; s < k; s += THREADS) out[s] = s < n ? s : -1;
+            return;
         }
-        __syncthreads();
-        if (tid < 32) {
-            // Lane l owns bins 8l .. 8l+7; find the digit where the count from the top
-            // first reaches `remaining`.
-            uint32_t cnt[8], lane_sum = 0;
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                cnt[b] = hist[8 * tid + b];
-                lane_sum += cnt[b];
-            }
-            uint32_t suffix = lane_sum;          // bins of lanes >= tid
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const uint32_t o = __shfl_down_sync(0xffffffffu, suffix, off);
-                if (tid + off < 32) suffix += o;
-            }
-            uint32_t above = suffix - lane_sum;  // bins of lanes > tid
-#pragma unroll
-            for (int b = 7; b >= 0; --b) {
-                if (above < remaining && above + cnt[b] >= remaining) {
-                    s_digit = 8u * tid + b;
-                    s_above = above;
-                }
-                above += cnt[b];
+        for (int j = tid; j < n; j += THREADS) {
+            const uint32_t key = order_key(row[j]);
+            keys[j] = key;
+            kor |= key;
+            kand &= key;
+            ++cand;
+        }
+    } else {
+        n = mask_cols;
+        const uint8_t* mrow = vis_mask + (size_t)t * mask_ld;
+        for (int j = tid; j < n; j += THREADS) {
+            const bool v = mrow[j] != 0;
+            const uint32_t key = v ? order_key(row[j]) : 0u;
+            keys[j] = key;
+            if (v) {
+                kor |= key;
+                kand &= key;
+                ++cand;
             }
         }
-        __syncthreads();
-        prefix |= s_digit << shift;
-        mask |= 255u << shift;
-        remaining -= s_above;
-        __syncthreads();                         // s_digit / hist reused next pass
     }
-    const uint32_t thr = prefix;                 // the k-th largest key
-    const uint32_t need = remaining;             // keys == thr to keep, lowest j first
+    uint32_t all_or, all_and, n_cand;
+    block_key_stats<THREADS>(kor, kand, cand, w_or, w_and, w_cnt, all_or, all_and, n_cand);
 
-    const int per = (nv + THREADS - 1) / THREADS;
-    const int jb = min(nv, tid * per), je = min(nv, jb + per);
+    uint32_t thr = 0, need = 0;                  // without selection: every key > 0
+    if (n_cand <= (uint32_t)k) {
+        keep = (int)n_cand;                      // keep every candidate
+    } else {
+        RadixSelect rs(all_or, all_and, (uint32_t)k);
+        while (rs.active) {
+            rs.clear(hist, THREADS);
+            for (int j = tid; j < n; j += THREADS) {
+                const uint32_t key = keys[j];
+                if (key != 0u && (key & rs.digits) == rs.prefix)
+                    atomicAdd(&hist[(key >> rs.shift) & 255u], 1u);
+            }
+            rs.step(hist, &s_digit, &s_above);
+        }
+        thr = rs.thr;                            // the k-th largest key
+        need = rs.need;                          // keys == thr to keep, lowest j first
+    }
+
+    const int per = (n + THREADS - 1) / THREADS;
+    const int jb = min(n, tid * per), je = min(n, jb + per);
     uint32_t gt = 0, eq = 0;
     for (int j = jb; j < je; ++j) {
         const uint32_t key = keys[j];
@@ -128,6 +252,7 @@ topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int
             ++eq_rank;
         }
     }
+    for (int s = keep + tid; s < k; s += THREADS) out[s] = -1;
 }
 
 }  // namespace ds4sp

@@ -32,7 +32,7 @@ class ds4sp_config(ctypes.Structure):
                 ("ratio", ctypes.c_int), ("n_idx_heads", ctypes.c_int), ("d_idx", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("n_swa", ctypes.c_int), ("band", ctypes.c_int),
                 ("max_tokens", ctypes.c_int), ("softmax_scale", ctypes.c_float),
-                ("exp_mode", ctypes.c_int)]
+                ("exp_mode", ctypes.c_int), ("pv_mode", ctypes.c_int)]
 
 
 class ds4sp_io(ctypes.Structure):
@@ -60,6 +60,7 @@ _SIGS = {
     "ds4sp_profile_enable": (_i32, [_vp, _i32]),
     "ds4sp_profile_read": (_i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i32)]),
     "ds4sp_debug_fail_launches": (_i32, [_vp, _i32]),
+    "ds4sp_debug_set_mask": (_i32, [_vp, _vp, _i32, _i32]),
     "ds4sp_indexer_topk_noalloc": (_i32, [ctypes.POINTER(ds4sp_config), _vp, _vp, _vp, _i32,
                                           _i32, _vp, _vp]),
     "ds4sp_status_string": (ctypes.c_char_p, [_i32]),
@@ -123,6 +124,7 @@ class Handle:
     def __init__(self, ptr: int, cfg: ds4sp_config):
         self.ptr = ptr
         self.cfg = cfg
+        self.mask = None       # tensor set by ds4sp_debug_set_mask, kept alive here
 
     def __enter__(self):
         return self
@@ -140,9 +142,10 @@ class Handle:
 
 def make_config(n_idx_heads: int, d_idx: int, top_k: int, n_swa: int, max_tokens: int,
                 band: int = 2048, softmax_scale: float = 0.0, n_heads: int = 16, d_qk: int = 576,
-                d_v: int = 512, ratio: int = 4, exp_mode: int = 0) -> ds4sp_config:
+                d_v: int = 512, ratio: int = 4, exp_mode: int = 0,
+                pv_mode: int = 0) -> ds4sp_config:
     return ds4sp_config(n_heads, d_qk, d_v, ratio, n_idx_heads, d_idx, top_k, n_swa, band,
-                        max_tokens, softmax_scale, exp_mode)
+                        max_tokens, softmax_scale, exp_mode, pv_mode)
 
 
 def ds4sp_create(cfg: ds4sp_config) -> Handle:
@@ -240,6 +243,22 @@ def ds4sp_profile_read(h: Handle) -> Dict[str, Tuple[float, int]]:
 
 def ds4sp_debug_fail_launches(h: Handle, n: int) -> None:
     _check(load_library().ds4sp_debug_fail_launches(h.ptr, n), "ds4sp_debug_fail_launches")
+
+
+def ds4sp_debug_set_mask(h: Handle, mask: Optional[torch.Tensor]) -> None:
+    """Explicit-mask visibility: ``mask`` is uint8 [rows, cols] on the device (row t,
+    column j: compressed row j visible to token t), or None to return to the formula.
+    The handle keeps a reference to the tensor while it is set."""
+    lib = load_library()
+    if mask is None:
+        _check(lib.ds4sp_debug_set_mask(h.ptr, None, 0, 0), "ds4sp_debug_set_mask")
+        h.mask = None
+        return
+    if mask.dim() != 2:
+        raise Ds4spError(ERR_INVALID_ARG, "mask", "mask must be 2-D [rows, cols]")
+    _check(lib.ds4sp_debug_set_mask(h.ptr, _ptr(mask, "mask", torch.uint8), mask.shape[0],
+                                    mask.shape[1]), "ds4sp_debug_set_mask")
+    h.mask = mask
 
 
 def ds4sp_status_string(status: int) -> str:

@@ -56,6 +56,8 @@ def _cfg(**kw):
     (dict(max_tokens=(1 << 24) + 1), D.ERR_INVALID_ARG),
     (dict(softmax_scale=float("nan")), D.ERR_INVALID_ARG),
     (dict(exp_mode=2), D.ERR_INVALID_ARG),
+    (dict(pv_mode=2), D.ERR_INVALID_ARG),
+    (dict(pv_mode=-1), D.ERR_INVALID_ARG),
 ])
 def test_create_rejects_bad_config_before_touching_the_device(lib, kw, status):
     out = ctypes.c_void_p(123)
@@ -76,6 +78,8 @@ def test_null_handle_paths(lib):
     io = D.ds4sp_io()
     assert lib.ds4sp_prefill_host(None, 16, ctypes.byref(io), ctypes.byref(io), None, 0,
                                   None) == D.ERR_INVALID_ARG
+    assert lib.ds4sp_debug_set_mask(None, None, 0, 0) == D.ERR_INVALID_ARG
+    assert lib.ds4sp_debug_set_mask(None, 256, 16, 4) == D.ERR_INVALID_ARG
 
 
 def test_status_strings(lib):
