@@ -45,9 +45,9 @@ def _stricter_mask(T: int, n_c: int, seed: int, hide: float = 0.3) -> np.ndarray
     return oracle.explicit_visibility_mask(T, n_c) & (rng.random((T, n_c)) >= hide)
 
 
-@pytest.mark.parametrize("name", ["tiny", "band"])
-def test_formula_mask_is_bit_identical(name):
-    wl = workload(name)
+@pytest.mark.parametrize("name,T", [("tiny", None), ("band", None), ("band", 4096)])
+def test_formula_mask_is_bit_identical(name, T):
+    wl = workload(name) if T is None else workload(name, T=T)   # 4096: two bands
     inp = generate(wl)
     dev = to_device(inp)
     mask = oracle.explicit_visibility_mask(wl.T, inp["kv_cmp"].shape[0])
@@ -129,3 +129,27 @@ def test_mask_shorter_than_the_call_is_rejected():
         assert lib.ds4sp_debug_set_mask(h.ptr, m.data_ptr(), 0, m.shape[1]) == D.ERR_INVALID_ARG
         assert lib.ds4sp_debug_set_mask(h.ptr, m.data_ptr(), m.shape[0], -1) == D.ERR_INVALID_ARG
         torch.cuda.synchronize()
+
+
+def test_mask_wide_rows_few_tokens():
+    """Rows longer than 4,096 scores (the 1,024-thread top-k) and a few-token call (split
+    attention with the merge): the last 5 tokens of a 16,400-token context."""
+    wl = workload("verify", T=16400, seed=11)
+    inp = generate(wl)
+    npi = _np(inp)
+    n_c = inp["kv_cmp"].shape[0]
+    t0, n_q = wl.q_start, wl.verify_q
+    t = np.arange(wl.T)[:, None]
+    j = np.arange(n_c)[None, :]
+    mask = 4 * j + 3 <= t                                   # the formula's mask
+    rng = np.random.default_rng(5)
+    mask[t0:] &= rng.random((n_q, n_c)) >= 0.3              # the query rows: stricter
+    with handle_for(wl) as h:
+        D.ds4sp_debug_set_mask(h, _dev_mask(mask))
+        tk, out = run_range(h, to_device(inp), t0, n_q, wl.top_k)
+    scores = oracle.indexer_scores(npi["q_idx"], npi["k_idx"], npi["w"], t0)
+    want = np.stack([oracle.topk_row_masked(scores[i], mask[t0 + i], wl.top_k)
+                     for i in range(n_q)])
+    assert np.array_equal(tk.cpu().numpy(), want)
+    ref = oracle.sparse_mla_attention(npi["q"], npi["kv_raw"], npi["kv_cmp"], want, t0, wl.n_swa)
+    assert_attention_close(out.cpu().numpy(), ref, "wide rows, masked")
