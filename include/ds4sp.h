@@ -155,13 +155,16 @@ typedef struct ds4sp_io {
 } ds4sp_io;
 
 /* A whole n_tokens prefill from host memory to host memory: every band in order, as
- * ds4sp_prefill_band does, with the transfers overlapped. Band b's rows of q, q_idx and
- * w, and the KV, compressed-KV and index-key rows it is the first band to need, are
- * copied in on a copy stream of the handle; band b computes on `stream` once they have
- * arrived; band b's rows of out (and topk) go back on a second copy stream of the
- * handle, so copies in, compute and copies out of neighbouring bands run at the same
- * time. The pages commit bands in order ("perf(ds4): extend sparse prefill scheduling
- * to 10K", Summary); this entry point is the host side of that loop.
+ * ds4sp_prefill_band does, with the transfers overlapped. Each band is taken in steps of
+ * about 1,024 tokens, in token order. A step's rows of q, q_idx and w, and the KV,
+ * compressed-KV and index-key rows it is the first step to need, are copied in on a
+ * copy stream of the handle; the step computes (steps 1-3 for its tokens) on `stream`
+ * once they have arrived; its rows of out (and topk) go back on a second copy stream of
+ * the handle, so copies in, compute and copies out of neighbouring steps run at the
+ * same time and only the last step's copy out trails. Every token's result is the same
+ * bits as in ds4sp_prefill_band (a token's indices and output do not depend on the
+ * other tokens of a call). The pages commit bands in order ("perf(ds4): extend sparse
+ * prefill scheduling to 10K", Summary); this entry point is the host side of that loop.
  *   host  inputs and outputs in host memory; dev  device buffers of the same shapes
  *   (all of them required, including topk when top_k > 0), overwritten by the call;
  *   ws    device scratch of ws_bytes >= ds4sp_workspace_bytes(h, t0, band) for every

@@ -40,6 +40,7 @@ ds4sp_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 constexpr int kMaxTopkCandidates = 51200;  // top-k keeps a token's row in shared memory
+constexpr int kHostChunk = 1024;           // ds4sp_prefill_host: tokens per copy/compute step
 
 enum Kind { kIndexer = 0, kTopk = 1, kAttn = 2 };
 
@@ -62,7 +63,7 @@ struct ds4sp_handle {
     std::vector<TimedLaunch> timed;
     std::vector<cudaEvent_t> event_pool;
     bool smem_set[3] = {false, false, false};
-    // ds4sp_prefill_host: copy streams (in, out) and per-band events, made on first use.
+    // ds4sp_prefill_host: copy streams (in, out) and per-chunk events, made on first use.
     cudaStream_t copy_in = nullptr, copy_out = nullptr;
     std::vector<cudaEvent_t> band_in, band_done;
     cudaEvent_t host_start = nullptr, host_end = nullptr;
@@ -463,6 +464,23 @@ ds4sp_status sparse_attn_impl(ds4sp_handle* h, const void* q, const void* kv_raw
     return record_last(h, stream);
 }
 
+// Steps 1-3 for tokens [t0, t0+n_q) on whole-sequence base pointers (q, q_idx, w,
+// topk, out are offset here to row t0; the KV tensors are used as given).
+ds4sp_status prefill_range(ds4sp_handle* h, int t0, int n_q, const void* q, const void* q_idx,
+                           const float* w, const void* kv_raw, const void* kv_cmp,
+                           const void* k_idx, int32_t* topk, float* out, void* ws,
+                           size_t ws_bytes, cudaStream_t s, const void* prefetch,
+                           size_t prefetch_bytes) {
+    const ds4sp_config& c = h->cfg;
+    auto* qh = static_cast<const __half*>(q) + (size_t)t0 * c.n_heads * c.d_qk;
+    auto* qi = static_cast<const __half*>(q_idx) + (size_t)t0 * c.n_idx_heads * c.d_idx;
+    const float* wt = w + (size_t)t0 * c.n_idx_heads;
+    int32_t* tk = c.top_k > 0 ? topk + (size_t)t0 * c.top_k : nullptr;
+    float* ot = out + (size_t)t0 * c.n_heads * c.d_v;
+    if (c.top_k > 0) DS4SP_TRY(indexer_topk_impl(h, qi, k_idx, wt, t0, n_q, tk, ws, ws_bytes, s));
+    return sparse_attn_impl(h, qh, kv_raw, kv_cmp, tk, t0, n_q, ot, s, prefetch, prefetch_bytes);
+}
+
 }  // namespace
 
 extern "C" {
@@ -592,17 +610,9 @@ ds4sp_status ds4sp_prefill_band(ds4sp_handle* h, int b, int n_tokens, const void
         }
     }
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    auto* qh = static_cast<const __half*>(q) + (size_t)t0 * c.n_heads * c.d_qk;
-    auto* qi = static_cast<const __half*>(q_idx) + (size_t)t0 * c.n_idx_heads * c.d_idx;
-    const float* wt = w + (size_t)t0 * c.n_idx_heads;
-    int32_t* tk = c.top_k > 0 ? topk + (size_t)t0 * c.top_k : nullptr;
-    float* ot = out + (size_t)t0 * c.n_heads * c.d_v;
-    if (c.top_k > 0) {
-        if (ws_bytes < ds4sp_workspace_bytes(h, t0, n_q))
-            return fail(DS4SP_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes,
-                        ds4sp_workspace_bytes(h, t0, n_q));
-        DS4SP_TRY(indexer_topk_impl(h, qi, k_idx, wt, t0, n_q, tk, ws, ws_bytes, s));
-    }
+    if (c.top_k > 0 && ws_bytes < ds4sp_workspace_bytes(h, t0, n_q))
+        return fail(DS4SP_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes,
+                    ds4sp_workspace_bytes(h, t0, n_q));
     // The next band's indexer queries (read first thing by its indexer) are brought into
     // L2 at the tail of this band's attention.
     const int t1 = t0 + n_q, n_next = std::min(c.band, n_tokens - t1);
@@ -612,7 +622,8 @@ ds4sp_status ds4sp_prefill_band(ds4sp_handle* h, int b, int n_tokens, const void
         pf = static_cast<const __half*>(q_idx) + (size_t)t1 * c.n_idx_heads * c.d_idx;
         pf_bytes = (size_t)n_next * c.n_idx_heads * c.d_idx * 2;
     }
-    DS4SP_TRY(sparse_attn_impl(h, qh, kv_raw, kv_cmp, tk, t0, n_q, ot, s, pf, pf_bytes));
+    DS4SP_TRY(prefill_range(h, t0, n_q, q, q_idx, w, kv_raw, kv_cmp, k_idx, topk, out, ws,
+                            ws_bytes, s, pf, pf_bytes));
     h->next_band = b + 1;
     return DS4SP_OK;
 }
@@ -639,6 +650,34 @@ ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* h
                                               n_tokens - (n_bands - 1) * c.band);
     if (sel && ws_bytes < need)
         return fail(DS4SP_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    if (sel) {
+        DS4SP_TRY(check_ptr(dev->topk, "dev: topk"));
+        DS4SP_TRY(check_ptr(ws, "ws"));
+    }
+    for (const void* p : {static_cast<const void*>(dev->q), static_cast<const void*>(dev->q_idx),
+                          static_cast<const void*>(dev->w), static_cast<const void*>(dev->kv_raw),
+                          static_cast<const void*>(dev->out)})
+        DS4SP_TRY(check_ptr(p, "dev tensor"));
+
+    // Steps of at most kHostChunk tokens inside each band, in order: band b's tokens
+    // [b*band, (b+1)*band) are cut into chunks; a chunk's copies in, its compute and its
+    // copies out are queued on three streams, so that copies in, compute and copies out
+    // of neighbouring chunks overlap and only the last chunk's output copy trails.
+    // A remainder small enough for the few-token attention path joins the chunk before
+    // it, so that no chunk takes that path unless its whole band does (the device path
+    // then takes it too): every token sees the same kernels as in ds4sp_prefill_band.
+    struct Chunk { int band, t0, n; };
+    std::vector<Chunk> chunks;
+    for (int b = 0; b < n_bands; ++b) {
+        const int t0 = b * c.band, t1 = std::min(n_tokens, t0 + c.band);
+        for (int u = t0; u < t1;) {
+            const int left = t1 - u;
+            const int n = left - kHostChunk <= attn::SPLIT_MAX_TOKENS ? left : kHostChunk;
+            chunks.push_back({b, u, n});
+            u += n;
+        }
+    }
+    const int n_chunks = (int)chunks.size();
 
     cudaError_t e = cudaSuccess;
     if (!h->copy_in) e = cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking);
@@ -648,7 +687,7 @@ ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* h
         e = cudaEventCreateWithFlags(&h->host_start, cudaEventDisableTiming);
     if (e == cudaSuccess && !h->host_end)
         e = cudaEventCreateWithFlags(&h->host_end, cudaEventDisableTiming);
-    while (e == cudaSuccess && (int)h->band_in.size() < n_bands) {
+    while (e == cudaSuccess && (int)h->band_in.size() < n_chunks) {
         cudaEvent_t a = nullptr, b = nullptr;
         e = cudaEventCreateWithFlags(&a, cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&b, cudaEventDisableTiming);
@@ -682,10 +721,10 @@ ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* h
         return cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off,
                                bytes, cudaMemcpyDeviceToHost, h->copy_out);
     };
-    // Inputs: per band, its token rows and the KV rows it is the first to need.
+    // Inputs: per chunk, its token rows and the KV rows it is the first to need.
     int raw_done = 0, cmp_done = 0;
-    for (int b = 0; b < n_bands && e == cudaSuccess; ++b) {
-        const int t0 = b * c.band, t1 = std::min(n_tokens, t0 + c.band), n = t1 - t0;
+    for (int i = 0; i < n_chunks && e == cudaSuccess; ++i) {
+        const int t0 = chunks[i].t0, n = chunks[i].n, t1 = t0 + n;
         e = h2d(dev->q, host->q, t0 * q_row, n * q_row);
         if (e == cudaSuccess && sel) e = h2d(dev->q_idx, host->q_idx, t0 * qi_row, n * qi_row);
         if (e == cudaSuccess && sel) e = h2d(dev->w, host->w, t0 * w_row, n * w_row);
@@ -698,21 +737,23 @@ ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* h
                 e = h2d(dev->k_idx, host->k_idx, cmp_done * ki_row, (cmp_need - cmp_done) * ki_row);
             cmp_done = cmp_need;
         }
-        if (e == cudaSuccess) e = cudaEventRecord(h->band_in[b], h->copy_in);
+        if (e == cudaSuccess) e = cudaEventRecord(h->band_in[i], h->copy_in);
     }
     if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: copies in");
 
-    // Compute, band by band, each after its inputs; outputs copied back band by band.
+    // Compute, chunk by chunk in band order, each after its inputs; outputs copied back
+    // chunk by chunk.
     h->next_band = 0;
-    for (int b = 0; b < n_bands; ++b) {
-        const int t0 = b * c.band, n = std::min(n_tokens, t0 + c.band) - t0;
-        e = cudaStreamWaitEvent(s, h->band_in[b], 0);
+    for (int i = 0; i < n_chunks; ++i) {
+        const int t0 = chunks[i].t0, n = chunks[i].n;
+        e = cudaStreamWaitEvent(s, h->band_in[i], 0);
         if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: wait for inputs");
-        DS4SP_TRY(ds4sp_prefill_band(h, b, n_tokens, dev->q, dev->q_idx, dev->w, dev->kv_raw,
-                                     dev->kv_cmp, dev->k_idx, dev->topk, dev->out, ws, ws_bytes,
-                                     stream));
-        e = cudaEventRecord(h->band_done[b], s);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->band_done[b], 0);
+        DS4SP_TRY(prefill_range(h, t0, n, dev->q, dev->q_idx, dev->w, dev->kv_raw, dev->kv_cmp,
+                                dev->k_idx, dev->topk, dev->out, ws, ws_bytes, s, nullptr, 0));
+        if (i + 1 == n_chunks || chunks[i + 1].band != chunks[i].band)
+            h->next_band = chunks[i].band + 1;
+        e = cudaEventRecord(h->band_done[i], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->band_done[i], 0);
         if (e == cudaSuccess) e = d2h(host->out, dev->out, t0 * o_row, n * o_row);
         if (e == cudaSuccess && sel && host->topk)
             e = d2h(host->topk, dev->topk, t0 * tk_row, n * tk_row);

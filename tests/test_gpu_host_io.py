@@ -1,7 +1,7 @@
-"""ds4sp_prefill_host: the whole prefill from pinned host buffers to host buffers, with
-the copies overlapped across bands, must give exactly what the device-resident path
-gives (same kernels, same inputs), including an uneven last band, no top-k, and a
-call queued behind other work on the stream."""
+"""ds4sp_prefill_host: the whole prefill from pinned host buffers to host buffers, in
+steps of about 1,024 tokens with the copies overlapped, must give exactly what the
+device-resident band path gives (same kernels, same inputs), including an uneven last
+band, small remainders, no top-k, and a call queued behind other work on the stream."""
 import numpy as np
 import pytest
 import torch
@@ -35,7 +35,13 @@ def _host_run(h, host, T, top_k, stream=None):
 
 
 @pytest.mark.parametrize("T,top_k,band", [(600, 32, 256), (1024, 64, 256), (300, 0, 128),
-                                          (2048, 128, 2048)])
+                                          (2048, 128, 2048),
+                                          # 1,024-token steps: a 40-token last step,
+                                          # an 18-token remainder folded into the step
+                                          # before it, a 20-token band (few-token
+                                          # attention on both paths)
+                                          (3112, 64, 2048), (3090, 128, 2048),
+                                          (2068, 32, 2048)])
 def test_host_path_matches_device_path(T, top_k, band):
     wl = Workload("host", T=T, H_i=8, D_i=64, top_k=top_k, n_swa=32, seed=3, band=band)
     inp = generate_small(T, wl.H_i, wl.D_i, seed=11)
