@@ -40,7 +40,7 @@ ds4sp_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 constexpr int kMaxTopkCandidates = 51200;  // top-k keeps a token's row in shared memory
-constexpr int kHostChunk = 1024;           // ds4sp_prefill_host: tokens per copy/compute step
+constexpr int kHostStep = 1024;            // ds4sp_prefill_host: tokens per copy/compute step
 
 enum Kind { kIndexer = 0, kTopk = 1, kAttn = 2 };
 
@@ -63,9 +63,9 @@ struct ds4sp_handle {
     std::vector<TimedLaunch> timed;
     std::vector<cudaEvent_t> event_pool;
     bool smem_set[3] = {false, false, false};
-    // ds4sp_prefill_host: copy streams (in, out) and per-chunk events, made on first use.
+    // ds4sp_prefill_host: copy streams (in, out) and per-step events, made on first use.
     cudaStream_t copy_in = nullptr, copy_out = nullptr;
-    std::vector<cudaEvent_t> band_in, band_done;
+    std::vector<cudaEvent_t> step_in, step_done;
     cudaEvent_t host_start = nullptr, host_end = nullptr;
     // Split-mode attention partials (few tokens): capacity in 32-row units.
     int split_cap = 0;
@@ -546,8 +546,8 @@ ds4sp_status ds4sp_destroy(ds4sp_handle* h) {
         s = fail(DS4SP_ERR_CUDA, "pending copies failed before destroy");
     if (h->copy_out && cudaStreamSynchronize(h->copy_out) != cudaSuccess)
         s = fail(DS4SP_ERR_CUDA, "pending copies failed before destroy");
-    for (auto e : h->band_in) cudaEventDestroy(e);
-    for (auto e : h->band_done) cudaEventDestroy(e);
+    for (auto e : h->step_in) cudaEventDestroy(e);
+    for (auto e : h->step_done) cudaEventDestroy(e);
     if (h->host_start) cudaEventDestroy(h->host_start);
     if (h->host_end) cudaEventDestroy(h->host_end);
     if (h->copy_in) cudaStreamDestroy(h->copy_in);
@@ -659,25 +659,25 @@ ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* h
                           static_cast<const void*>(dev->out)})
         DS4SP_TRY(check_ptr(p, "dev tensor"));
 
-    // Steps of at most kHostChunk tokens inside each band, in order: band b's tokens
-    // [b*band, (b+1)*band) are cut into chunks; a chunk's copies in, its compute and its
+    // Steps of about kHostStep tokens inside each band, in order: band b's tokens
+    // [b*band, (b+1)*band) are cut into steps; a step's copies in, its compute and its
     // copies out are queued on three streams, so that copies in, compute and copies out
-    // of neighbouring chunks overlap and only the last chunk's output copy trails.
-    // A remainder small enough for the few-token attention path joins the chunk before
-    // it, so that no chunk takes that path unless its whole band does (the device path
+    // of neighbouring steps overlap and only the last step's output copy trails.
+    // A remainder small enough for the few-token attention path joins the step before
+    // it, so that no step takes that path unless its whole band does (the device path
     // then takes it too): every token sees the same kernels as in ds4sp_prefill_band.
-    struct Chunk { int band, t0, n; };
-    std::vector<Chunk> chunks;
+    struct Step { int band, t0, n; };
+    std::vector<Step> steps;
     for (int b = 0; b < n_bands; ++b) {
         const int t0 = b * c.band, t1 = std::min(n_tokens, t0 + c.band);
         for (int u = t0; u < t1;) {
             const int left = t1 - u;
-            const int n = left - kHostChunk <= attn::SPLIT_MAX_TOKENS ? left : kHostChunk;
-            chunks.push_back({b, u, n});
+            const int n = left - kHostStep <= attn::SPLIT_MAX_TOKENS ? left : kHostStep;
+            steps.push_back({b, u, n});
             u += n;
         }
     }
-    const int n_chunks = (int)chunks.size();
+    const int n_steps = (int)steps.size();
 
     cudaError_t e = cudaSuccess;
     if (!h->copy_in) e = cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking);
@@ -687,7 +687,7 @@ ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* h
         e = cudaEventCreateWithFlags(&h->host_start, cudaEventDisableTiming);
     if (e == cudaSuccess && !h->host_end)
         e = cudaEventCreateWithFlags(&h->host_end, cudaEventDisableTiming);
-    while (e == cudaSuccess && (int)h->band_in.size() < n_chunks) {
+    while (e == cudaSuccess && (int)h->step_in.size() < n_steps) {
         cudaEvent_t a = nullptr, b = nullptr;
         e = cudaEventCreateWithFlags(&a, cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&b, cudaEventDisableTiming);
@@ -695,8 +695,8 @@ ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* h
             if (a) cudaEventDestroy(a);
             break;
         }
-        h->band_in.push_back(a);
-        h->band_done.push_back(b);
+        h->step_in.push_back(a);
+        h->step_done.push_back(b);
     }
     if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: streams/events");
 
@@ -721,10 +721,10 @@ ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* h
         return cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off,
                                bytes, cudaMemcpyDeviceToHost, h->copy_out);
     };
-    // Inputs: per chunk, its token rows and the KV rows it is the first to need.
+    // Inputs: per step, its token rows and the KV rows it is the first to need.
     int raw_done = 0, cmp_done = 0;
-    for (int i = 0; i < n_chunks && e == cudaSuccess; ++i) {
-        const int t0 = chunks[i].t0, n = chunks[i].n, t1 = t0 + n;
+    for (int i = 0; i < n_steps && e == cudaSuccess; ++i) {
+        const int t0 = steps[i].t0, n = steps[i].n, t1 = t0 + n;
         e = h2d(dev->q, host->q, t0 * q_row, n * q_row);
         if (e == cudaSuccess && sel) e = h2d(dev->q_idx, host->q_idx, t0 * qi_row, n * qi_row);
         if (e == cudaSuccess && sel) e = h2d(dev->w, host->w, t0 * w_row, n * w_row);
@@ -737,23 +737,23 @@ ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* h
                 e = h2d(dev->k_idx, host->k_idx, cmp_done * ki_row, (cmp_need - cmp_done) * ki_row);
             cmp_done = cmp_need;
         }
-        if (e == cudaSuccess) e = cudaEventRecord(h->band_in[i], h->copy_in);
+        if (e == cudaSuccess) e = cudaEventRecord(h->step_in[i], h->copy_in);
     }
     if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: copies in");
 
-    // Compute, chunk by chunk in band order, each after its inputs; outputs copied back
-    // chunk by chunk.
+    // Compute, step by step in band order, each after its inputs; outputs copied back
+    // step by step.
     h->next_band = 0;
-    for (int i = 0; i < n_chunks; ++i) {
-        const int t0 = chunks[i].t0, n = chunks[i].n;
-        e = cudaStreamWaitEvent(s, h->band_in[i], 0);
+    for (int i = 0; i < n_steps; ++i) {
+        const int t0 = steps[i].t0, n = steps[i].n;
+        e = cudaStreamWaitEvent(s, h->step_in[i], 0);
         if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: wait for inputs");
         DS4SP_TRY(prefill_range(h, t0, n, dev->q, dev->q_idx, dev->w, dev->kv_raw, dev->kv_cmp,
                                 dev->k_idx, dev->topk, dev->out, ws, ws_bytes, s, nullptr, 0));
-        if (i + 1 == n_chunks || chunks[i + 1].band != chunks[i].band)
-            h->next_band = chunks[i].band + 1;
-        e = cudaEventRecord(h->band_done[i], s);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->band_done[i], 0);
+        if (i + 1 == n_steps || steps[i + 1].band != steps[i].band)
+            h->next_band = steps[i].band + 1;
+        e = cudaEventRecord(h->step_done[i], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->step_done[i], 0);
         if (e == cudaSuccess) e = d2h(host->out, dev->out, t0 * o_row, n * o_row);
         if (e == cudaSuccess && sel && host->topk)
             e = d2h(host->topk, dev->topk, t0 * tk_row, n * tk_row);
