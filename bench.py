@@ -161,21 +161,38 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ reference arm (oracle)
 
-def cpu_oracle_sample(wl, n_sample, inputs_np=None):
-    """Time the float64 CPU oracle on a spread sample of tokens; tokens/s."""
-    import numpy as np
+def cpu_oracle_sample(wl, n_sample, inputs_np=None, return_result=False):
+    """Time the float64 CPU oracle on a spread sample of tokens; tokens/s (and, with
+    return_result, the oracle's indices and outputs for those tokens)."""
     import oracle
     if inputs_np is None:
         inputs_np = {k: v.numpy() for k, v in generate(wl).items()}
     stride = max(1, wl.T // n_sample)
     toks = list(range(stride - 1, wl.T, stride))[:n_sample]
     t0 = time.perf_counter()
-    oracle.prefill_tokens(inputs_np, toks, wl.top_k, wl.n_swa)
+    ref = oracle.prefill_tokens(inputs_np, toks, wl.top_k, wl.n_swa)
     dt = time.perf_counter() - t0
-    return {"value": len(toks) / dt, "unit": "tokens/s", "cores": torch.get_num_threads(),
+    line = {"value": len(toks) / dt, "unit": "tokens/s", "cores": torch.get_num_threads(),
             "kind": "oracle",
             "sample": f"{len(toks)} of {wl.T} tokens (every {stride}th), float64 NumPy, "
                       f"{dt:.1f} s"}
+    return (line, ref) if return_result else line
+
+
+def sampled_parity(ref, topk_gpu, out_gpu):
+    """The end-to-end result against the oracle on its sampled tokens: indices bit for
+    bit, attention max-abs and NMSE over every element of those tokens."""
+    import numpy as np
+    toks = ref["tokens"]
+    got = out_gpu[toks].astype(np.float64)
+    err = got - ref["out"]
+    max_abs = float(np.abs(err).max())
+    nmse = float((err ** 2).sum() / (ref["out"] ** 2).sum())
+    exact = bool(np.array_equal(topk_gpu[toks], ref["topk"]))
+    return {"tokens": int(len(toks)), "topk_bit_exact": exact, "max_abs": max_abs, "nmse": nmse,
+            "bar": {"max_abs": 2e-3, "nmse": 1e-6},
+            "pass": exact and max_abs <= 2e-3 and nmse <= 1e-6,
+            "of": "ds4sp_prefill_host result (pinned host buffers)"}
 
 
 def run_reference(args, rank, world):
@@ -328,6 +345,10 @@ def run_ours(args, rank, world, local_rank):
     st, bits = D.ds4sp_device_status(h)
     if st != D.OK:
         raise RuntimeError(f"device status {bits:#x} after timing")
+    # The end-to-end result, kept for the parity check against the oracle's sample below
+    # (the variants after this overwrite the device buffers).
+    out_e2e = out_host.numpy().copy()
+    topk_e2e = topk.cpu().numpy()
 
     verify = None
     if rank == 0 and world == 1 and not args.no_verify:
@@ -361,9 +382,12 @@ def run_ours(args, rank, world, local_rank):
             finally:
                 D.ds4sp_destroy(hv)
 
-    cpu_base = None
+    cpu_base = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu_base = cpu_oracle_sample(wl, args.cpu_sample, {k: v.numpy() for k, v in host.items()})
+        cpu_base, ref = cpu_oracle_sample(wl, args.cpu_sample,
+                                          {k: v.numpy() for k, v in host.items()},
+                                          return_result=True)
+        parity = sampled_parity(ref, topk_e2e, out_e2e)
 
     if rank == 0:
         value = job_throughput(wl.T, world, args.steps, ms_max)
@@ -403,6 +427,7 @@ def run_ours(args, rank, world, local_rank):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "clocks": clk,
             "cpu_baseline": cpu_base,
+            "parity": parity,
         }
         print(json.dumps(line), flush=True)
     D.ds4sp_destroy(h)

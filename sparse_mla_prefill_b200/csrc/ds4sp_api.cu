@@ -3,6 +3,7 @@
 // computes runs in the kernels included below; this file only validates and launches.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdarg>
@@ -79,6 +80,15 @@ struct ds4sp_handle {
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range around each entry point that queues work, named after it, so that a
+// profiler's timeline shows the library's calls (no cost without a profiler attached).
+struct TraceRange {
+    explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+    TraceRange(const TraceRange&) = delete;
+    TraceRange& operator=(const TraceRange&) = delete;
+};
 
 int nvis(int t, int ratio) { return (t + 1) / ratio; }
 
@@ -570,6 +580,7 @@ size_t ds4sp_workspace_bytes(const ds4sp_handle* h, int t0, int n_q) {
 ds4sp_status ds4sp_indexer_topk(ds4sp_handle* h, const void* q_idx, const void* k_idx,
                                 const float* w, int t0, int n_q, int32_t* topk, void* ws,
                                 size_t ws_bytes, void* stream) {
+    const TraceRange trace("ds4sp_indexer_topk");
     DS4SP_TRY(check_handle(h));
     return indexer_topk_impl(h, q_idx, k_idx, w, t0, n_q, topk, ws, ws_bytes,
                              static_cast<cudaStream_t>(stream));
@@ -578,6 +589,7 @@ ds4sp_status ds4sp_indexer_topk(ds4sp_handle* h, const void* q_idx, const void* 
 ds4sp_status ds4sp_sparse_attn(ds4sp_handle* h, const void* q, const void* kv_raw,
                                const void* kv_cmp, const int32_t* topk, int t0, int n_q,
                                float* out, void* stream) {
+    const TraceRange trace("ds4sp_sparse_attn");
     DS4SP_TRY(check_handle(h));
     return sparse_attn_impl(h, q, kv_raw, kv_cmp, topk, t0, n_q, out,
                             static_cast<cudaStream_t>(stream));
@@ -587,6 +599,7 @@ ds4sp_status ds4sp_prefill_band(ds4sp_handle* h, int b, int n_tokens, const void
                                 const void* q_idx, const float* w, const void* kv_raw,
                                 const void* kv_cmp, const void* k_idx, int32_t* topk,
                                 float* out, void* ws, size_t ws_bytes, void* stream) {
+    const TraceRange trace("ds4sp_prefill_band");
     DS4SP_TRY(check_handle(h));
     const ds4sp_config& c = h->cfg;
     if (n_tokens < 1 || n_tokens > c.max_tokens)
@@ -630,6 +643,7 @@ ds4sp_status ds4sp_prefill_band(ds4sp_handle* h, int b, int n_tokens, const void
 
 ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* host,
                                 const ds4sp_io* dev, void* ws, size_t ws_bytes, void* stream) {
+    const TraceRange trace("ds4sp_prefill_host");
     DS4SP_TRY(check_handle(h));
     if (!host || !dev) return fail(DS4SP_ERR_INVALID_ARG, "host or dev is null");
     const ds4sp_config& c = h->cfg;
@@ -924,6 +938,7 @@ ds4sp_status check_static_config(const ds4sp_config* cfg) {
 extern "C" ds4sp_status ds4sp_indexer_topk_noalloc(const ds4sp_config* cfg, const void* q_idx,
                                                    const void* k_idx, const float* w, int t0,
                                                    int n_q, int32_t* topk, void* stream) {
+    const TraceRange trace("ds4sp_indexer_topk_noalloc");
     DS4SP_TRY(check_static_config(cfg));
     if (t0 < 0 || n_q < 0 || (long long)t0 + n_q > cfg->max_tokens)
         return fail(DS4SP_ERR_INVALID_ARG, "token range [%d, %d+%d) outside [0, %d)", t0, t0, n_q,
