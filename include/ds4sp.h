@@ -27,8 +27,9 @@
  *     KV tensors (kv_raw, kv_cmp, k_idx) are whole-sequence base pointers holding at
  *     least max_tokens (raw) or max_tokens/4 (compressed) rows.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
- *     stream). The library launches kernels only; it never allocates, frees or copies
- *     caller memory, and never synchronises the caller's stream except where stated.
+ *     stream). The library launches kernels only; it never allocates or frees caller
+ *     memory, copies it only in ds4sp_prefill_host (between the caller's host and
+ *     device buffers), and never synchronises the caller's stream except where stated.
  *   - Argument, shape, order and workspace errors are returned before any launch.
  *     A failed launch returns DS4SP_ERR_CUDA. Index checks inside the kernels never
  *     fault: an out-of-range index is skipped and recorded in a device status word
@@ -116,13 +117,13 @@ ds4sp_status ds4sp_indexer_topk(ds4sp_handle* h, const void* q_idx, const void* 
  *   fp16, topk [n_q, top_k] int32 as written by ds4sp_indexer_topk (entries
  *   0 .. min(k, n_vis(t))-1 hold visible rows), out [n_q, 16, 512] fp32 (output).
  * Rows are fp16; logits, softmax and accumulation are fp32; probabilities enter the
- * value product as fp16. Calls of at most 36 tokens whose tokens attend at most 64 x 32
- * rows each, and that fit the handle's partial buffer, spread each token's rows over
- * the GPU 32 at a time and merge the partial softmax results per token in a second
- * kernel (each unit's O and sum rescaled to the largest reference max, added in unit
- * order): a token's result then depends only on the token, not on the other tokens of
- * the call. Such calls use the handle's partial buffer, so two of them must not run
- * concurrently on one handle. */
+ * value product as fp16 (pv_mode 0) or as two fp16 terms (pv_mode 1). Calls of at most
+ * 36 tokens whose tokens attend at most 64 x 32 rows each, and that fit the handle's
+ * partial buffer, spread each token's rows over the GPU 32 at a time and merge the
+ * partial softmax results per token in a second kernel (each unit's O and sum rescaled
+ * to the largest reference max, added in unit order): a token's result then depends
+ * only on the token, not on the other tokens of the call. Such calls use the handle's
+ * partial buffer, so two of them must not run concurrently on one handle. */
 ds4sp_status ds4sp_sparse_attn(ds4sp_handle* h, const void* q, const void* kv_raw,
                                const void* kv_cmp, const int32_t* topk, int t0, int n_q,
                                float* out, void* stream);
@@ -222,7 +223,7 @@ ds4sp_status ds4sp_debug_fail_launches(ds4sp_handle* h, int n);
 ds4sp_status ds4sp_debug_set_mask(ds4sp_handle* h, const uint8_t* mask, int rows, int cols);
 
 /* Steps 1-2 like ds4sp_indexer_topk, for callers that cannot allocate device memory.
- * The paper has no counterpart to this entry point; it exists for the host side only.
+ * The pages have no counterpart to this entry point; it exists for the host side only.
  * Some callers cannot call cudaMalloc: a framework whose allocator reserves all device
  * memory up front (a raw cudaMalloc then fails or splits its pool), or a latency-bound
  * loop where cudaMalloc/cudaFree would synchronise the device. This entry point needs
