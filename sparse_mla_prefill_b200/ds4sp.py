@@ -144,6 +144,8 @@ def make_config(n_idx_heads: int, d_idx: int, top_k: int, n_swa: int, max_tokens
                 band: int = 2048, softmax_scale: float = 0.0, n_heads: int = 16, d_qk: int = 576,
                 d_v: int = 512, ratio: int = 4, exp_mode: int = 0,
                 pv_mode: int = 0) -> ds4sp_config:
+    """A ds4sp_config in field order. exp_mode: 0 = ex2.approx, 1 = exp2f for the
+    softmax; pv_mode: 0 = fp16 probabilities in P . V, 1 = fp32-staged (hi + lo fp16)."""
     return ds4sp_config(n_heads, d_qk, d_v, ratio, n_idx_heads, d_idx, top_k, n_swa, band,
                         max_tokens, softmax_scale, exp_mode, pv_mode)
 
