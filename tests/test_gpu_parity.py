@@ -117,6 +117,31 @@ def test_edge_cases(T, H_i, D_i, k, n_swa, band, scale):
     assert_attention_close(out.cpu().numpy(), ref["out"], f"edge T={T}")
 
 
+@pytest.mark.parametrize("T,k,band,tail", [(600, 16, 256, None), (16400, 64, 2048, 3)])
+def test_all_scores_equal(T, k, band, tail):
+    """Zero index weights make every score 0, so every candidate key is the same: the
+    select's all-keys-equal path must keep the k lowest rows (ties to the lower j). A
+    600-token prefill (256-thread top-k) and the last 3 tokens of a 16,400-token context
+    (rows of 4,100 scores: the 1,024-thread top-k, and few-token attention)."""
+    wl = Workload("ties", T=T, H_i=4, D_i=64, top_k=k, n_swa=16, seed=T, band=band)
+    inp = generate_small(T, 4, 64, seed=T + 2, weight_max=0)
+    if tail is None:
+        toks = list(range(T))
+        with handle_for(wl) as h:
+            topk, out = run_prefill(h, to_device(inp), T, k)
+    else:
+        t0 = T - tail
+        toks = list(range(t0, T))
+        dev = to_device({n: (v[t0:] if n in ("q", "q_idx", "w") else v) for n, v in inp.items()})
+        with handle_for(wl) as h:
+            topk, out = run_range(h, dev, t0, tail, k)
+    ref = oracle_tokens(_np(inp), toks, wl)
+    nv = (np.asarray(toks) + 1) // 4
+    assert (ref["topk"][nv >= k] == np.arange(k)).all()      # the lowest k rows
+    assert np.array_equal(topk.cpu().numpy(), ref["topk"])
+    assert_attention_close(out.cpu().numpy(), ref["out"], f"equal scores T={T}")
+
+
 def test_causal_reduction_against_sdpa():
     """k = 0 and n_swa >= T: the CUDA path equals causal attention (torch SDPA, float64)."""
     T = 160
