@@ -292,13 +292,38 @@ def pin_bands_equal_oneshot(o):
     assert np.array_equal(one["out"], bands["out"])
 
 
+def pin_prefill_tokens_composition(o, T: int = 120, s: int = 37):
+    """The whole path for a shuffled subset of tokens whose per-token inputs start at
+    q_start = s > 0 equals the pinned steps called one by one on the full arrays:
+    topk_row(indexer_scores_token(q_idx[t], k_idx, w[t], t)), then sparse_mla_attention
+    of token t alone (t0 = t). This fixes the offset between a token's position t and
+    its row t - s in the per-token arrays, and the order in which the steps compose."""
+    full = _np(generate_small(T, 4, 64, seed=41))
+    sliced = dict(full)
+    for name in ("q", "q_idx", "w"):
+        sliced[name] = full[name][s:]
+    rng = np.random.default_rng(6)
+    toks = [int(t) for t in rng.permutation(np.arange(s, T))[:40]]
+    k, n_swa = 6, 9
+    got = o.prefill_tokens(sliced, toks, top_k=k, n_swa=n_swa, q_start=s)
+    assert got["tokens"].tolist() == toks
+    assert got["topk"].shape == (len(toks), k) and got["out"].shape == (len(toks), 16, 512)
+    for n, t in enumerate(toks):
+        sc = o.indexer_scores_token(full["q_idx"][t], full["k_idx"], full["w"][t], t)
+        idx = o.topk_row(sc, k)
+        assert np.array_equal(got["topk"][n], idx), t
+        want = o.sparse_mla_attention(full["q"][t:t + 1], full["kv_raw"], full["kv_cmp"],
+                                      idx[None], t, n_swa)
+        assert np.array_equal(got["out"][n], want[0]), t
+
+
 ALL_PINS = [
     pin_visibility_mask, pin_visibility_golden,
     pin_scores_exact, pin_scores_relu_identities, pin_scores_bruteforce,
     pin_topk_golden, pin_topk_bruteforce, pin_topk_masked_bruteforce,
     pin_attention_sdpa_causal, pin_attention_sdpa_window, pin_attention_dense_mask,
     pin_attention_bruteforce, pin_attention_closed_forms,
-    pin_bands_equal_oneshot,
+    pin_bands_equal_oneshot, pin_prefill_tokens_composition,
 ]
 
 

@@ -112,6 +112,35 @@ def _mut_masked_ties_by_candidate_rank(o):
     o.topk_row_masked = f
 
 
+def _prefill_with(o, attend_pos, q_row):
+    """prefill_tokens rebuilt with a planted offset mistake: `attend_pos(t, i)` is the
+    position handed to attended_rows, `q_row(t, i)` the per-token row read."""
+    def f(inputs, tokens, top_k, n_swa, q_start=0, scale=None, d_v=512, ratio=4):
+        tokens = list(tokens)
+        q, q_idx, w = inputs["q"], inputs["q_idx"], inputs["w"]
+        sc = o.default_scale(q.shape[2]) if scale is None else scale
+        idx = np.zeros((len(tokens), top_k), dtype=np.int32)
+        out = np.zeros((len(tokens), q.shape[1], d_v))
+        for n, t in enumerate(tokens):
+            i = t - q_start
+            r = q_row(t, i)
+            idx[n] = o.topk_row(o.indexer_scores_token(q_idx[r], inputs["k_idx"], w[r], t, ratio), top_k)
+            rows = o.attended_rows(attend_pos(t, i), idx[n], inputs["kv_raw"], inputs["kv_cmp"], n_swa)
+            out[n] = o.attention_token(q[r], rows, sc, d_v)
+        return {"tokens": np.asarray(tokens, dtype=np.int64), "topk": idx, "out": out}
+    return f
+
+
+def _mut_prefill_window_at_row(o):
+    # The attended rows taken at the token's row i = t - q_start instead of its position t.
+    o.prefill_tokens = _prefill_with(o, lambda t, i: i, lambda t, i: i)
+
+
+def _mut_prefill_inputs_at_position(o):
+    # Per-token inputs read at the position t instead of the row t - q_start.
+    o.prefill_tokens = _prefill_with(o, lambda t, i: t, lambda t, i: t)
+
+
 MUTATIONS = [
     (_mut_visibility_first_token, [P.pin_visibility_mask, P.pin_visibility_golden]),
     (_mut_no_relu, [P.pin_scores_exact, P.pin_scores_relu_identities, P.pin_scores_bruteforce]),
@@ -125,7 +154,17 @@ MUTATIONS = [
     (_mut_window_excludes_self, [P.pin_attention_sdpa_causal, P.pin_attention_sdpa_window]),
     (_mut_scale_ignored, [P.pin_attention_sdpa_causal, P.pin_attention_bruteforce]),
     (_mut_dedup_window, [P.pin_attention_dense_mask, P.pin_attention_closed_forms]),
+    (_mut_prefill_window_at_row, [P.pin_prefill_tokens_composition]),
+    (_mut_prefill_inputs_at_position, [P.pin_prefill_tokens_composition]),
 ]
+
+
+def test_offset_harness_without_mistake_passes():
+    """The rebuilt prefill_tokens used by the offset mutations passes the pin when given
+    the right offsets, so those mutations fail for their planted mistake alone."""
+    o = fresh_oracle()
+    o.prefill_tokens = _prefill_with(o, lambda t, i: t, lambda t, i: i)
+    P.pin_prefill_tokens_composition(o)
 
 
 @pytest.mark.parametrize("mutate,pins", MUTATIONS, ids=[m[0].__name__ for m in MUTATIONS])
