@@ -82,12 +82,13 @@ typedef struct {
                             1 = fp32-staged: P = hi + lo, two fp16 terms (hi = fp16(p),
                             lo = fp16(p - hi)), about 22 significant bits, at twice the
                             P . V tensor work ("FP32-staged streaming MLA" of "perf(ds4):
-                            extend sparse prefill scheduling to 10K"); other values are
-                            DS4SP_ERR_INVALID_ARG */
+                            unify gfx1151 sparse-prefill stack", Validation completed);
+                            other values are DS4SP_ERR_INVALID_ARG */
 } ds4sp_config;
 
 /* Validate cfg and create a handle bound to the current CUDA device. The handle owns
- * a 4-byte device status word, the partial-result buffer of few-token attention calls
+ * two device words (the status word and the abort word of the kernels' bounded waits),
+ * the partial-result buffer of few-token attention calls
  * (2 x SMs x 16 x 512 fp32 plus 2 x SMs x 32 fp32: about 9.7 MB on a 148-SM B200) and
  * some host state. *out is NULL on error. */
 ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out);
@@ -201,6 +202,18 @@ ds4sp_status ds4sp_profile_read(ds4sp_handle* h, double ms[3], int launches[3]);
  * not made, and the call that would make them returns DS4SP_ERR_CUDA. */
 ds4sp_status ds4sp_debug_fail_launches(ds4sp_handle* h, int n);
 
+/* Bounded waits, for tests of the give-up path. Every pipeline wait inside the kernels
+ * (one role waiting for another through a shared-memory barrier) gives up after a limit,
+ * by default 1,000,000,000 ns (about one second); the kernel then records bit 1 of the
+ * status word, every other wait of the same launch gives up at once, and the launch
+ * returns with its outputs undefined. Waits for copies and tensor-core work a thread
+ * issued itself, before the memory they write is released, keep the default limit
+ * whatever is set here (they complete on their own). A give-up in one launch does not
+ * shorten the waits of later launches.
+ *   ns  the limit for this handle's later launches, in nanoseconds; 0 = give up at the
+ *       first wait that is not already complete; negative = back to the default. */
+ds4sp_status ds4sp_debug_set_wait_limit_ns(ds4sp_handle* h, long long ns);
+
 /* Explicit-mask visibility, a debug form of the path for the "explicit-mask versus
  * analytic-mask" oracle check ("perf(ds4): extend sparse prefill scheduling to 10K",
  * Qualification). While a mask is set, the top-k and the attention take the visibility
@@ -234,7 +247,8 @@ ds4sp_status ds4sp_debug_set_mask(ds4sp_handle* h, const uint8_t* mask, int rows
  *   q_idx, k_idx, w, t0, n_q, topk, stream  as for ds4sp_indexer_topk.
  * n_q * ld must be <= 2^21, with ld = n_vis(t0+n_q-1) rounded up to 4 (for example, a
  * 2048-token band whose last token sees up to 1024 rows, or up to 5 tokens at a
- * 122,880-token context); larger ranges return DS4SP_ERR_WORKSPACE before any launch.
+ * 122,880-token context); larger ranges return DS4SP_ERR_WORKSPACE. Every argument error
+ * is returned before any work is queued.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  * with that device current; make that first call before any stream capture. All calls
  * share the one array, which keeps the last call's scores: calls whose kernels overlap on

@@ -11,9 +11,14 @@ namespace ds4sp {
 constexpr uint32_t kStatusBounds = 1u;   // an index was out of range and skipped
 constexpr uint32_t kStatusTimeout = 2u;  // a bounded wait gave up
 
-// A wait gives up after this many nanoseconds of the global timer (about one
-// second): far above any legitimate wait inside one of these kernels.
+// Default limit of a pipeline wait, in nanoseconds of the global timer (about one
+// second): far above any legitimate wait inside one of these kernels. A handle can
+// lower it for tests (ds4sp_debug_set_wait_limit_ns).
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+// Limit of a drain wait (an issued bulk copy or committed MMA landing before the CTA
+// releases the memory it writes). Those complete on their own, so a drain wait is
+// bounded by time alone: never by a lowered limit and never by another CTA giving up.
+constexpr unsigned long long kDrainLimitNs = 1000000000ull;
 
 __device__ __forceinline__ void record_status(uint32_t* status, uint32_t bits) {
     if (status) atomicOr(status, bits);
@@ -62,26 +67,59 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase of the given parity to complete, giving up after
-// kWaitLimitNs. Returns false (and records kStatusTimeout) when it gives up.
-// Once `abort` is set, returns false at once, so every role drains quickly.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* status,
+// How the pipeline waits of one launch give up. `abort_word` is shared by every launch
+// of a handle; a wait that gives up writes this launch's `epoch` (never 0, new for
+// every launch) into it, and a wait of the same launch that sees its own epoch there
+// gives up at once, so that every role of every CTA drains quickly. A word left by an
+// earlier launch holds another epoch and is ignored: one launch's give-up never
+// shortens the waits of a later one.
+struct WaitCtl {
+    uint32_t* status;              // device status word (kStatusTimeout is recorded here)
+    uint32_t* abort_word;          // may be NULL: no cross-CTA signal
+    uint32_t epoch;
+    unsigned long long limit_ns;   // 0: give up at the first miss
+};
+
+__device__ __forceinline__ bool launch_gave_up(const WaitCtl& w) {
+    return w.abort_word && *reinterpret_cast<volatile uint32_t*>(w.abort_word) == w.epoch;
+}
+
+__device__ __forceinline__ void give_up(const WaitCtl& w) {
+    record_status(w.status, kStatusTimeout);
+    if (w.abort_word) *reinterpret_cast<volatile uint32_t*>(w.abort_word) = w.epoch;
+}
+
+// Wait for the phase of the given parity to complete. Gives up (returns false, records
+// kStatusTimeout and sets `abort`) once w.limit_ns has passed since the first miss, or
+// as soon as another wait of the same launch has given up. Once `abort` is set it
+// returns false at once, so every role drains quickly.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& w,
                                           bool& abort) {
     if (abort) return false;
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (true) {
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
-        // Give up after the limit, or at once if another CTA of the grid already gave up.
-        const bool other_gave_up =
-            status && (*reinterpret_cast<volatile uint32_t*>(status) & kStatusTimeout);
-        if (other_gave_up || global_ns() - t0 > kWaitLimitNs) {
-            record_status(status, kStatusTimeout);
+        if (launch_gave_up(w) || global_ns() - t0 >= w.limit_ns) {
+            give_up(w);
             abort = true;
             return false;
         }
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
     }
+}
+
+// Wait for a phase that completes without any other role's help (bulk copies this
+// thread issued, MMAs it committed), before the memory they write is released. Bounded
+// by kDrainLimitNs only; records kStatusTimeout if even that runs out.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, const WaitCtl& w) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (global_ns() - t0 < kDrainLimitNs)
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+    record_status(w.status, kStatusTimeout);
+    return false;
 }
 
 // ---------------------------------------------------------------- cp.async

@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <new>
 #include <string>
@@ -56,7 +57,11 @@ struct ds4sp_handle {
     ds4sp_config cfg;
     int device = 0;
     int sm_count = 148;
+    // Device words: [0] the status word ds4sp_device_status reads, [1] the abort word of
+    // the kernels' bounded waits (see WaitCtl).
     uint32_t* d_status = nullptr;
+    uint32_t epoch = 0;                                  // of the last launch
+    unsigned long long wait_limit_ns = kWaitLimitNs;     // ds4sp_debug_set_wait_limit_ns
     cudaEvent_t last = nullptr;
     int next_band = 0;
     int fail_launches = 0;
@@ -92,6 +97,35 @@ struct TraceRange {
 
 int nvis(int t, int ratio) { return (t + 1) / ratio; }
 
+// The bounded-wait settings of the handle's next launch, with a fresh epoch.
+WaitCtl next_wait(ds4sp_handle* h) {
+    if (++h->epoch == 0) h->epoch = 1;   // epoch 0 would match a cleared abort word
+    return WaitCtl{h->d_status, h->d_status + 1, h->epoch, h->wait_limit_ns};
+}
+
+constexpr int kMaxDevices = 64;
+
+// cudaFuncSetAttribute(kernel, max dynamic shared memory) once per (device, kernel): the
+// attribute belongs to the device's copy of the function.
+ds4sp_status set_smem_once(ds4sp_handle* h, const void* fn, int bytes, int slot, const char* what) {
+    static std::mutex mu;
+    static bool done[kMaxDevices][16] = {};
+    if (h->device < 0 || h->device >= kMaxDevices || slot < 0 || slot >= 16)
+        return fail(DS4SP_ERR_UNSUPPORTED, "device %d", h->device);
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[h->device][slot]) return DS4SP_OK;
+    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    done[h->device][slot] = true;
+    return DS4SP_OK;
+}
+
+// Slot of an indexer instantiation in set_smem_once's table: D_i in {64, 128} x H_i in
+// {4, 8, 16, 32, 64}.
+constexpr int indexer_slot(int d_idx, int h_idx) {
+    return (d_idx == 128 ? 5 : 0) + (h_idx == 4 ? 0 : h_idx == 8 ? 1 : h_idx == 16 ? 2 : h_idx == 32 ? 3 : 4);
+}
+
 int score_ld(int t_last, int ratio) {
     const int nv = nvis(t_last, ratio);
     return ((nv > 0 ? nv : 1) + 3) / 4 * 4;
@@ -100,6 +134,12 @@ int score_ld(int t_last, int ratio) {
 float scale_of(const ds4sp_config& c) {
     return c.softmax_scale > 0.f ? c.softmax_scale : 1.0f / std::sqrt((float)c.d_qk);
 }
+
+#define DS4SP_TRY(x)                      \
+    do {                                  \
+        const ds4sp_status s_ = (x);      \
+        if (s_ != DS4SP_OK) return s_;    \
+    } while (0)
 
 cudaEvent_t pooled_event(ds4sp_handle* h) {
     if (!h->event_pool.empty()) {
@@ -185,18 +225,12 @@ ds4sp_status launch_indexer(ds4sp_handle* h, const void* q_idx, const void* k_id
     if (!make_tmap_2d(&tk, k_idx, D_I, n_rows, C::BM) ||
         !make_tmap_2d(&tq, q_idx, D_I, n_q * H_I, C::BN))
         return fail(DS4SP_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-    static bool attr_done[2][65] = {};  // per instantiation; the attribute is per function
-    if (!attr_done[D_I / 128][H_I]) {
-        const cudaError_t e = cudaFuncSetAttribute(indexer_tcgen05_kernel<D_I, H_I>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   C::SMEM_BYTES);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(indexer)");
-        attr_done[D_I / 128][H_I] = true;
-    }
+    DS4SP_TRY(set_smem_once(h, reinterpret_cast<const void*>(indexer_tcgen05_kernel<D_I, H_I>),
+                            C::SMEM_BYTES, indexer_slot(D_I, H_I), "cudaFuncSetAttribute(indexer)"));
     IndexerParams p;
     p.w = w;
     p.scores = scores;
-    p.status = h->d_status;
+    p.wc = next_wait(h);
     p.t0 = t0;
     p.n_q = n_q;
     p.ld = ld;
@@ -334,7 +368,7 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
     p.kv_cmp = static_cast<const __half*>(kv_cmp);
     p.topk = topk;
     p.out = out;
-    p.status = h->d_status;
+    p.wc = next_wait(h);
     p.t0 = t0;
     p.n_q = n_q;
     p.k = h->cfg.top_k;
@@ -413,11 +447,6 @@ ds4sp_status check_ptr(const void* p, const char* name) {
     return DS4SP_OK;
 }
 
-#define DS4SP_TRY(x)                      \
-    do {                                  \
-        const ds4sp_status s_ = (x);      \
-        if (s_ != DS4SP_OK) return s_;    \
-    } while (0)
 
 ds4sp_status record_last(ds4sp_handle* h, cudaStream_t stream) {
     const cudaError_t e = cudaEventRecord(h->last, stream);
@@ -523,8 +552,8 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
     cudaError_t e = cudaGetDevice(&h->device);
     if (e == cudaSuccess)
         e = cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, h->device);
-    if (e == cudaSuccess) e = cudaMalloc(&h->d_status, sizeof(uint32_t));
-    if (e == cudaSuccess) e = cudaMemset(h->d_status, 0, sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMalloc(&h->d_status, 2 * sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMemset(h->d_status, 0, 2 * sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->last, cudaEventDisableTiming);
     // Partials of split-mode attention (calls of few tokens): two 32-row units per SM.
     if (e == cudaSuccess) {
@@ -837,6 +866,12 @@ ds4sp_status ds4sp_debug_fail_launches(ds4sp_handle* h, int n) {
     return DS4SP_OK;
 }
 
+ds4sp_status ds4sp_debug_set_wait_limit_ns(ds4sp_handle* h, long long ns) {
+    DS4SP_TRY(check_handle(h));
+    h->wait_limit_ns = ns < 0 ? kWaitLimitNs : (unsigned long long)ns;
+    return DS4SP_OK;
+}
+
 ds4sp_status ds4sp_debug_set_mask(ds4sp_handle* h, const uint8_t* mask, int rows, int cols) {
     DS4SP_TRY(check_handle(h));
     if (mask == nullptr) {
@@ -887,13 +922,14 @@ __device__ __align__(256) uint32_t g_static_status[4];
 
 struct StaticScratch {
     float* scores = nullptr;
-    uint32_t* status = nullptr;
+    uint32_t* status = nullptr;   // [0] status word, [1] abort word of the bounded waits
+    int device = 0;
     int sm_count = 0;
     bool ready = false;
 };
 
-constexpr int kMaxDevices = 64;
 StaticScratch g_static[kMaxDevices];
+std::atomic<uint32_t> g_static_epoch{0};
 std::mutex g_static_mu;
 
 // Device addresses of the static arrays on the current device (set-up on first use).
@@ -911,6 +947,7 @@ ds4sp_status static_scratch(StaticScratch* out) {
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
         e = cudaDeviceGetAttribute(&s.sm_count, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        s.device = dev;
         s.ready = true;
     }
     *out = s;
@@ -949,28 +986,31 @@ extern "C" ds4sp_status ds4sp_indexer_topk_noalloc(const ds4sp_config* cfg, cons
         return fail(DS4SP_ERR_WORKSPACE,
                     "%d tokens x %d score columns exceed the static scratch of %zu floats (8 MiB)",
                     n_q, ld, kStaticScoreFloats);
+    const int t_last = t0 + n_q - 1;
+    DS4SP_TRY(check_ptr(q_idx, "q_idx"));
+    if (nvis(t_last, cfg->ratio) > 0) DS4SP_TRY(check_ptr(k_idx, "k_idx"));
+    DS4SP_TRY(check_ptr(w, "w"));
+    DS4SP_TRY(check_ptr(topk, "topk"));
+    if (nvis(t_last, cfg->ratio) > kMaxTopkCandidates)
+        return fail(DS4SP_ERR_UNSUPPORTED, "%d candidate rows exceed the top-k limit %d",
+                    nvis(t_last, cfg->ratio), kMaxTopkCandidates);
     StaticScratch sc;
     DS4SP_TRY(static_scratch(&sc));
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // The status word steers the kernels' bounded waits, so each call starts it at zero.
-    const cudaError_t e = cudaMemsetAsync(sc.status, 0, sizeof(uint32_t), s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
-    // A handle on the stack carries the launch settings; it owns no device memory.
+    // A handle on the stack carries the launch settings; it owns no device memory. Its
+    // status and abort words are the library's static ones; each call takes fresh wait
+    // epochs, so a give-up in an earlier call never shortens this call's waits.
     ds4sp_handle tmp;
     tmp.cfg = *cfg;
+    tmp.device = sc.device;
     tmp.d_status = sc.status;
     tmp.sm_count = sc.sm_count;
-    ds4sp_status st = DS4SP_OK;
-    const int t_last = t0 + n_q - 1;
-    st = check_ptr(q_idx, "q_idx");
-    if (st == DS4SP_OK && nvis(t_last, cfg->ratio) > 0) st = check_ptr(k_idx, "k_idx");
-    if (st == DS4SP_OK) st = check_ptr(w, "w");
-    if (st == DS4SP_OK) st = check_ptr(topk, "topk");
-    if (st == DS4SP_OK && nvis(t_last, cfg->ratio) > kMaxTopkCandidates)
-        st = fail(DS4SP_ERR_UNSUPPORTED, "%d candidate rows exceed the top-k limit %d",
-                  nvis(t_last, cfg->ratio), kMaxTopkCandidates);
-    if (st != DS4SP_OK) return st;
-    st = cfg->d_idx == 64
+    tmp.epoch = g_static_epoch.fetch_add(16);
+    // The status word is internal to this entry point; clear it once the arguments
+    // have passed every check.
+    const cudaError_t e = cudaMemsetAsync(sc.status, 0, sizeof(uint32_t), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+    ds4sp_status st = cfg->d_idx == 64
              ? dispatch_indexer_h<64>(&tmp, q_idx, k_idx, w, t0, n_q, sc.scores, ld, s)
              : dispatch_indexer_h<128>(&tmp, q_idx, k_idx, w, t0, n_q, sc.scores, ld, s);
     if (st != DS4SP_OK) return st;

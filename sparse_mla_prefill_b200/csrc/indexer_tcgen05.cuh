@@ -65,7 +65,7 @@ constexpr int kIndexerMaxGrid = 160;
 struct IndexerParams {
     const float* w;        // [n_q, H_i] fp32, row 0 = token t0
     float* scores;         // [n_q, ld] fp32 scratch
-    uint32_t* status;      // device status word
+    WaitCtl wc;            // bounded waits of this launch
     int t0, n_q, ld, ratio;
     int n_tb;              // token blocks of TB tokens
     // CTA b's share: count[b] consecutive (token block, j-tile) pairs from token block
@@ -190,7 +190,7 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             IndexerUnit w;
             while (!abort && wk.next<C::TB>(p, w)) {
                 const int bb = bi & 1;
-                if (!mbar_wait(bempty(bb), ((bi >> 1) & 1) ^ 1, p.status, abort)) break;
+                if (!mbar_wait(bempty(bb), ((bi >> 1) & 1) ^ 1, p.wc, abort)) break;
                 mbar_arrive_expect_tx(bfull(bb), C::B_BYTES);
                 for (int ks = 0; ks < C::KSUB; ++ks)
                     tma_load_2d(base + C::OFF_B + bb * C::B_BYTES + ks * C::B_SUB, &tmap_q,
@@ -198,11 +198,10 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 ++b_issued[bb];
                 ++bi;
             }
-            // Every bulk copy this CTA started must land before the CTA exits.
-            for (int i = 0; i < 2; ++i) {
-                bool d = false;
-                if (b_issued[i]) mbar_wait(bfull(i), (b_issued[i] - 1) & 1, p.status, d);
-            }
+            // Every bulk copy this CTA started must land before the CTA exits (a drain
+            // wait: the copies complete on their own, whatever the other roles did).
+            for (int i = 0; i < 2; ++i)
+                if (b_issued[i]) mbar_wait_drain(bfull(i), (b_issued[i] - 1) & 1, p.wc);
         } else if (warp == 0 && lane == 0) {
             int a_it = 0;
             int a_issued[C::A_STAGES] = {};
@@ -211,7 +210,7 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             while (!abort && wk.next<C::TB>(p, w)) {
                 for (int it = 0; it < w.n_tiles; ++it, ++a_it) {
                     const int s = a_it % C::A_STAGES;
-                    if (!mbar_wait(aempty(s), ((a_it / C::A_STAGES) & 1) ^ 1, p.status, abort))
+                    if (!mbar_wait(aempty(s), ((a_it / C::A_STAGES) & 1) ^ 1, p.wc, abort))
                         break;
                     mbar_arrive_expect_tx(afull(s), C::A_STAGE);
 #pragma unroll
@@ -221,10 +220,8 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     ++a_issued[s];
                 }
             }
-            for (int s = 0; s < C::A_STAGES; ++s) {
-                bool d = false;
-                if (a_issued[s]) mbar_wait(afull(s), (a_issued[s] - 1) & 1, p.status, d);
-            }
+            for (int s = 0; s < C::A_STAGES; ++s)
+                if (a_issued[s]) mbar_wait_drain(afull(s), (a_issued[s] - 1) & 1, p.wc);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -239,12 +236,12 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             IndexerUnit w;
             while (!abort && wk.next<C::TB>(p, w)) {
                 const int bb = bi & 1;
-                if (!mbar_wait(bfull(bb), (bi >> 1) & 1, p.status, abort)) break;
+                if (!mbar_wait(bfull(bb), (bi >> 1) & 1, p.wc, abort)) break;
                 const uint64_t b_desc = b_desc0 + (uint64_t)((bb * C::B_BYTES) >> 4);
                 for (int it = 0; it < w.n_tiles; ++it, ++tc) {
                     const int buf = tc & 1, s = tc % C::A_STAGES;
-                    if (!mbar_wait(tempty(buf), ((tc >> 1) & 1) ^ 1, p.status, abort)) break;
-                    if (!mbar_wait(afull(s), (tc / C::A_STAGES) & 1, p.status, abort)) break;
+                    if (!mbar_wait(tempty(buf), ((tc >> 1) & 1) ^ 1, p.wc, abort)) break;
+                    if (!mbar_wait(afull(s), (tc / C::A_STAGES) & 1, p.wc, abort)) break;
                     tc_fence_after();
                     const uint32_t d = tmem_base + buf * C::BN;
                     const uint64_t a_desc = a_desc0 + (uint64_t)((s * C::A_STAGE) >> 4);
@@ -262,10 +259,10 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 umma_commit(bempty(bb));                 // B buffer free once the unit's MMAs finish
                 ++bi;
             }
-            // All MMAs issued by this thread must finish before TMEM is released.
+            // All MMAs issued by this thread must finish before TMEM is released (a
+            // drain wait: committed MMAs complete on their own).
             umma_commit(done_bar);
-            bool d = false;
-            mbar_wait(done_bar, 0, p.status, d);
+            mbar_wait_drain(done_bar, 0, p.wc);
         }
         __syncwarp();
     } else {
@@ -303,8 +300,11 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const int buf = tc & 1;
                 // The tile's A-stage barrier completes when its MMAs do.
                 const bool ready = mbar_wait(aempty(tc % C::A_STAGES), (tc / C::A_STAGES) & 1,
-                                             p.status, abort);
-                if (!__all_sync(0xffffffffu, ready)) continue;   // warp-uniform skip
+                                             p.wc, abort);
+                if (!__all_sync(0xffffffffu, ready)) {           // warp-uniform skip
+                    abort = true;
+                    continue;
+                }
                 tc_fence_after();
                 const int j = w.jt(it) * C::BM + quarter * 32 + lane;
                 // All 128 columns of this warp into registers, then release the accumulator

@@ -115,7 +115,7 @@ struct AttnParams {
     const __half* kv_cmp;  // [>= n_vis(t0+n_q-1), 576]
     const int32_t* topk;   // [n_q, k]
     float* out;            // [n_q, 16, 512]
-    uint32_t* status;
+    WaitCtl wc;            // bounded waits of this launch; wc.status also takes index errors
     int t0, n_q, k, n_swa, ratio;
     float scale_log2;      // softmax scale * log2(e)
     // Optional: a region the next kernel will read (the next band's indexer queries);
@@ -277,33 +277,39 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         named_barrier(PRODUCER_BAR, PTHREADS);
         MergedCursor mc;
         mc.start(p);
+        // A producer warp whose wait gives up stops copying but keeps walking the units
+        // (its waits then return at once), so that it still meets every producer barrier
+        // that the other producer warps reach.
         for (int uc = 0; mc.valid(); ++uc, mc.advance(p)) {
             const int s = uc % NS;
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait(empty_bar(s), ((uc / NS) & 1) ^ 1, p.status, abort)))
-                break;
+            if (!abort &&
+                !__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ((uc / NS) & 1) ^ 1, p.wc, abort)))
+                abort = true;                      // the whole warp gives up together
             const uint32_t dst = sbase + OFF_RING + s * SLOT;
             const GroupCursor cu = mc.group(mc.turn);
             if (cu.u == 0) {
-                // Q of the token, and the group's next top-k row one token ahead.
-                stage_idx(mc.turn, cu.m + 1);
-                const __half* qt = p.q + (size_t)cu.tr.i * H * DQK;
+                if (!abort) {
+                    // Q of the token, and the group's next top-k row one token ahead.
+                    stage_idx(mc.turn, cu.m + 1);
+                    const __half* qt = p.q + (size_t)cu.tr.i * H * DQK;
 #pragma unroll
-                for (int m = 0; m < H * CH / PTHREADS; ++m) {
-                    const int e = ptid + m * PTHREADS, r = e / CH, ch = e % CH;
-                    cp_async_16(chunk_addr(dst, r, ch), qt + r * DQK + ch * 8, true);
+                    for (int m = 0; m < H * CH / PTHREADS; ++m) {
+                        const int e = ptid + m * PTHREADS, r = e / CH, ch = e % CH;
+                        cp_async_16(chunk_addr(dst, r, ch), qt + r * DQK + ch * 8, true);
+                    }
+                    cp_async_commit();
+                    cp_async_arrive_noinc(full_bar(s));
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(full_bar(s));
+                    // This token's top-k row (staged at the group's previous Q unit, an
+                    // earlier commit group) must be in shared memory, for every producer
+                    // thread, before its row units are resolved.
+                    cp_async_wait<1>();
                 }
-                cp_async_commit();
-                cp_async_arrive_noinc(full_bar(s));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(full_bar(s));
-                // This token's top-k row (staged at the group's previous Q unit, an earlier
-                // commit group) must be in shared memory, for every producer thread,
-                // before its row units are resolved.
-                cp_async_wait<1>();
                 named_barrier(PRODUCER_BAR, PTHREADS);
                 continue;
             }
+            if (abort) continue;
             const int* tk = reinterpret_cast<const int*>(smem + idx_buf(mc.turn, cu.m));
             const int r = 8 * pw + (lane >> 2);   // this lane's row of the unit
             const int gr = (cu.tr.u0 + cu.u - 1) * BR + r;
@@ -316,7 +322,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                         row = p.kv_cmp + (size_t)j * DQK;
                         ok = true;
                     } else if ((lane & 3) == 0) {
-                        record_status(p.status, kStatusBounds);
+                        record_status(p.wc.status, kStatusBounds);
                     }
                 } else if (j >= 0 && j < p.mask_cols) {
                     if (p.vis_mask[(size_t)cu.tr.t * p.mask_ld + j] != 0) {
@@ -324,7 +330,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                         ok = true;
                     }
                 } else if (j != -1 && (lane & 3) == 0) {
-                    record_status(p.status, kStatusBounds);
+                    record_status(p.wc.status, kStatusBounds);
                 }
             } else if (gr < cu.tr.nrows) {
                 row = p.kv_raw + (size_t)(cu.tr.s_lo + gr - cu.tr.nsel) * DQK;
@@ -380,7 +386,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         float m_g = -INFINITY, m_g8 = -INFINITY; // reference max, heads g and g+8 (log2 units)
         float l_g = 0.f, l_g8 = 0.f;             // this warp's share of the softmax sums
         auto wait_full = [&](int q) {
-            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(q % NS), (q / NS) & 1, p.status, abort)))
+            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(q % NS), (q / NS) & 1, p.wc, abort)))
                 flags[2] = 1;
         };
         MergedCursor mc;

@@ -61,6 +61,7 @@ _SIGS = {
     "ds4sp_profile_read": (_i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i32)]),
     "ds4sp_debug_fail_launches": (_i32, [_vp, _i32]),
     "ds4sp_debug_set_mask": (_i32, [_vp, _vp, _i32, _i32]),
+    "ds4sp_debug_set_wait_limit_ns": (_i32, [_vp, ctypes.c_longlong]),
     "ds4sp_indexer_topk_noalloc": (_i32, [ctypes.POINTER(ds4sp_config), _vp, _vp, _vp, _i32,
                                           _i32, _vp, _vp]),
     "ds4sp_status_string": (ctypes.c_char_p, [_i32]),
@@ -245,6 +246,13 @@ def ds4sp_profile_read(h: Handle) -> Dict[str, Tuple[float, int]]:
 
 def ds4sp_debug_fail_launches(h: Handle, n: int) -> None:
     _check(load_library().ds4sp_debug_fail_launches(h.ptr, n), "ds4sp_debug_fail_launches")
+
+
+def ds4sp_debug_set_wait_limit_ns(h: Handle, ns: int) -> None:
+    """Limit of the kernels' pipeline waits for this handle's later launches (ns; 0 =
+    give up at the first miss; negative = back to the default of about one second)."""
+    _check(load_library().ds4sp_debug_set_wait_limit_ns(h.ptr, int(ns)),
+           "ds4sp_debug_set_wait_limit_ns")
 
 
 def ds4sp_debug_set_mask(h: Handle, mask: Optional[torch.Tensor]) -> None:

@@ -1,8 +1,8 @@
 """fp32-staged probabilities in P . V (pv_mode 1) against the default fp16 P.
 
-"perf(ds4): extend sparse prefill scheduling to 10K" compares an FP32-staged
-streaming MLA with fast exponentials against the precise path (its summary gives
-NMSE 1.97e-14). Here pv_mode 1 carries each probability as two fp16 terms
+"perf(ds4): unify gfx1151 sparse-prefill stack", Validation completed, compares an
+FP32-staged streaming MLA with fast exponentials against the precise path (NMSE
+1.97e-14). Here pv_mode 1 carries each probability as two fp16 terms
 (hi + lo), about 22 significant bits, so P . V loses no more than fp32 rounding.
 
 Bar for pv_mode 1 against the float64 oracle, derived from the arithmetic: logits
