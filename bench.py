@@ -161,25 +161,43 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ reference arm (oracle)
 
-def cpu_oracle_sample(wl, n_sample, inputs_np=None, return_result=False):
+def blas_threads():
+    """Threads NumPy's BLAS runs the oracle's matrix products on."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return torch.get_num_threads()
+
+
+def cpu_oracle_sample(wl, n_sample, inputs_np=None, return_result=False, one_core=False):
     """Time the float64 CPU oracle on a spread sample of tokens; tokens/s (and, with
-    return_result, the oracle's indices and outputs for those tokens)."""
+    return_result, the oracle's indices and outputs for those tokens). one_core limits
+    NumPy's BLAS to one thread for the timing."""
+    import contextlib
     import oracle
     if inputs_np is None:
         inputs_np = {k: v.numpy() for k, v in generate(wl).items()}
     stride = max(1, wl.T // n_sample)
     toks = list(range(stride - 1, wl.T, stride))[:n_sample]
-    t0 = time.perf_counter()
-    ref = oracle.prefill_tokens(inputs_np, toks, wl.top_k, wl.n_swa)
-    dt = time.perf_counter() - t0
-    line = {"value": len(toks) / dt, "unit": "tokens/s", "cores": torch.get_num_threads(),
+    ctx = contextlib.nullcontext()
+    if one_core:
+        from threadpoolctl import threadpool_limits
+        ctx = threadpool_limits(limits=1)
+    with ctx:
+        cores = 1 if one_core else blas_threads()
+        t0 = time.perf_counter()
+        ref = oracle.prefill_tokens(inputs_np, toks, wl.top_k, wl.n_swa)
+        dt = time.perf_counter() - t0
+    line = {"value": len(toks) / dt, "unit": "tokens/s", "cores": cores,
             "kind": "oracle",
             "sample": f"{len(toks)} of {wl.T} tokens (every {stride}th), float64 NumPy, "
                       f"{dt:.1f} s"}
     return (line, ref) if return_result else line
 
 
-def sampled_parity(ref, topk_gpu, out_gpu):
+def sampled_parity(ref, topk_gpu, out_gpu, of="ds4sp_prefill_host result (pinned host buffers)"):
     """The end-to-end result against the oracle on its sampled tokens: indices bit for
     bit, attention max-abs and NMSE over every element of those tokens."""
     import numpy as np
@@ -191,8 +209,7 @@ def sampled_parity(ref, topk_gpu, out_gpu):
     exact = bool(np.array_equal(topk_gpu[toks], ref["topk"]))
     return {"tokens": int(len(toks)), "topk_bit_exact": exact, "max_abs": max_abs, "nmse": nmse,
             "bar": {"max_abs": 2e-3, "nmse": 1e-6},
-            "pass": exact and max_abs <= 2e-3 and nmse <= 1e-6,
-            "of": "ds4sp_prefill_host result (pinned host buffers)"}
+            "pass": exact and max_abs <= 2e-3 and nmse <= 1e-6, "of": of}
 
 
 def run_reference(args, rank, world):
@@ -274,6 +291,64 @@ def verify_latency(dev, reps: int = 50):
             "unit": "us per step (indexer + top-k + attention)", **res}
 
 
+def config_throughput(name, dev, steps, stream):
+    """tokens/s of one prefill workload (device-resident inputs, `steps` whole prefills
+    between CUDA events on the launching stream); returns the line and the last result."""
+    wl = workload(name)
+    host = generate(wl)
+    inputs = {k: v.to(dev) for k, v in host.items()}
+    cfg = D.make_config(n_idx_heads=wl.H_i, d_idx=wl.D_i, top_k=wl.top_k, n_swa=wl.n_swa,
+                        max_tokens=wl.T, band=wl.band)
+    h = D.ds4sp_create(cfg)
+    try:
+        topk = torch.empty((wl.T, wl.top_k), dtype=torch.int32, device=dev)
+        out = torch.empty((wl.T, 16, 512), dtype=torch.float32, device=dev)
+        ws = D.band_workspace(h, wl.T, dev)
+        for _ in range(3):
+            D.prefill(h, inputs, wl.T, topk, out, ws, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            D.prefill(h, inputs, wl.T, topk, out, ws, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        st, bits = D.ds4sp_device_status(h)
+        if st != D.OK:
+            raise RuntimeError(f"device status {bits:#x} after {name} timing")
+        line = {"workload": config_name(wl), "tokens_per_s": wl.T * steps / (ms / 1e3),
+                "ms_per_prefill": ms / steps, "steps": steps}
+        return line, host, topk.cpu().numpy(), out.cpu().numpy()
+    finally:
+        D.ds4sp_destroy(h)
+
+
+def gather_ceiling(dev, stream, rows_table=12800, n=6_020_672, reps=5):
+    """Bandwidth of random 1152-byte row gathers from an L2-resident table of the 10K
+    prefill's size (its 10,240 raw + 2,560 compressed rows, 14.75 MB), through the
+    library's gather probe: the ceiling for the attention kernel's row traffic."""
+    g = torch.Generator(device="cpu").manual_seed(5)
+    table = torch.randn(rows_table, 576, generator=g).half().to(dev)
+    idx = torch.randint(0, rows_table, (n,), generator=g, dtype=torch.int32).to(dev)
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    props = torch.cuda.get_device_properties(dev)
+    grid = props.multi_processor_count * 4
+    for _ in range(3):
+        D.ds4sp_probe_gather(table, idx, sink, grid, stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        D.ds4sp_probe_gather(table, idx, sink, grid, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    return {"GBps": 1152 * n / (ms / 1e3) / 1e9, "rows": n, "table_MB": rows_table * 1152 / 1e6,
+            "ms": ms, "how": "ds4sp_probe_gather: random rows, 16-byte loads into registers, "
+                             f"{grid} CTAs x 512 threads"}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
     torch.cuda.set_device(local_rank)
@@ -281,6 +356,7 @@ def run_ours(args, rank, world, local_rank):
     wl = workload(WORKLOAD)
     alg = algorithmic(wl)
     pk = peaks()
+    solo = rank == 0 and world == 1          # extras that only a single-GPU run reports
 
     host = generate(wl)
     inputs = {k: v.to(dev) for k, v in host.items()}
@@ -306,12 +382,12 @@ def run_ours(args, rank, world, local_rank):
     if st != D.OK:
         raise RuntimeError(f"device status {bits:#x} after warm-up")
 
-    def timed_steps():
+    def timed_steps(n):
         barrier()
         torch.cuda.synchronize()
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(n):
             step()
         ev1.record(stream)
         torch.cuda.synchronize()
@@ -324,13 +400,20 @@ def run_ours(args, rank, world, local_rank):
     # around each kernel put a timestamp between every two launches, which by itself
     # lengthens a prefill by about 6% (1.39 -> 1.47 ms at 10K on B200), so the per-kernel
     # split and the roofline come from a second pass of the same K steps with them on.
-    ms = timed_steps()
+    ms = timed_steps(args.steps)
     D.ds4sp_profile_enable(h, True)
     D.ds4sp_profile_read(h)
-    ms_prof = timed_steps()
+    ms_prof = timed_steps(args.steps)
     prof = D.ds4sp_profile_read(h)
     D.ds4sp_profile_enable(h, False)
+    # The K timed steps last tens of milliseconds, shorter than the sampler's 100 ms
+    # period; the same step keeps running for about `soak` seconds more so that the clock
+    # record holds enough samples under this load.
+    soak_steps = max(1, int(args.soak * 1e3 / max(ms / args.steps, 1e-3)))
+    ms_soak = timed_steps(soak_steps)
     clk = clocks.stop()
+    clk["window"] = (f"sampled every 100 ms over the timed steps, the profiled pass and "
+                     f"{soak_steps} more steps ({ms_soak / 1e3:.2f} s) of the same prefill")
     ms_max = max_over_ranks(ms, world, dev)
     ms_prof_max = max_over_ranks(ms_prof, world, dev)
 
@@ -360,18 +443,16 @@ def run_ours(args, rank, world, local_rank):
     topk_e2e = topk.cpu().numpy()
 
     verify = None
-    if rank == 0 and world == 1 and not args.no_verify:
+    if solo and not args.no_verify:
         verify = verify_latency(dev)
 
     # The same step with CUDA's exp2f for the softmax exponentials (exp_mode 1), and with
     # fp32-staged probabilities in P . V (pv_mode 1, fast and precise exponentials), for
     # the fast-versus-precise and fp16-versus-fp32-staged comparisons; not the headline.
     variants = None
-    if rank == 0 and world == 1 and not args.no_verify:
+    if solo and not args.no_verify:
         variants = {}
-        for name, modes in (("exp2f_softmax", dict(exp_mode=1)),
-                            ("fp32_staged_pv", dict(pv_mode=1)),
-                            ("fp32_staged_pv_exp2f", dict(pv_mode=1, exp_mode=1))):
+        for name, modes in VARIANTS:
             cfg_v = D.make_config(n_idx_heads=wl.H_i, d_idx=wl.D_i, top_k=wl.top_k,
                                   n_swa=wl.n_swa, max_tokens=wl.T, band=wl.band, **modes)
             hv = D.ds4sp_create(cfg_v)
@@ -379,23 +460,57 @@ def run_ours(args, rank, world, local_rank):
                 for _ in range(3):
                     D.prefill(hv, inputs, wl.T, topk, out, ws, stream)
                 torch.cuda.synchronize()
+                n_var = 20
+                ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                ev0.record(stream)
+                for _ in range(n_var):
+                    D.prefill(hv, inputs, wl.T, topk, out, ws, stream)
+                ev1.record(stream)
+                torch.cuda.synchronize()
                 D.ds4sp_profile_enable(hv, True)
                 D.ds4sp_profile_read(hv)
-                n_var = 20
                 for _ in range(n_var):
                     D.prefill(hv, inputs, wl.T, topk, out, ws, stream)
                 torch.cuda.synchronize()
                 vprof = D.ds4sp_profile_read(hv)
-                variants[name] = {"attention_ms_per_step": vprof["attention"][0] / n_var,
+                st, bits = D.ds4sp_device_status(hv)
+                if st != D.OK:
+                    raise RuntimeError(f"device status {bits:#x} in variant {name}")
+                variants[name] = {"ms_per_step": ev0.elapsed_time(ev1) / n_var,
+                                  **{f"{k}_ms_per_step": v[0] / n_var for k, v in vprof.items()},
                                   "steps": n_var, **modes}
             finally:
                 D.ds4sp_destroy(hv)
 
+    # tokens/s of every prefill workload (the 10K line is the headline; the others use the
+    # same step on their own sizes), and all-token parity of the 8K prefill.
+    per_config = parity_8k = None
+    if solo and not args.no_per_config:
+        per_config = {}
+        for name in ("band", "8k"):
+            line_c, host_c, tk_c, out_c = config_throughput(name, dev, max(args.steps, 20), stream)
+            per_config[name] = line_c
+            if name == "8k" and not args.no_cpu_baseline:
+                wl8 = workload("8k")
+                ref8 = cpu_oracle_sample(wl8, wl8.T, {k: v.numpy() for k, v in host_c.items()},
+                                         return_result=True)[1]
+                parity_8k = sampled_parity(ref8, tk_c, out_c,
+                                           of="every token of the 8,192-token prefill "
+                                              "(ds4sp_prefill_band, device buffers)")
+        per_config["10k"] = {"workload": config_name(wl), "tokens_per_s": wl.T * args.steps / (ms / 1e3),
+                             "ms_per_prefill": ms / args.steps, "steps": args.steps}
+
+    l2 = None
+    if solo:
+        l2 = gather_ceiling(dev, stream)
+
     cpu_base = parity = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if solo and not args.no_cpu_baseline:
         cpu_base, ref = cpu_oracle_sample(wl, args.cpu_sample,
                                           {k: v.numpy() for k, v in host.items()},
                                           return_result=True)
+        one = cpu_oracle_sample(wl, 256, {k: v.numpy() for k, v in host.items()}, one_core=True)
+        cpu_base["one_core"] = {"value": one["value"], "cores": 1, "sample": one["sample"]}
         parity = sampled_parity(ref, topk_e2e, out_e2e)
 
     if rank == 0:
@@ -406,6 +521,16 @@ def run_ours(args, rank, world, local_rank):
         steps = args.steps
         attn_achieved = alg["attention_bytes"] * steps / (attn_ms / 1e3) / 1e9
         idx_achieved = alg["indexer_flops"] * steps / (idx_ms / 1e3) / 1e12
+        attn_kernel = {"ms_per_step": attn_ms / steps, "launches": attn_n,
+                       "alg_GBps": attn_achieved,
+                       "frac_hbm": attn_achieved / pk["hbm_gbs"],
+                       "alg_bytes_per_step": alg["attention_bytes"]}
+        if l2:
+            # the rows and Q the kernel reads through L2, against the measured gather ceiling
+            l2_bytes = 1152 * alg["rows"] + 18432 * wl.T
+            l2_gbs = l2_bytes * steps / (attn_ms / 1e3) / 1e9
+            attn_kernel["l2_GBps"] = l2_gbs
+            attn_kernel["frac_l2_gather"] = l2_gbs / l2["GBps"]
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": steps, "warmup": args.warmup, "ms_per_step": ms_max / steps,
@@ -416,12 +541,10 @@ def run_ours(args, rank, world, local_rank):
             "roofline": {"bound": "hbm", "achieved": attn_achieved, "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": attn_achieved / pk["hbm_gbs"],
                          "traffic": attention_traffic(), "kernel": "sparse_attn_mma_kernel",
-                         "peak_source": f"{pk['source']} hbm_gbs (of {pk['source']})"},
+                         "peak_source": f"{pk['source']} hbm_gbs (of {pk['source']})",
+                         "l2_gather_frac": attn_kernel.get("frac_l2_gather")},
             "kernels": {
-                "attention": {"ms_per_step": attn_ms / steps, "launches": attn_n,
-                              "alg_GBps": attn_achieved,
-                              "frac_hbm": attn_achieved / pk["hbm_gbs"],
-                              "alg_bytes_per_step": alg["attention_bytes"]},
+                "attention": attn_kernel,
                 "indexer": {"ms_per_step": idx_ms / steps, "launches": idx_n,
                             "TFLOPs": idx_achieved,
                             "frac_tensor": idx_achieved / pk["bf16_tflops"],
@@ -433,6 +556,8 @@ def run_ours(args, rank, world, local_rank):
             "kernel_timing": {"steps": steps, "ms_per_step": ms_prof_max / steps,
                               "how": "a second pass of the same steps with CUDA events "
                                      "around each kernel on the launching stream"},
+            "per_config": per_config,
+            "l2_gather_ceiling": l2,
             "verify": verify,
             "variants": variants,
             "e2e": {"value": job_throughput(wl.T, world, e2e_steps, e2e_ms), "unit": "tokens/s",
@@ -440,9 +565,19 @@ def run_ours(args, rank, world, local_rank):
             "clocks": clk,
             "cpu_baseline": cpu_base,
             "parity": parity,
+            "parity_8k": parity_8k,
         }
         print(json.dumps(line), flush=True)
     D.ds4sp_destroy(h)
+
+
+# Same step, other arithmetic choices (config fields), timed for comparison only.
+VARIANTS = [
+    ("fused_indexer_topk", dict(topk_mode=1)),
+    ("exp2f_softmax", dict(exp_mode=1)),
+    ("fp32_staged_pv", dict(pv_mode=1)),
+    ("fp32_staged_pv_exp2f", dict(pv_mode=1, exp_mode=1)),
+]
 
 
 def main():
@@ -454,7 +589,12 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=8192)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-verify", action="store_true",
-                    help="skip the few-token latency of the 122,880-token verify workload")
+                    help="skip the few-token latency of the 122,880-token verify workload "
+                         "and the variants")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the band and 8K prefill lines (and the 8K parity check)")
+    ap.add_argument("--soak", type=float, default=1.5,
+                    help="seconds of extra steps under the clock sampler")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -84,6 +84,17 @@ typedef struct {
                             P . V tensor work ("FP32-staged streaming MLA" of "perf(ds4):
                             unify gfx1151 sparse-prefill stack", Validation completed);
                             other values are DS4SP_ERR_INVALID_ARG */
+    int topk_mode;       /* steps 1-2: 0 = the indexer writes fp32 scores to the caller's
+                            workspace and a top-k kernel reads them back; 1 = one fused
+                            kernel keeps each token block's scores in shared memory and
+                            selects there, so no score reaches global memory. A call takes
+                            the fused kernel when no explicit mask is set and a token
+                            block's score rows fit its 64 KB key buffer (256/n_idx_heads
+                            tokens x 128 x ceil(n_vis(last token)/128) x 4 bytes, e.g. up
+                            to 4,096 visible rows at 64 indexer heads) in a call of at most
+                            1,024 token blocks; otherwise the two kernels run. Indices are
+                            the same bits either way. Other values are
+                            DS4SP_ERR_INVALID_ARG */
 } ds4sp_config;
 
 /* Validate cfg and create a handle bound to the current CUDA device. The handle owns
@@ -243,7 +254,8 @@ ds4sp_status ds4sp_debug_set_mask(ds4sp_handle* h, const uint8_t* mask, int rows
  * no handle and no workspace, and calls no cudaMalloc, cudaFree or allocating library
  * routine. Its score scratch is a fixed 8 MiB array inside the library (2^21 fp32
  * scores); every GPU that loads the library holds that array until the process exits.
- *   cfg     the same configuration ds4sp_create takes (validated the same way);
+ *   cfg     the same configuration ds4sp_create takes (validated the same way; this
+ *           entry point always runs the two-kernel form, whatever cfg->topk_mode says);
  *   q_idx, k_idx, w, t0, n_q, topk, stream  as for ds4sp_indexer_topk.
  * n_q * ld must be <= 2^21, with ld = n_vis(t0+n_q-1) rounded up to 4 (for example, a
  * 2048-token band whose last token sees up to 1024 rows, or up to 5 tokens at a
@@ -258,6 +270,19 @@ ds4sp_status ds4sp_debug_set_mask(ds4sp_handle* h, const uint8_t* mask, int rows
 ds4sp_status ds4sp_indexer_topk_noalloc(const ds4sp_config* cfg, const void* q_idx,
                                         const void* k_idx, const float* w, int t0, int n_q,
                                         int32_t* topk, void* stream);
+
+/* Measurement helper, not a step of the path: the bandwidth ceiling of the attention
+ * kernel's access pattern. Reads n rows of row_bytes (a multiple of 16, at most 1152)
+ * from `table` [table_rows, row_bytes] at the row indices idx[0..n) (each in
+ * [0, table_rows); the caller guarantees it, the kernel does not check), with 16-byte
+ * loads into registers, and XORs every word into *sink (4 bytes, device memory) so that
+ * no load is dead. Timing it with events around the call gives bytes/s for random row
+ * gathers: with an L2-resident table (such as the KV of a 10K prefill, 14.75 MB) it is
+ * the L2-to-SM gather ceiling that the attention kernel's rows are served under.
+ * grid = CTAs of 512 threads (a multiple of the SM count is best). Asynchronous on
+ * `stream`; argument errors are returned before the launch. */
+ds4sp_status ds4sp_probe_gather(const void* table, int table_rows, int row_bytes,
+                                const int32_t* idx, int n, uint32_t* sink, int grid, void* stream);
 
 /* Static description of a status code. */
 const char* ds4sp_status_string(ds4sp_status s);

@@ -291,6 +291,18 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Ties 32 registers written by an earlier tcgen05.ld to a point after tmem_ld_wait():
+// the compiler sees them rewritten here, so no use of them moves above the wait.
+__device__ __forceinline__ void tmem_regs_after_wait(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31]));
+}
+
 // Shared-memory matrix descriptor for a K-major operand in the 128-byte swizzle
 // layout that TMA writes with CU_TENSOR_MAP_SWIZZLE_128B: 8-row groups of
 // 128-byte rows, 1024 bytes apart. Bits: start>>4 [0,14), LBO>>4 [16,30),

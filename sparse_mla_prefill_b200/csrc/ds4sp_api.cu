@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <new>
@@ -17,6 +18,8 @@
 
 #include "ds4sp.h"
 #include "indexer_tcgen05.cuh"
+#include "indexer_topk_fused.cuh"
+#include "probe_gather.cuh"
 #include "sparse_attn_mma.cuh"
 #include "topk_radix.cuh"
 
@@ -109,8 +112,8 @@ constexpr int kMaxDevices = 64;
 // attribute belongs to the device's copy of the function.
 ds4sp_status set_smem_once(ds4sp_handle* h, const void* fn, int bytes, int slot, const char* what) {
     static std::mutex mu;
-    static bool done[kMaxDevices][16] = {};
-    if (h->device < 0 || h->device >= kMaxDevices || slot < 0 || slot >= 16)
+    static bool done[kMaxDevices][32] = {};
+    if (h->device < 0 || h->device >= kMaxDevices || slot < 0 || slot >= 32)
         return fail(DS4SP_ERR_UNSUPPORTED, "device %d", h->device);
     std::lock_guard<std::mutex> lock(mu);
     if (done[h->device][slot]) return DS4SP_OK;
@@ -125,6 +128,8 @@ ds4sp_status set_smem_once(ds4sp_handle* h, const void* fn, int bytes, int slot,
 constexpr int indexer_slot(int d_idx, int h_idx) {
     return (d_idx == 128 ? 5 : 0) + (h_idx == 4 ? 0 : h_idx == 8 ? 1 : h_idx == 16 ? 2 : h_idx == 32 ? 3 : 4);
 }
+// Slots 0-9: indexer_tcgen05_kernel; 10-19 (tables of 32): the fused kernel.
+constexpr int fused_slot(int d_idx, int h_idx) { return 10 + indexer_slot(d_idx, h_idx); }
 
 int score_ld(int t_last, int ratio) {
     const int nv = nvis(t_last, ratio);
@@ -308,6 +313,92 @@ ds4sp_status dispatch_indexer_h(ds4sp_handle* h, const void* q_idx, const void* 
     return fail(DS4SP_ERR_UNSUPPORTED, "n_idx_heads %d", h->cfg.n_idx_heads);
 }
 
+// Indexer and top-k in one launch (indexer_topk_fused_kernel), when the call qualifies:
+// no explicit mask, some token sees a compressed row, the key rows of a token block fit
+// the kernel's 64 KB key buffer and the launch has at most kFusedMaxBlocks token blocks.
+// Returns DS4SP_ERR_UNSUPPORTED (with nothing launched) when it does not qualify.
+template <int D_I, int H_I>
+ds4sp_status launch_fused(ds4sp_handle* h, const void* q_idx, const void* k_idx, const float* w,
+                          int t0, int n_q, int32_t* topk, cudaStream_t stream) {
+    using C = FusedTile<D_I, H_I>;
+    const int ratio = h->cfg.ratio, k = h->cfg.top_k;
+    const int n_rows = nvis(t0 + n_q - 1, ratio);
+    const int n_tb = (n_q + C::TB - 1) / C::TB;
+    const int max_tiles = (n_rows + C::BM - 1) / C::BM;
+    const int kld = C::BM * max_tiles;
+    if (h->mask || n_rows == 0 || n_tb > kFusedMaxBlocks ||
+        (long long)C::TB * kld * 4 > C::KEY_BYTES)
+        return DS4SP_ERR_UNSUPPORTED;
+    CUtensorMap tk, tq;
+    if (!make_tmap_2d(&tk, k_idx, D_I, n_rows, C::BM) ||
+        !make_tmap_2d(&tq, q_idx, D_I, n_q * H_I, C::BN))
+        return fail(DS4SP_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    DS4SP_TRY(set_smem_once(h, reinterpret_cast<const void*>(indexer_topk_fused_kernel<D_I, H_I>),
+                            C::SMEM_BYTES, fused_slot(D_I, H_I),
+                            "cudaFuncSetAttribute(fused indexer)"));
+    FusedParams p;
+    p.w = w;
+    p.topk = topk;
+    p.wc = next_wait(h);
+    p.t0 = t0;
+    p.n_q = n_q;
+    p.k = k;
+    p.ratio = ratio;
+    p.kld = kld;
+    // Longest-processing-time assignment of the token blocks to the persistent CTAs: cost
+    // = the block's tiles, plus kSelectCost per token that needs a select (n_vis > k),
+    // in tile-equivalents; blocks go heaviest first to the least loaded CTA.
+    constexpr double kSelectCost = 1.5;
+    const int grid = std::min(n_tb, std::min(h->sm_count, kIndexerMaxGrid));
+    std::vector<std::pair<double, int>> cost(n_tb);
+    for (int tb = 0; tb < n_tb; ++tb) {
+        const int tok0 = t0 + tb * C::TB, tok_end = std::min(tok0 + C::TB, t0 + n_q);
+        const int tiles = (nvis(tok_end - 1, ratio) + C::BM - 1) / C::BM;
+        int sel = 0;
+        for (int t = tok0; t < tok_end; ++t) sel += nvis(t, ratio) > k;
+        cost[tb] = {tiles + kSelectCost * sel, tb};
+    }
+    std::sort(cost.begin(), cost.end(), [](const std::pair<double, int>& a, const std::pair<double, int>& b) {
+        return a.first != b.first ? a.first > b.first : a.second > b.second;
+    });
+    std::vector<std::vector<int>> lists(grid);
+    std::vector<std::pair<double, int>> heap;   // (load, cta), min-heap by load then cta
+    for (int c = 0; c < grid; ++c) heap.push_back({0.0, c});
+    auto cmp = [](const std::pair<double, int>& a, const std::pair<double, int>& b) {
+        return a.first != b.first ? a.first > b.first : a.second > b.second;
+    };
+    std::make_heap(heap.begin(), heap.end(), cmp);
+    for (const auto& cb : cost) {
+        std::pop_heap(heap.begin(), heap.end(), cmp);
+        auto& top = heap.back();
+        lists[top.second].push_back(cb.second);
+        top.first += cb.first;
+        std::push_heap(heap.begin(), heap.end(), cmp);
+    }
+    int u = 0;
+    for (int c = 0; c < grid; ++c) {
+        p.first[c] = (uint16_t)u;
+        for (int tb : lists[c]) p.blk[u++] = (uint16_t)tb;
+    }
+    p.first[grid] = (uint16_t)u;
+    return launch(h, kIndexer, stream, [&] {
+        indexer_topk_fused_kernel<D_I, H_I><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tq, p);
+    });
+}
+
+template <int D_I>
+ds4sp_status dispatch_fused_h(ds4sp_handle* h, const void* q_idx, const void* k_idx,
+                              const float* w, int t0, int n_q, int32_t* topk, cudaStream_t s) {
+    switch (h->cfg.n_idx_heads) {
+        case 4: return launch_fused<D_I, 4>(h, q_idx, k_idx, w, t0, n_q, topk, s);
+        case 8: return launch_fused<D_I, 8>(h, q_idx, k_idx, w, t0, n_q, topk, s);
+        case 16: return launch_fused<D_I, 16>(h, q_idx, k_idx, w, t0, n_q, topk, s);
+        case 32: return launch_fused<D_I, 32>(h, q_idx, k_idx, w, t0, n_q, topk, s);
+        case 64: return launch_fused<D_I, 64>(h, q_idx, k_idx, w, t0, n_q, topk, s);
+    }
+    return fail(DS4SP_ERR_UNSUPPORTED, "n_idx_heads %d", h->cfg.n_idx_heads);
+}
+
 ds4sp_status launch_topk(ds4sp_handle* h, const float* scores, int ld, int t0, int n_q,
                          int32_t* topk, cudaStream_t stream) {
     const int k = h->cfg.top_k, ratio = h->cfg.ratio;
@@ -474,6 +565,14 @@ ds4sp_status indexer_topk_impl(ds4sp_handle* h, const void* q_idx, const void* k
     const size_t need = ds4sp_workspace_bytes(h, t0, n_q);
     if (ws_bytes < need)
         return fail(DS4SP_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    if (h->cfg.topk_mode == 1) {
+        // Fused indexer + top-k where the call qualifies, else the two kernels below.
+        const ds4sp_status fs =
+            h->cfg.d_idx == 64 ? dispatch_fused_h<64>(h, q_idx, k_idx, w, t0, n_q, topk, stream)
+                               : dispatch_fused_h<128>(h, q_idx, k_idx, w, t0, n_q, topk, stream);
+        if (fs == DS4SP_OK) return record_last(h, stream);
+        if (fs != DS4SP_ERR_UNSUPPORTED) return fs;
+    }
     const int ld = score_ld(t_last, h->cfg.ratio);
     float* scores = static_cast<float*>(ws);
     const ds4sp_status s =
@@ -546,6 +645,8 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
         return fail(DS4SP_ERR_INVALID_ARG, "exp_mode %d (0 = ex2.approx, 1 = exp2f)", c.exp_mode);
     if (c.pv_mode != 0 && c.pv_mode != 1)
         return fail(DS4SP_ERR_INVALID_ARG, "pv_mode %d (0 = fp16 P, 1 = fp32-staged P)", c.pv_mode);
+    if (c.topk_mode != 0 && c.topk_mode != 1)
+        return fail(DS4SP_ERR_INVALID_ARG, "topk_mode %d (0 = separate top-k, 1 = fused)", c.topk_mode);
     ds4sp_handle* h = new (std::nothrow) ds4sp_handle();
     if (!h) return fail(DS4SP_ERR_INVALID_ARG, "out of host memory");
     h->cfg = c;
@@ -884,6 +985,25 @@ ds4sp_status ds4sp_debug_set_mask(ds4sp_handle* h, const uint8_t* mask, int rows
     h->mask_rows = rows;
     h->mask_cols = cols;
     return DS4SP_OK;
+}
+
+ds4sp_status ds4sp_probe_gather(const void* table, int table_rows, int row_bytes,
+                                const int32_t* idx, int n, uint32_t* sink, int grid, void* stream) {
+    const TraceRange trace("ds4sp_probe_gather");
+    if (row_bytes < 16 || row_bytes % 16 != 0 || row_bytes > 16 * 8 * 9)
+        return fail(DS4SP_ERR_INVALID_ARG, "row_bytes %d (a multiple of 16, at most 1152)", row_bytes);
+    if (table_rows < 1 || n < 0 || grid < 1 || grid > 65535)
+        return fail(DS4SP_ERR_INVALID_ARG, "table_rows %d, n %d, grid %d", table_rows, n, grid);
+    if (n == 0) return DS4SP_OK;
+    DS4SP_TRY(check_ptr(table, "table"));
+    DS4SP_TRY(check_ptr(idx, "idx"));
+    if (!sink || (reinterpret_cast<uintptr_t>(sink) & 3u))
+        return fail(DS4SP_ERR_INVALID_ARG, "sink is null or not 4-byte aligned");
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    probe_gather_kernel<9><<<grid, kProbeThreads, 0, s>>>(static_cast<const uint4*>(table),
+                                                          row_bytes / 16, idx, n, sink);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? DS4SP_OK : cuda_fail(e, "probe_gather launch");
 }
 
 const char* ds4sp_status_string(ds4sp_status s) {

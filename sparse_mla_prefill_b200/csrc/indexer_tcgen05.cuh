@@ -19,7 +19,8 @@
 // units ahead; warp 0 streams whole k_idx tiles (one 64-dim TMA box per K sub-tile)
 // into a ring of two (D_i = 128) or four (D_i = 64) stages;
 // warp 1 owns TMEM and issues the MMAs; warps 2-9 run the epilogue (ReLU, head
-// weights, sum, store), two warps per TMEM lane quarter, each on half of the columns.
+// weights, sum, store), two warps per TMEM lane quarter, each on half of the columns,
+// the second 64 of its columns loading from TMEM while the first 64 are reduced.
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i overlap the MMAs
 // of tile i+1.
 // Every wait is bounded (device_common.cuh).
@@ -128,6 +129,62 @@ __device__ __forceinline__ void ffma2(float& acc_x, float& acc_y, float a_x, flo
         "mov.b64 {%0, %1}, rc;\n\t}"
         : "+f"(acc_x), "+f"(acc_y)
         : "f"(a_x), "f"(a_y), "f"(b_x), "f"(b_y));
+}
+
+// Epilogue of one 64-column half of a warp's accumulator columns: the scores of its
+// 64 / H_I tokens. The ReLU is taken as x + |x| = 2 ReLU(x), exact and on the FMA pipe,
+// against head weights stored halved (0.5 w, exact), so every product equals
+// w * ReLU(x) bit for bit (for |x| < 2^127 and w not subnormal). NP independent packed
+// accumulators per token keep the FMA chains short. store(token of the half, score).
+template <int H_I, class Store>
+__device__ __forceinline__ void epilogue_half(const uint32_t (&vh)[2][32], const float* wh_half,
+                                              Store store) {
+    constexpr int TPH = 64 / H_I;
+    constexpr int NP = H_I >= 16 ? 4 : H_I / 4;
+#pragma unroll
+    for (int tk = 0; tk < TPH; ++tk) {
+        float acc[2 * NP];
+#pragma unroll
+        for (int i = 0; i < 2 * NP; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int c = tk * H_I; c < (tk + 1) * H_I; c += 4) {
+            const float4 wv = *reinterpret_cast<const float4*>(wh_half + c);
+            const int pr = (c / 4) % NP;
+            const float x0 = __uint_as_float(vh[c / 32][c % 32]);
+            const float x1 = __uint_as_float(vh[c / 32][c % 32 + 1]);
+            const float x2 = __uint_as_float(vh[c / 32][c % 32 + 2]);
+            const float x3 = __uint_as_float(vh[c / 32][c % 32 + 3]);
+            ffma2(acc[2 * pr], acc[2 * pr + 1], wv.x, wv.y, x0 + fabsf(x0), x1 + fabsf(x1));
+            ffma2(acc[2 * pr], acc[2 * pr + 1], wv.z, wv.w, x2 + fabsf(x2), x3 + fabsf(x3));
+        }
+#pragma unroll
+        for (int i = 2; i < 2 * NP; i += 2) {
+            acc[0] += acc[i];
+            acc[1] += acc[i + 1];
+        }
+        store(tk, acc[0] + acc[1]);
+    }
+}
+
+// A warp's 128 accumulator columns of one tile (lane = row j): the first 64 columns are
+// loaded and, while they are turned into scores, the other 64 load; the accumulator is
+// released (`release`) once both halves are in registers.
+template <int H_I, class Release, class Store>
+__device__ __forceinline__ void epilogue_tile(uint32_t taddr, const float* wh, Release release,
+                                              Store store) {
+    uint32_t va[2][32], vb[2][32];
+    tmem_ld_x32(taddr, va[0]);
+    tmem_ld_x32(taddr + 32, va[1]);
+    tmem_ld_wait();
+    tmem_ld_x32(taddr + 64, vb[0]);
+    tmem_ld_x32(taddr + 96, vb[1]);
+    constexpr int TPH = 64 / H_I;
+    epilogue_half<H_I>(va, wh, [&](int tk, float s) { store(tk, s); });
+    tmem_ld_wait();
+    tmem_regs_after_wait(vb[0]);
+    tmem_regs_after_wait(vb[1]);
+    release();
+    epilogue_half<H_I>(vb, wh + 64, [&](int tk, float s) { store(TPH + tk, s); });
 }
 
 template <int D_I, int H_I>
@@ -291,7 +348,7 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             w_next = have ? unit_weight(w_nx) : 0.f;
             // Head weights of the unit's tokens, in column order (col = token*H_i + h).
             float* swb = sw + (bi & 1) * C::BN;
-            swb[col] = w_this;
+            swb[col] = 0.5f * w_this;           // halved: see epilogue_half
             named_barrier(1, C::EPI_WARPS * 32);
             const float* wh = swb + half * 128;
             // After a wait gives up this warp keeps walking the units (waits then return at
@@ -307,45 +364,21 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
                 tc_fence_after();
                 const int j = w.jt(it) * C::BM + quarter * 32 + lane;
-                // All 128 columns of this warp into registers, then release the accumulator
-                // at once so the next tile's MMAs never wait on this epilogue's arithmetic.
-                uint32_t v[4][32];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) tmem_ld_x32(lane_addr + buf * C::BN + q * 32, v[q]);
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(tempty(buf));
-                // Per token: NP independent packed accumulators keep the FMA chains short.
-                constexpr int TPW = 128 / H_I;           // tokens in this warp's 128 columns
-                constexpr int NP = H_I >= 16 ? 4 : H_I / 4;
-                const int t_first = w.tok0 + half * TPW;
-#pragma unroll
-                for (int tk = 0; tk < TPW; ++tk) {
-                    float acc[2 * NP];
-#pragma unroll
-                    for (int i = 0; i < 2 * NP; ++i) acc[i] = 0.f;
-#pragma unroll
-                    for (int c = tk * H_I; c < (tk + 1) * H_I; c += 4) {
-                        const float4 wv = *reinterpret_cast<const float4*>(wh + c);
-                        const int pr = (c / 4) % NP;
-                        ffma2(acc[2 * pr], acc[2 * pr + 1], wv.x, wv.y,
-                              fmaxf(__uint_as_float(v[c / 32][c % 32]), 0.f),
-                              fmaxf(__uint_as_float(v[c / 32][c % 32 + 1]), 0.f));
-                        ffma2(acc[2 * pr], acc[2 * pr + 1], wv.z, wv.w,
-                              fmaxf(__uint_as_float(v[c / 32][c % 32 + 2]), 0.f),
-                              fmaxf(__uint_as_float(v[c / 32][c % 32 + 3]), 0.f));
-                    }
-#pragma unroll
-                    for (int i = 2; i < 2 * NP; i += 2) {
-                        acc[0] += acc[i];
-                        acc[1] += acc[i + 1];
-                    }
-                    const int t = t_first + tk;
-                    // j < n_vis(t) = floor((t+1)/ratio)  <=>  ratio*(j+1) <= t+1
-                    if (t < w.tok_end && p.ratio * (j + 1) <= t + 1)
-                        p.scores[(size_t)(t - p.t0) * p.ld + j] = acc[0] + acc[1];
-                }
+                const int t_first = w.tok0 + half * (128 / H_I);
+                epilogue_tile<H_I>(
+                    lane_addr + buf * C::BN, wh,
+                    [&] {
+                        // the accumulator may be overwritten by the tile after next
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(tempty(buf));
+                    },
+                    [&](int tk, float score) {
+                        const int t = t_first + tk;
+                        // j < n_vis(t) = floor((t+1)/ratio)  <=>  ratio*(j+1) <= t+1
+                        if (t < w.tok_end && p.ratio * (j + 1) <= t + 1)
+                            p.scores[(size_t)(t - p.t0) * p.ld + j] = score;
+                    });
             }
             ++bi;
         }

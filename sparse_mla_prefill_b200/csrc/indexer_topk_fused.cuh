@@ -1,0 +1,345 @@
+// Indexer and top-k in one kernel: the scores never leave the SM.
+//
+// Same scores as indexer_tcgen05_kernel -- score(t, j) = sum_h w[t,h] *
+// ReLU(q_idx[t,h,:] . k_idx[j,:]) for the rows j visible to t (4j+3 <= t), computed as
+// D[j, (t,h)] tiles on the tensor cores with the ReLU and the head-weighted sum in the
+// epilogue -- and the same selection as topk_radix_kernel: the min(k, n_vis(t)) largest
+// scores, equal scores to the lower j, listed by ascending j, then -1. The pages hand
+// the long-prefill top-k rows straight to attention ("pass authoritative long-prefill
+// top-k rows directly", "perf(ds4): extend sparse prefill scheduling to 10K", Summary;
+// "direct long-prefill top-k handoff", "perf(ds4): unify gfx1151 sparse-prefill stack",
+// Composition); here the handoff goes one step further and the score rows themselves
+// are never written to global memory.
+//
+// Work: a unit is one whole token block (256/H_i tokens) with all the 128-row j-tiles
+// its last token needs, so a CTA ends a unit holding complete score rows. The host
+// assigns the launch's token blocks to the persistent CTAs by longest-processing-time
+// on their cost (tiles, plus the select), heaviest first.
+// Per unit: the epilogue warps turn each tile's accumulator into order-preserving keys
+// of the scores (the top-k kernel's mapping) in a shared-memory key buffer [tokens of
+// the block][128 x tiles]; after the last tile the same warps run the radix select of
+// topk_radix.cuh on each token's row, 256 threads synchronised by a named barrier, and
+// write the token's indices. Meanwhile the q_idx loader brings the next unit's block
+// into the (single) B buffer as soon as this unit's MMAs have read it, and the MMA warp
+// runs ahead by the two TMEM accumulators.
+// Roles and pipelines are those of indexer_tcgen05_kernel (warp 0 streams k_idx tiles,
+// warp 10 loads q_idx blocks, warp 1 issues the MMAs, warps 2-9 run the epilogue and the
+// select); every wait is bounded (device_common.cuh).
+#pragma once
+
+#include <cuda.h>
+
+#include "device_common.cuh"
+#include "indexer_tcgen05.cuh"
+#include "topk_radix.cuh"
+
+namespace ds4sp {
+
+template <int D_I, int H_I>
+struct FusedTile {
+    using T = IndexerTile<D_I, H_I>;
+    static constexpr int BM = T::BM, BN = T::BN, TB = T::TB, KSUB = T::KSUB;
+    static constexpr int A_SUB = T::A_SUB, A_STAGE = T::A_STAGE, B_SUB = T::B_SUB;
+    static constexpr int B_BYTES = T::B_BYTES, A_STAGES = T::A_STAGES;
+    static constexpr int EPI_WARPS = 8, EPI_THREADS = EPI_WARPS * 32;
+    static constexpr int B_WARP = 2 + EPI_WARPS;
+    static constexpr int THREADS = (3 + EPI_WARPS) * 32;
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int KEY_BYTES = 64 * 1024;                   // [TB][kld] uint32 keys
+    static constexpr int OFF_B = 0;                               // one B buffer
+    static constexpr int OFF_A = B_BYTES;
+    static constexpr int OFF_KEYS = OFF_A + A_STAGES * A_STAGE;
+    static constexpr int OFF_W = OFF_KEYS + KEY_BYTES;            // two w buffers
+    static constexpr int OFF_SEL = OFF_W + 2 * BN * 4;            // select scratch
+    // hist[256], w_or/w_and/w_cnt[8], s_digit, s_above, abort flag, pad, warp_tot[8]
+    // (8-byte aligned)
+    static constexpr int SEL_BYTES = 256 * 4 + 3 * 8 * 4 + 4 * 4 + 8 * 8;
+    static constexpr int SEL_ABORT = 256 * 4 + 3 * 8 * 4 + 2 * 4;   // byte offset of the flag
+    static constexpr int OFF_BAR = OFF_SEL + SEL_BYTES;
+    // afull[A_STAGES], aempty[A_STAGES], bfull, bempty, tempty[2], done
+    static constexpr int N_BARS = 2 * A_STAGES + 1 + 1 + 2 + 1;
+    static constexpr int OFF_TMEM_PTR = OFF_BAR + N_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;   // + alignment slack
+    static constexpr uint32_t IDESC = T::IDESC;
+    static_assert(SEL_BYTES % 8 == 0 && OFF_SEL % 8 == 0, "8-byte aligned select scratch");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+constexpr int kFusedMaxBlocks = 1024;     // token blocks of one launch
+
+struct FusedParams {
+    const float* w;        // [n_q, H_i] fp32, row 0 = token t0
+    int32_t* topk;         // [n_q, k] int32 output, row 0 = token t0
+    WaitCtl wc;
+    int t0, n_q, k, ratio;
+    int kld;               // key row stride (128 x the launch's largest tile count)
+    // CTA b processes token blocks blk[first[b]] .. blk[first[b+1]-1], in that order.
+    uint16_t first[kIndexerMaxGrid + 1];
+    uint16_t blk[kFusedMaxBlocks];
+};
+
+// Named barrier of the epilogue warps (they also run the select).
+struct EpiSync {
+    __device__ __forceinline__ void operator()() const { named_barrier(1, 8 * 32); }
+};
+
+// Top-k of one token's key row (n candidates, n > k) by the 256 epilogue threads: the
+// radix select and compaction of topk_radix_kernel on keys already in shared memory.
+__device__ __forceinline__ void fused_select_row(const uint32_t* keys, int n, int k, int32_t* out,
+                                                 uint8_t* sel, int tid) {
+    constexpr int NT = 256;
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sel);
+    uint32_t* w_or = hist + 256;
+    uint32_t* w_and = w_or + 8;
+    uint32_t* w_cnt = w_and + 8;
+    uint32_t* s_digit = w_cnt + 8;
+    uint32_t* s_above = s_digit + 1;
+    unsigned long long* warp_tot = reinterpret_cast<unsigned long long*>(s_digit + 4);
+    const EpiSync sync{};
+    uint32_t kor = 0u, kand = 0xffffffffu, cand = 0u;
+    for (int j = tid; j < n; j += NT) {
+        const uint32_t key = keys[j];
+        kor |= key;
+        kand &= key;
+        ++cand;
+    }
+    uint32_t all_or, all_and, n_cand;
+    block_key_stats<NT>(kor, kand, cand, w_or, w_and, w_cnt, all_or, all_and, n_cand, tid, sync);
+    RadixSelect<EpiSync> rs(all_or, all_and, (uint32_t)k, tid, sync);
+    while (rs.active) {
+        rs.clear(hist, NT);
+        for (int j = tid; j < n; j += NT) {
+            const uint32_t key = keys[j];
+            if (key != 0u && (key & rs.digits) == rs.prefix)
+                atomicAdd(&hist[(key >> rs.shift) & 255u], 1u);
+        }
+        rs.step(hist, s_digit, s_above);
+    }
+    const uint32_t thr = rs.thr, need = rs.need;
+    const int per = (n + NT - 1) / NT;
+    const int jb = min(n, tid * per), je = min(n, jb + per);
+    uint32_t gt = 0, eq = 0;
+    for (int j = jb; j < je; ++j) {
+        const uint32_t key = keys[j];
+        gt += key > thr;
+        eq += key == thr;
+    }
+    const unsigned long long before =
+        block_exclusive_scan<NT>(((unsigned long long)gt << 32) | eq, warp_tot, tid, sync);
+    const uint32_t gt_before = (uint32_t)(before >> 32), eq_before = (uint32_t)before;
+    uint32_t pos = gt_before + min(eq_before, need), eq_rank = eq_before;
+    for (int j = jb; j < je; ++j) {
+        const uint32_t key = keys[j];
+        if (key > thr) {
+            out[pos++] = j;
+        } else if (key == thr) {
+            if (eq_rank < need) out[pos++] = j;
+            ++eq_rank;
+        }
+    }
+    // exactly k entries were written (n > k); the scratch is reused by the next row
+    sync();
+}
+
+template <int D_I, int H_I>
+__global__ void __launch_bounds__(FusedTile<D_I, H_I>::THREADS, 1)
+indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                          const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ FusedParams p) {
+    using C = FusedTile<D_I, H_I>;
+    const int b = blockIdx.x;
+    const int u_begin = p.first[b], u_end = p.first[b + 1];
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t base = (raw_u32 + 1023u) & ~1023u;         // 128B-swizzle atoms need 1 KB alignment
+    uint8_t* smem = smem_raw + (base - raw_u32);
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem + C::OFF_KEYS);
+    float* sw = reinterpret_cast<float*>(smem + C::OFF_W);
+    const uint32_t bar0 = base + C::OFF_BAR;
+    auto afull = [&](int s) { return bar0 + 8u * s; };
+    auto aempty = [&](int s) { return bar0 + 8u * (C::A_STAGES + s); };
+    const uint32_t bfull = bar0 + 8u * (2 * C::A_STAGES);
+    const uint32_t bempty = bar0 + 8u * (2 * C::A_STAGES + 1);
+    auto tempty = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + 2 + i); };
+    const uint32_t done_bar = bar0 + 8u * (2 * C::A_STAGES + 4);
+    uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_PTR);
+
+    // Token block tb of the launch: tokens [tok0, tok_end), j-tiles 0 .. n_tiles-1.
+    auto unit_of = [&](int u, int& tok0, int& tok_end, int& n_tiles) {
+        const int tb = p.blk[u];
+        tok0 = p.t0 + tb * C::TB;
+        tok_end = min(tok0 + C::TB, p.t0 + p.n_q);
+        n_tiles = (n_vis(tok_end - 1, p.ratio) + C::BM - 1) / C::BM;
+    };
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::A_STAGES; ++s) {
+            mbar_init(afull(s), 1);
+            mbar_init(aempty(s), 1);
+        }
+        mbar_init(bfull, 1);
+        mbar_init(bempty, 1);
+        for (int i = 0; i < 2; ++i) mbar_init(tempty(i), C::EPI_WARPS);
+        mbar_init(done_bar, 1);
+        *reinterpret_cast<volatile uint32_t*>(smem + C::OFF_SEL + C::SEL_ABORT) = 0u;
+        fence_mbar_init();
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_ptr), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_ptr;
+
+    bool abort = false;
+    if (warp == C::B_WARP || warp == 0) {
+        // ------------------------------------------------------------ TMA producers
+        if (warp == C::B_WARP && lane == 0) {
+            int issued = 0;
+            for (int u = u_begin; u < u_end && !abort; ++u) {
+                int tok0, tok_end, n_tiles;
+                unit_of(u, tok0, tok_end, n_tiles);
+                // the single B buffer is free once the previous unit's MMAs have read it
+                if (!mbar_wait(bempty, ((u - u_begin) & 1) ^ 1, p.wc, abort)) break;
+                mbar_arrive_expect_tx(bfull, C::B_BYTES);
+                for (int ks = 0; ks < C::KSUB; ++ks)
+                    tma_load_2d(base + C::OFF_B + ks * C::B_SUB, &tmap_q, bfull, ks * 64,
+                                (tok0 - p.t0) * H_I);
+                ++issued;
+            }
+            // Every bulk copy this CTA started must land before the CTA exits.
+            if (issued) mbar_wait_drain(bfull, (issued - 1) & 1, p.wc);
+        } else if (warp == 0 && lane == 0) {
+            int a_it = 0;
+            int a_issued[C::A_STAGES] = {};
+            for (int u = u_begin; u < u_end && !abort; ++u) {
+                int tok0, tok_end, n_tiles;
+                unit_of(u, tok0, tok_end, n_tiles);
+                for (int it = 0; it < n_tiles; ++it, ++a_it) {
+                    const int s = a_it % C::A_STAGES;
+                    if (!mbar_wait(aempty(s), ((a_it / C::A_STAGES) & 1) ^ 1, p.wc, abort)) break;
+                    mbar_arrive_expect_tx(afull(s), C::A_STAGE);
+#pragma unroll
+                    for (int ks = 0; ks < C::KSUB; ++ks)
+                        tma_load_2d(base + C::OFF_A + s * C::A_STAGE + ks * C::A_SUB, &tmap_k,
+                                    afull(s), ks * 64, it * C::BM);
+                    ++a_issued[s];
+                }
+            }
+            for (int s = 0; s < C::A_STAGES; ++s)
+                if (a_issued[s]) mbar_wait_drain(afull(s), (a_issued[s] - 1) & 1, p.wc);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint64_t a_desc0 = umma_desc_sw128(base + C::OFF_A);
+            const uint64_t b_desc = umma_desc_sw128(base + C::OFF_B);
+            int tc = 0;
+            for (int u = u_begin; u < u_end && !abort; ++u) {
+                int tok0, tok_end, n_tiles;
+                unit_of(u, tok0, tok_end, n_tiles);
+                if (!mbar_wait(bfull, (u - u_begin) & 1, p.wc, abort)) break;
+                for (int it = 0; it < n_tiles; ++it, ++tc) {
+                    const int buf = tc & 1, s = tc % C::A_STAGES;
+                    if (!mbar_wait(tempty(buf), ((tc >> 1) & 1) ^ 1, p.wc, abort)) break;
+                    if (!mbar_wait(afull(s), (tc / C::A_STAGES) & 1, p.wc, abort)) break;
+                    tc_fence_after();
+                    const uint32_t d = tmem_base + buf * C::BN;
+                    const uint64_t a_desc = a_desc0 + (uint64_t)((s * C::A_STAGE) >> 4);
+#pragma unroll
+                    for (int ks = 0; ks < C::KSUB; ++ks)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_f16(d, a_desc + (uint64_t)((ks * C::A_SUB + kk * 32) >> 4),
+                                     b_desc + (uint64_t)((ks * C::B_SUB + kk * 32) >> 4), C::IDESC,
+                                     ks > 0 || kk > 0);
+                    umma_commit(aempty(s));      // frees the A stage; the accumulator is final
+                }
+                umma_commit(bempty);             // B free once the unit's MMAs finish
+            }
+            umma_commit(done_bar);
+            mbar_wait_drain(done_bar, 0, p.wc);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue + select
+        const int e = warp - 2;                      // 0..7
+        const int etid = threadIdx.x - 64;           // 0..255
+        const int quarter = warp & 3;                // TMEM lanes 32*quarter .. +31
+        const int half = e / 4;                      // columns 128*half .. +127
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + half * 128;
+        const int col = e * 32 + lane;
+        auto unit_weight = [&](int u) {
+            int tok0, tok_end, n_tiles;
+            unit_of(u, tok0, tok_end, n_tiles);
+            const int tl = col / H_I;
+            return (tok0 + tl < tok_end) ? p.w[(size_t)(tok0 - p.t0 + tl) * H_I + (col % H_I)] : 0.f;
+        };
+        uint8_t* sel = smem + C::OFF_SEL;
+        volatile uint32_t* sel_abort = reinterpret_cast<volatile uint32_t*>(sel + C::SEL_ABORT);
+        int tc = 0;
+        float w_next = u_begin < u_end ? unit_weight(u_begin) : 0.f;
+        for (int u = u_begin; u < u_end; ++u) {
+            int tok0, tok_end, n_tiles;
+            unit_of(u, tok0, tok_end, n_tiles);
+            const float w_this = w_next;
+            w_next = u + 1 < u_end ? unit_weight(u + 1) : 0.f;
+            float* swb = sw + ((u - u_begin) & 1) * C::BN;
+            swb[col] = 0.5f * w_this;                // halved: see epilogue_half
+            // also orders the previous unit's select (key reads) before this unit's key writes
+            named_barrier(1, C::EPI_THREADS);
+            const float* wh = swb + half * 128;
+            for (int it = 0; it < n_tiles; ++it, ++tc) {
+                const int buf = tc & 1;
+                const bool ready = mbar_wait(aempty(tc % C::A_STAGES), (tc / C::A_STAGES) & 1,
+                                             p.wc, abort);
+                if (!__all_sync(0xffffffffu, ready)) {           // warp-uniform skip
+                    abort = true;
+                    *sel_abort = 1u;                             // read by all after the barrier
+                    continue;
+                }
+                tc_fence_after();
+                const int j = it * C::BM + quarter * 32 + lane;
+                const int tl_first = half * (128 / H_I);
+                epilogue_tile<H_I>(
+                    lane_addr + buf * C::BN, wh,
+                    [&] {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(tempty(buf));
+                    },
+                    [&](int tk, float score) {
+                        const int tl = tl_first + tk, t = tok0 + tl;
+                        if (t < tok_end && p.ratio * (j + 1) <= t + 1)
+                            keys[tl * p.kld + j] = order_key(score);
+                    });
+            }
+            named_barrier(1, C::EPI_THREADS);       // every key of the unit is in place
+            // A warp that gave up a wait skipped tiles; then no warp runs the select (its
+            // barriers need all eight), and the launch ends with its outputs undefined.
+            if (*sel_abort) continue;
+            for (int tl = 0; tl < tok_end - tok0; ++tl) {
+                const int t = tok0 + tl, n = n_vis(t, p.ratio);
+                int32_t* out = p.topk + (size_t)(t - p.t0) * p.k;
+                if (n <= p.k) {                     // every visible row is kept
+                    for (int s = etid; s < p.k; s += C::EPI_THREADS) out[s] = s < n ? s : -1;
+                    continue;
+                }
+                fused_select_row(keys + tl * p.kld, n, p.k, out, sel, etid);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+}  // namespace ds4sp

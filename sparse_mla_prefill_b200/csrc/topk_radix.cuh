@@ -38,14 +38,22 @@ __device__ __forceinline__ uint32_t order_key(float x) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The select helpers below run on a group of THREADS threads that synchronise through
+// `sync` (the whole block with __syncthreads, or the epilogue warps of the fused indexer
+// with a named barrier); `tid` is the thread's index inside the group (0 .. THREADS-1),
+// and the group starts on a warp boundary.
+struct BlockSync {
+    __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+
 // Block-wide OR and AND of the candidates' keys and their count (every thread gets
 // them): bits where OR and AND agree are the same in every candidate.
-template <int THREADS>
+template <int THREADS, class Sync>
 __device__ __forceinline__ void block_key_stats(uint32_t kor, uint32_t kand, uint32_t cand,
                                                 uint32_t* w_or, uint32_t* w_and, uint32_t* w_cnt,
                                                 uint32_t& all_or, uint32_t& all_and,
-                                                uint32_t& n_cand) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+                                                uint32_t& n_cand, int tid, Sync sync) {
+    const int lane = tid & 31, warp = tid >> 5;
     kor = __reduce_or_sync(0xffffffffu, kor);
     kand = __reduce_and_sync(0xffffffffu, kand);
     cand = __reduce_add_sync(0xffffffffu, cand);
@@ -54,7 +62,7 @@ __device__ __forceinline__ void block_key_stats(uint32_t kor, uint32_t kand, uin
         w_and[warp] = kand;
         w_cnt[warp] = cand;
     }
-    __syncthreads();
+    sync();
     all_or = 0u;
     all_and = 0xffffffffu;
     n_cand = 0u;
@@ -99,7 +107,7 @@ __device__ __forceinline__ void radix_find_digit(const uint32_t* hist, uint32_t 
 // AND all_and. The 8-bit windows run from the highest bit where the candidates differ
 // down to the lowest; bits above the first window are the common prefix, bits below
 // the last are common too. The caller runs the passes:
-//     RadixSelect rs(all_or, all_and, k);
+//     RadixSelect<Sync> rs(all_or, all_and, k, tid, sync);
 //     while (rs.active) {
 //         rs.clear(hist, threads);                      // barrier inside
 //         each key x with x != 0 && (x & rs.digits) == rs.prefix:
@@ -107,13 +115,17 @@ __device__ __forceinline__ void radix_find_digit(const uint32_t* hist, uint32_t 
 //         rs.step(hist, &s_digit, &s_above);            // barriers inside
 //     }
 //     rs.thr, rs.need
+template <class Sync>
 struct RadixSelect {
     uint32_t all_or, digits, prefix, remaining, thr, need;
     int shift, lo_bit;
     bool active;
+    int tid;
+    Sync sync;
 
-    __device__ __forceinline__ RadixSelect(uint32_t or_, uint32_t and_, uint32_t k)
-        : all_or(or_), remaining(k), thr(or_), need(k) {
+    __device__ __forceinline__ RadixSelect(uint32_t or_, uint32_t and_, uint32_t k, int tid_,
+                                           Sync sync_)
+        : all_or(or_), remaining(k), thr(or_), need(k), tid(tid_), sync(sync_) {
         const uint32_t diff = or_ ^ and_;
         active = diff != 0u;                     // all candidates equal: the first k
         const int hi_bit = active ? 31 - __clz(diff) : 0;
@@ -123,18 +135,18 @@ struct RadixSelect {
         shift = max(hi_bit - 7, 0);
     }
     __device__ __forceinline__ void clear(uint32_t* hist, int threads) const {
-        for (int b = threadIdx.x; b < 256; b += threads) hist[b] = 0;
-        __syncthreads();
+        for (int b = tid; b < 256; b += threads) hist[b] = 0;
+        sync();
     }
     __device__ __forceinline__ void step(const uint32_t* hist, uint32_t* s_digit,
                                          uint32_t* s_above) {
-        __syncthreads();                         // the histogram is complete
-        if (threadIdx.x < 32) radix_find_digit(hist, remaining, s_digit, s_above);
-        __syncthreads();
+        sync();                                  // the histogram is complete
+        if (tid < 32) radix_find_digit(hist, remaining, s_digit, s_above);
+        sync();
         prefix |= *s_digit << shift;
         digits |= 255u << shift;
         remaining -= *s_above;
-        __syncthreads();                         // s_digit / hist reused next pass
+        sync();                                  // s_digit / hist reused next pass
         if (shift <= lo_bit) {
             active = false;
             thr = prefix | (all_or & ((1u << shift) - 1u));
@@ -146,10 +158,11 @@ struct RadixSelect {
 };
 
 // Exclusive block scan of a pair of counts packed as (hi << 32 | lo).
-template <int THREADS>
+template <int THREADS, class Sync>
 __device__ __forceinline__ unsigned long long block_exclusive_scan(unsigned long long v,
-                                                                    unsigned long long* warp_tot) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+                                                                    unsigned long long* warp_tot,
+                                                                    int tid, Sync sync) {
+    const int lane = tid & 31, warp = tid >> 5;
     unsigned long long incl = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -157,7 +170,7 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan(unsigned long
         if (lane >= off) incl += o;
     }
     if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
+    sync();
     unsigned long long before = 0;
     for (int w = 0; w < warp; ++w) before += warp_tot[w];
     return before + incl - v;
@@ -211,13 +224,14 @@ topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int
         }
     }
     uint32_t all_or, all_and, n_cand;
-    block_key_stats<THREADS>(kor, kand, cand, w_or, w_and, w_cnt, all_or, all_and, n_cand);
+    block_key_stats<THREADS>(kor, kand, cand, w_or, w_and, w_cnt, all_or, all_and, n_cand, tid,
+                             BlockSync{});
 
     uint32_t thr = 0, need = 0;                  // without selection: every key > 0
     if (n_cand <= (uint32_t)k) {
         keep = (int)n_cand;                      // keep every candidate
     } else {
-        RadixSelect rs(all_or, all_and, (uint32_t)k);
+        RadixSelect<BlockSync> rs(all_or, all_and, (uint32_t)k, tid, BlockSync{});
         while (rs.active) {
             rs.clear(hist, THREADS);
             for (int j = tid; j < n; j += THREADS) {
@@ -240,7 +254,7 @@ topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int
         eq += key == thr;
     }
     const unsigned long long before =
-        block_exclusive_scan<THREADS>(((unsigned long long)gt << 32) | eq, warp_tot);
+        block_exclusive_scan<THREADS>(((unsigned long long)gt << 32) | eq, warp_tot, tid, BlockSync{});
     const uint32_t gt_before = (uint32_t)(before >> 32), eq_before = (uint32_t)before;
     uint32_t pos = gt_before + min(eq_before, need), eq_rank = eq_before;
     for (int j = jb; j < je; ++j) {

@@ -32,7 +32,8 @@ class ds4sp_config(ctypes.Structure):
                 ("ratio", ctypes.c_int), ("n_idx_heads", ctypes.c_int), ("d_idx", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("n_swa", ctypes.c_int), ("band", ctypes.c_int),
                 ("max_tokens", ctypes.c_int), ("softmax_scale", ctypes.c_float),
-                ("exp_mode", ctypes.c_int), ("pv_mode", ctypes.c_int)]
+                ("exp_mode", ctypes.c_int), ("pv_mode", ctypes.c_int),
+                ("topk_mode", ctypes.c_int)]
 
 
 class ds4sp_io(ctypes.Structure):
@@ -64,6 +65,7 @@ _SIGS = {
     "ds4sp_debug_set_wait_limit_ns": (_i32, [_vp, ctypes.c_longlong]),
     "ds4sp_indexer_topk_noalloc": (_i32, [ctypes.POINTER(ds4sp_config), _vp, _vp, _vp, _i32,
                                           _i32, _vp, _vp]),
+    "ds4sp_probe_gather": (_i32, [_vp, _i32, _i32, _vp, _i32, _vp, _i32, _vp]),
     "ds4sp_status_string": (ctypes.c_char_p, [_i32]),
     "ds4sp_last_error": (ctypes.c_char_p, []),
 }
@@ -76,9 +78,11 @@ def header_symbols(path: str = HEADER) -> List[str]:
     return sorted(set(re.findall(r"\b(ds4sp_[a-z_]+)\s*\(", text)))
 
 
-def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load libds4sp.so and declare every signature. Raises if it is missing."""
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libds4sp.so (LIB_PATH unless a path is given) and declare every signature.
+    Raises if it is missing."""
     global _lib
+    path = LIB_PATH if path is None else path
     if _lib is not None and path == LIB_PATH:
         return _lib
     if not os.path.exists(path):
@@ -144,11 +148,13 @@ class Handle:
 def make_config(n_idx_heads: int, d_idx: int, top_k: int, n_swa: int, max_tokens: int,
                 band: int = 2048, softmax_scale: float = 0.0, n_heads: int = 16, d_qk: int = 576,
                 d_v: int = 512, ratio: int = 4, exp_mode: int = 0,
-                pv_mode: int = 0) -> ds4sp_config:
+                pv_mode: int = 0, topk_mode: int = 0) -> ds4sp_config:
     """A ds4sp_config in field order. exp_mode: 0 = ex2.approx, 1 = exp2f for the
-    softmax; pv_mode: 0 = fp16 probabilities in P . V, 1 = fp32-staged (hi + lo fp16)."""
+    softmax; pv_mode: 0 = fp16 probabilities in P . V, 1 = fp32-staged (hi + lo fp16);
+    topk_mode: 0 = scores in the workspace and a separate top-k kernel, 1 = fused
+    indexer + top-k where the call qualifies."""
     return ds4sp_config(n_heads, d_qk, d_v, ratio, n_idx_heads, d_idx, top_k, n_swa, band,
-                        max_tokens, softmax_scale, exp_mode, pv_mode)
+                        max_tokens, softmax_scale, exp_mode, pv_mode, topk_mode)
 
 
 def ds4sp_create(cfg: ds4sp_config) -> Handle:
@@ -269,6 +275,17 @@ def ds4sp_debug_set_mask(h: Handle, mask: Optional[torch.Tensor]) -> None:
     _check(lib.ds4sp_debug_set_mask(h.ptr, _ptr(mask, "mask", torch.uint8), mask.shape[0],
                                     mask.shape[1]), "ds4sp_debug_set_mask")
     h.mask = mask
+
+
+def ds4sp_probe_gather(table, idx, sink, grid: int, stream=None) -> None:
+    """Row-gather bandwidth probe (measurement helper): reads table[idx[i]] for every i
+    (table [rows, row_bytes/2] fp16 or any 2-D tensor with 16-byte-multiple rows) and
+    XORs the words into sink (int32 [1])."""
+    row_bytes = table.shape[1] * table.element_size()
+    _check(load_library().ds4sp_probe_gather(_ptr(table, "table"), table.shape[0], row_bytes,
+                                             _ptr(idx, "idx", torch.int32), idx.numel(),
+                                             _ptr(sink, "sink", torch.int32), grid,
+                                             _stream(stream)), "ds4sp_probe_gather")
 
 
 def ds4sp_status_string(status: int) -> str:

@@ -5,7 +5,9 @@ ld = n_vis(t_last) rounded up to 4 floats, one row per token. With integer-value
 indexer inputs every score is an integer below 2^24, so the fp32 value is exact
 whatever the summation order; each defined column j < n_vis(t) of every token must
 have the bits of oracle.indexer_scores_token_exact (int64 arithmetic) converted to
-fp32. Columns j >= n_vis(t) are not defined and are not read.
+fp32. Columns j >= n_vis(t) are not defined and are not read. (The handles here use
+topk_mode 0, the path that writes the scores; the fused path keeps them on chip and is
+checked through its indices in test_gpu_fused_topk.py.)
 """
 import numpy as np
 import pytest
@@ -59,7 +61,7 @@ def test_scores_every_token(name):
     """Every token of the 256-token (4 x 64 indexer) and 2048-token (64 x 128) workloads."""
     wl = workload(name)
     inp = generate(wl)
-    with handle_for(wl) as h:
+    with handle_for(wl, topk_mode=0) as h:
         scores = _scores_of_call(h, to_device(inp), 0, wl.T, wl.top_k)
     _check_rows(scores, inp, 0, wl.T)
 
@@ -70,6 +72,6 @@ def test_scores_verify_width(q):
     wl = workload("verify")
     inp = generate(wl)                     # per-token tensors of the last 5 positions
     sl = {k: (v[5 - q:].contiguous() if k in ("q", "q_idx", "w") else v) for k, v in inp.items()}
-    with handle_for(wl) as h:
+    with handle_for(wl, topk_mode=0) as h:
         scores = _scores_of_call(h, to_device(sl), wl.T - q, q, wl.top_k)
     _check_rows(scores, sl, wl.T - q, q)
