@@ -35,6 +35,16 @@ or reordering. A reader can check each function against its definition:
   chronological state commit"): bands are scheduling units; running band after
   band gives the one-shot result.
 
+* Quantized KV rows -- "perf(ds4): extend sparse prefill scheduling to 10K",
+  Production workflow ("Q4_0 K/V cache") and its clean-head validation ("Q8 K / Q4
+  V"). The pages name the formats without defining them; this library reads them as
+  block formats of 32 values with one fp16 scale d each: Q8_0 stores q in [-127, 127]
+  with value d*q, d = max|x|/127; Q4_0 stores n in [0, 15] with value d*(n-8), d =
+  m/-8 where m is the block's first value of largest magnitude. Codes are decided in
+  fp32 (x / d rounded half to even), the value is d*q exactly. One latent row serves as
+  key and value, so a quantized cache stores each 576-wide row once
+  (``quantize_rows``, ``dequantize_rows``, ``prefill_tokens_quant``).
+
 Parity pins (tests/test_oracle_*.py) tie each function to something other than
 itself: an explicit mask, exact int64 arithmetic, the ReLU identities
 relu(x)-relu(-x)=x and relu(x)+relu(-x)=|x|, brute-force loops, dense masked
@@ -221,6 +231,117 @@ def sparse_mla_attention(q: np.ndarray, kv_raw: np.ndarray, kv_cmp: np.ndarray,
         rows = attended_rows(t0 + i, topk_idx[i], kv_raw, kv_cmp, n_swa)
         out[i] = attention_token(q[i], rows, sc, d_v)
     return out
+
+
+# --------------------------------------------------------------------------
+# Quantized KV rows (Q8_0, Q4_0)
+# --------------------------------------------------------------------------
+
+QBLOCK = 32
+Q8_0, Q4_0 = 1, 2
+
+
+def quantize_block_q8_0(x: np.ndarray):
+    """One block of 32 values -> (codes int8 [32], scale as fp16).
+
+    d = max|x| / 127 in fp32, stored as fp16; q = x / d in fp32, rounded half to even,
+    clamped to [-127, 127]. An all-zero block has d = 0 and q = 0."""
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(x)))
+    d16 = np.float16(amax / np.float32(127.0))
+    if d16 == 0:
+        return np.zeros(QBLOCK, np.int8), np.float16(0.0)
+    q = np.rint(x / np.float32(d16))
+    return np.clip(q, -127, 127).astype(np.int8), d16
+
+
+def quantize_block_q4_0(x: np.ndarray):
+    """One block of 32 values -> (codes uint8 [32] in 0..15, scale as fp16).
+
+    m = the first value of largest magnitude, d = m / -8 in fp32, stored as fp16;
+    n = x / d in fp32 rounded half to even, plus 8, clamped to [0, 15]; value d*(n-8).
+    An all-zero block has d = 0 and n = 8."""
+    x = np.asarray(x, dtype=np.float32)
+    i = int(np.argmax(np.abs(x)))            # first index of the largest magnitude
+    d16 = np.float16(x[i] / np.float32(-8.0))
+    if d16 == 0:
+        return np.full(QBLOCK, 8, np.uint8), np.float16(0.0)
+    n = np.rint(x / np.float32(d16)) + np.float32(8.0)
+    return np.clip(n, 0, 15).astype(np.uint8), d16
+
+
+def quantize_rows(x: np.ndarray, fmt: int):
+    """Rows [R, D] (D a multiple of 32) -> (codes [R, D], scales fp16 [R, D/32])."""
+    x = np.asarray(x, dtype=np.float32)
+    R, Dm = x.shape
+    f = quantize_block_q8_0 if fmt == Q8_0 else quantize_block_q4_0
+    codes = np.zeros((R, Dm), np.int8 if fmt == Q8_0 else np.uint8)
+    scales = np.zeros((R, Dm // QBLOCK), np.float16)
+    for r in range(R):
+        for b in range(Dm // QBLOCK):
+            codes[r, b * QBLOCK:(b + 1) * QBLOCK], scales[r, b] = f(x[r, b * QBLOCK:(b + 1) * QBLOCK])
+    return codes, scales
+
+
+def dequantize_rows(codes: np.ndarray, scales: np.ndarray, fmt: int) -> np.ndarray:
+    """Values of quantized rows in float64: d*q (Q8_0) or d*(n-8) (Q4_0)."""
+    d = np.repeat(np.asarray(scales, np.float64), QBLOCK, axis=1)
+    q = np.asarray(codes, np.float64)
+    return d * (q if fmt == Q8_0 else q - 8.0)
+
+
+def quant_row_bytes(fmt: int, dims: int) -> int:
+    """Bytes of one stored row: codes, then the fp16 scales, padded to 16 bytes."""
+    code_bytes = dims if fmt == Q8_0 else dims // 2
+    raw = code_bytes + 2 * (dims // QBLOCK)
+    return (raw + 15) // 16 * 16
+
+
+def pack_rows(codes: np.ndarray, scales: np.ndarray, fmt: int) -> np.ndarray:
+    """The stored row layout, uint8 [R, quant_row_bytes]: Q8_0 codes as bytes, or Q4_0
+    codes two per byte (byte b of a block holds value b in its low nibble and value
+    b+16 in its high nibble), then the scales as little-endian fp16, then zeros."""
+    R, Dm = codes.shape
+    out = np.zeros((R, quant_row_bytes(fmt, Dm)), np.uint8)
+    if fmt == Q8_0:
+        out[:, :Dm] = codes.astype(np.int8).view(np.uint8)
+        cb = Dm
+    else:
+        blk = codes.reshape(R, Dm // QBLOCK, QBLOCK).astype(np.uint8)
+        out[:, :Dm // 2] = (blk[:, :, :16] | (blk[:, :, 16:] << 4)).reshape(R, Dm // 2)
+        cb = Dm // 2
+    out[:, cb:cb + 2 * (Dm // QBLOCK)] = np.ascontiguousarray(
+        scales.astype("<f2")).view(np.uint8).reshape(R, -1)
+    return out
+
+
+def unpack_rows(packed: np.ndarray, fmt: int, dims: int):
+    """Inverse of pack_rows: (codes, scales)."""
+    packed = np.asarray(packed, np.uint8)
+    R = packed.shape[0]
+    nb = dims // QBLOCK
+    if fmt == Q8_0:
+        codes = packed[:, :dims].view(np.int8).copy()
+        cb = dims
+    else:
+        b = packed[:, :dims // 2].reshape(R, nb, 16)
+        codes = np.concatenate([b & 15, b >> 4], axis=2).reshape(R, dims)
+        cb = dims // 2
+    scales = np.ascontiguousarray(packed[:, cb:cb + 2 * nb]).view("<f2").astype(np.float16)
+    return codes, scales
+
+
+def prefill_tokens_quant(inputs: Dict[str, np.ndarray], tokens: Iterable[int], top_k: int,
+                         n_swa: int, fmt: int, q_start: int = 0, scale: Optional[float] = None,
+                         d_v: int = 512, ratio: int = RATIO) -> Dict[str, np.ndarray]:
+    """The whole path with a quantized KV cache: kv_raw and kv_cmp are quantized row by
+    row (quantize_rows) and attention reads their dequantized values; the indexer keys
+    are unchanged. Equals prefill_tokens on the dequantized cache."""
+    deq = dict(inputs)
+    for name in ("kv_raw", "kv_cmp"):
+        codes, scales = quantize_rows(inputs[name], fmt)
+        deq[name] = dequantize_rows(codes, scales, fmt)
+    return prefill_tokens(deq, tokens, top_k, n_swa, q_start, scale, d_v, ratio)
 
 
 # --------------------------------------------------------------------------

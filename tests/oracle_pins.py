@@ -317,6 +317,125 @@ def pin_prefill_tokens_composition(o, T: int = 120, s: int = 37):
         assert np.array_equal(got["out"][n], want[0]), t
 
 
+# ------------------------------------------------------------ quantized KV rows
+
+def pin_quant_golden(o):
+    """Hand-derived blocks: half-to-even rounding, clamping, the first-largest-magnitude
+    rule of Q4_0, the scale rounded to fp16, and the Q4_0 nibble order."""
+    with open(os.path.join(GOLDEN, "quant_blocks.txt")) as f:
+        lines = [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+    for ln in lines:
+        kind, xs, cs, sc = [part.strip() for part in ln.split("|")]
+        x = np.zeros(32, np.float32)
+        vals = [float(v) for v in xs.split()]
+        x[:len(vals)] = vals
+        fmt = o.Q8_0 if kind == "q8" else o.Q4_0
+        f = o.quantize_block_q8_0 if fmt == o.Q8_0 else o.quantize_block_q4_0
+        codes, d16 = f(x)
+        assert float(d16) == float(sc), (ln, float(d16))
+        if kind == "q4bytes":
+            packed = o.pack_rows(codes[None].astype(np.uint8), np.array([[d16]], np.float16), fmt)
+            want = [int(v, 16) for v in cs.split()]
+            assert packed[0, :16].tolist() == want, (packed[0, :16].tolist(), want)
+            continue
+        want = [int(v) for v in cs.split()]
+        zero_code = 0 if fmt == o.Q8_0 else 8
+        want = want + [zero_code] * (32 - len(want))
+        assert codes.astype(int).tolist() == want, (ln, codes.tolist())
+
+
+def _dequant_loops(packed, fmt, dims):
+    """Pure-Python reading of the stored row layout, element by element."""
+    import struct
+    nb = dims // 32
+    code_bytes = dims if fmt == 1 else dims // 2
+    out = []
+    for row in packed.tolist():
+        raw = bytes(row)
+        vals = []
+        for b in range(nb):
+            d = struct.unpack("<e", raw[code_bytes + 2 * b: code_bytes + 2 * b + 2])[0]
+            for i in range(32):
+                if fmt == 1:
+                    q = struct.unpack("b", raw[32 * b + i: 32 * b + i + 1])[0]
+                    vals.append(d * q)
+                else:
+                    byte = raw[16 * b + (i % 16)]
+                    n = (byte & 15) if i < 16 else (byte >> 4)
+                    vals.append(d * (n - 8))
+        out.append(vals)
+    return np.array(out, dtype=np.float64)
+
+
+def pin_quant_dequant_bruteforce(o, seed: int = 12):
+    """dequantize_rows(unpack_rows(bytes)) equals a byte-by-byte loop over the layout,
+    on random codes and scales, for both formats and both row widths."""
+    rng = np.random.default_rng(seed)
+    for fmt in (o.Q8_0, o.Q4_0):
+        for dims in (576, 512):
+            R = 3
+            nb = dims // 32
+            packed = np.zeros((R, o.quant_row_bytes(fmt, dims)), np.uint8)
+            cb = dims if fmt == o.Q8_0 else dims // 2
+            packed[:, :cb] = rng.integers(0, 256, (R, cb), dtype=np.uint8)
+            if fmt == o.Q8_0:                  # -128 is not a code
+                packed[:, :cb][packed[:, :cb] == 128] = 129
+            scales = (rng.standard_normal((R, nb)) * 0.1).astype("<f2")
+            packed[:, cb:cb + 2 * nb] = scales.view(np.uint8).reshape(R, -1)
+            got = o.dequantize_rows(*o.unpack_rows(packed, fmt, dims), fmt)
+            want = _dequant_loops(packed, fmt, dims)
+            assert got.shape == (R, dims) and np.array_equal(got, want), (fmt, dims)
+
+
+def pin_quant_properties(o, seed: int = 13):
+    """Codes in range; Q8_0 error <= d/2; the largest magnitude maps to +-127 (Q8_0) or
+    to 0 (Q4_0, the first one); Q4_0 error <= d/2 wherever |x/d| <= 7.5; pack/unpack
+    round trip."""
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((6, 576)) * rng.choice([0.01, 1.0, 40.0], (6, 1))).astype(np.float16)
+    x[0, :32] = 0                                          # an all-zero block
+    for fmt in (o.Q8_0, o.Q4_0):
+        codes, scales = o.quantize_rows(x, fmt)
+        c2, s2 = o.unpack_rows(o.pack_rows(codes, scales, fmt), fmt, 576)
+        assert np.array_equal(codes, c2) and np.array_equal(scales, s2)
+        deq = o.dequantize_rows(codes, scales, fmt)
+        d = np.repeat(np.abs(scales.astype(np.float64)), 32, axis=1)
+        xf = x.astype(np.float64)
+        assert np.all(deq[0, :32] == 0)
+        if fmt == o.Q8_0:
+            assert codes.min() >= -127 and codes.max() <= 127
+            assert np.all(np.abs(xf - deq) <= d * (0.5 + 1e-3))
+            blk = np.abs(xf).reshape(6, 18, 32).argmax(axis=2)
+            top = np.take_along_axis(codes.astype(int).reshape(6, 18, 32), blk[..., None], 2)
+            assert np.all((np.abs(top) == 127) | (scales.reshape(6, 18, 1) == 0))
+        else:
+            assert codes.min() >= 0 and codes.max() <= 15
+            inside = np.abs(xf) <= 7.5 * d
+            assert np.all(np.abs(xf - deq)[inside] <= d[inside] * (0.5 + 1e-3))
+            blk = np.abs(xf).reshape(6, 18, 32).argmax(axis=2)
+            top = np.take_along_axis(codes.astype(int).reshape(6, 18, 32), blk[..., None], 2)
+            assert np.all((top == 0) | (scales.reshape(6, 18, 1) == 0))
+
+
+def pin_quant_path_reduces_to_fp16(o, T: int = 64):
+    """When every cache value is already d * integer with the block's extreme at the
+    code limit, quantizing loses nothing: the quantized path equals prefill_tokens on
+    the original cache, exactly, for both formats."""
+    rng = np.random.default_rng(14)
+    base = _np(generate_small(T, 4, 64, seed=42))
+    for fmt, lim in ((o.Q8_0, 127), (o.Q4_0, 8)):
+        inp = dict(base)
+        for name, rows in (("kv_raw", T), ("kv_cmp", T // 4)):
+            d = np.float16(2.0 ** -6)
+            q = rng.integers(-lim + 1, lim, (rows, 576)).astype(np.float64)
+            q[:, ::32] = -lim                             # each block's first value is the extreme
+            inp[name] = (q * float(d)).astype(np.float16)
+        toks = list(range(0, T, 5))
+        a = o.prefill_tokens_quant(inp, toks, top_k=4, n_swa=5, fmt=fmt)
+        b = o.prefill_tokens(inp, toks, top_k=4, n_swa=5)
+        assert np.array_equal(a["topk"], b["topk"]) and np.array_equal(a["out"], b["out"]), fmt
+
+
 ALL_PINS = [
     pin_visibility_mask, pin_visibility_golden,
     pin_scores_exact, pin_scores_relu_identities, pin_scores_bruteforce,
@@ -324,6 +443,8 @@ ALL_PINS = [
     pin_attention_sdpa_causal, pin_attention_sdpa_window, pin_attention_dense_mask,
     pin_attention_bruteforce, pin_attention_closed_forms,
     pin_bands_equal_oneshot, pin_prefill_tokens_composition,
+    pin_quant_golden, pin_quant_dequant_bruteforce, pin_quant_properties,
+    pin_quant_path_reduces_to_fp16,
 ]
 
 

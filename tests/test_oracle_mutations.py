@@ -141,6 +141,66 @@ def _mut_prefill_inputs_at_position(o):
     o.prefill_tokens = _prefill_with(o, lambda t, i: t, lambda t, i: t)
 
 
+def _mut_q8_round_half_away(o):
+    orig = o.quantize_block_q8_0
+    def f(x):
+        x = np.asarray(x, np.float32)
+        _, d16 = orig(x)
+        if d16 == 0:
+            return np.zeros(32, np.int8), d16
+        q = np.sign(x) * np.floor(np.abs(x / np.float32(d16)) + 0.5)
+        return np.clip(q, -127, 127).astype(np.int8), d16
+    o.quantize_block_q8_0 = f
+
+
+def _mut_q4_scale_sign(o):
+    def f(x):
+        x = np.asarray(x, np.float32)
+        i = int(np.argmax(np.abs(x)))
+        d16 = np.float16(x[i] / np.float32(8.0))
+        if d16 == 0:
+            return np.full(32, 8, np.uint8), d16
+        return np.clip(np.rint(x / np.float32(d16)) + 8, 0, 15).astype(np.uint8), d16
+    o.quantize_block_q4_0 = f
+
+
+def _mut_q4_last_extreme(o):
+    def f(x):
+        x = np.asarray(x, np.float32)
+        a = np.abs(x)
+        i = int(len(a) - 1 - np.argmax(a[::-1]))          # the last largest magnitude
+        d16 = np.float16(x[i] / np.float32(-8.0))
+        if d16 == 0:
+            return np.full(32, 8, np.uint8), d16
+        return np.clip(np.rint(x / np.float32(d16)) + 8, 0, 15).astype(np.uint8), d16
+    o.quantize_block_q4_0 = f
+
+
+def _mut_q4_adjacent_nibbles(o):
+    orig_pack, orig_unpack = o.pack_rows, o.unpack_rows
+    def pack(codes, scales, fmt):
+        out = orig_pack(codes, scales, fmt)
+        if fmt == o.Q4_0:
+            R, Dm = codes.shape
+            c = codes.astype(np.uint8).reshape(R, Dm // 2, 2)
+            out[:, :Dm // 2] = c[:, :, 0] | (c[:, :, 1] << 4)
+        return out
+    def unpack(packed, fmt, dims):
+        codes, scales = orig_unpack(packed, fmt, dims)
+        if fmt == o.Q4_0:
+            b = np.asarray(packed, np.uint8)[:, :dims // 2]
+            codes = np.stack([b & 15, b >> 4], axis=2).reshape(b.shape[0], dims)
+        return codes, scales
+    o.pack_rows, o.unpack_rows = pack, unpack
+
+
+def _mut_q4_no_offset(o):
+    def f(codes, scales, fmt):
+        d = np.repeat(np.asarray(scales, np.float64), 32, axis=1)
+        return d * np.asarray(codes, np.float64)
+    o.dequantize_rows = f
+
+
 MUTATIONS = [
     (_mut_visibility_first_token, [P.pin_visibility_mask, P.pin_visibility_golden]),
     (_mut_no_relu, [P.pin_scores_exact, P.pin_scores_relu_identities, P.pin_scores_bruteforce]),
@@ -156,6 +216,12 @@ MUTATIONS = [
     (_mut_dedup_window, [P.pin_attention_dense_mask, P.pin_attention_closed_forms]),
     (_mut_prefill_window_at_row, [P.pin_prefill_tokens_composition]),
     (_mut_prefill_inputs_at_position, [P.pin_prefill_tokens_composition]),
+    (_mut_q8_round_half_away, [P.pin_quant_golden]),
+    (_mut_q4_scale_sign, [P.pin_quant_golden, P.pin_quant_properties]),
+    (_mut_q4_last_extreme, [P.pin_quant_golden]),
+    (_mut_q4_adjacent_nibbles, [P.pin_quant_golden, P.pin_quant_dequant_bruteforce]),
+    (_mut_q4_no_offset, [P.pin_quant_dequant_bruteforce, P.pin_quant_properties,
+                         P.pin_quant_path_reduces_to_fp16]),
 ]
 
 
