@@ -95,6 +95,18 @@ typedef struct {
                             1,024 token blocks; otherwise the two kernels run. Indices are
                             the same bits either way. Other values are
                             DS4SP_ERR_INVALID_ARG */
+    int kv_format;       /* storage of kv_raw and kv_cmp: 0 = fp16 rows of 576 values
+                            (1152 bytes); 1 = Q8_0 and 2 = Q4_0 quantized rows of
+                            ds4sp_kv_row_bytes(kv_format, 576) bytes (624 and 336), as
+                            ds4sp_quantize_kv writes them. The attention dequantizes the
+                            rows it gathers (value d*q or d*(n-8), rounded once to fp16)
+                            and otherwise computes as for fp16 rows; the indexer keys
+                            (k_idx) stay fp16. Quantized formats need exp_mode 0 and
+                            pv_mode 0 (else DS4SP_ERR_UNSUPPORTED); other values are
+                            DS4SP_ERR_INVALID_ARG ("Q4_0 K/V cache" and "Q8 K / Q4 V",
+                            "perf(ds4): extend sparse prefill scheduling to 10K",
+                            Production workflow and the clean-head validation; the pages
+                            name the formats without defining them) */
 } ds4sp_config;
 
 /* Validate cfg and create a handle bound to the current CUDA device. The handle owns
@@ -270,6 +282,28 @@ ds4sp_status ds4sp_debug_set_mask(ds4sp_handle* h, const uint8_t* mask, int rows
 ds4sp_status ds4sp_indexer_topk_noalloc(const ds4sp_config* cfg, const void* q_idx,
                                         const void* k_idx, const float* w, int t0, int n_q,
                                         int32_t* topk, void* stream);
+
+/* Quantized KV rows. The pages run their model on a quantized cache ("Q4_0 K/V cache",
+ * "Q8 K / Q4 V"; "perf(ds4): extend sparse prefill scheduling to 10K", Production
+ * workflow and the clean-head validation) without defining the formats; this library
+ * reads them as blocks of 32 values with one fp16 scale d each:
+ *   Q8_0 (kv_format 1)  codes q in [-127, 127], value d*q, d = max|x| / 127;
+ *   Q4_0 (kv_format 2)  codes n in [0, 15], value d*(n-8), d = m / -8, m the block's
+ *                       first value of largest magnitude.
+ * Codes are decided in fp32 (x / d, IEEE division, rounded half to even, clamped). A row
+ * is stored as its codes (Q8_0: one byte each; Q4_0: byte b of a block holds value b in
+ * the low nibble and value b+16 in the high nibble), then its fp16 scales, then zeros up
+ * to a multiple of 16 bytes. One latent row is key and value, so a cache stores each
+ * 576-wide row once.
+ *
+ * ds4sp_kv_row_bytes: bytes of one stored row of `dims` values (a multiple of 32, at most
+ * 4096) in kv_format 1 or 2, or 0 for anything else.
+ * ds4sp_quantize_kv: quantize x [rows, dims] fp16 (device) into out [rows,
+ * ds4sp_kv_row_bytes(kv_format, dims)] bytes (device, caller-owned). Asynchronous on
+ * `stream`; argument errors are returned before the launch. */
+int ds4sp_kv_row_bytes(int kv_format, int dims);
+ds4sp_status ds4sp_quantize_kv(const void* x, int rows, int dims, int kv_format, void* out,
+                               void* stream);
 
 /* Measurement helper, not a step of the path: the bandwidth ceiling of the attention
  * kernel's access pattern. Reads n rows of row_bytes (a multiple of 16, at most 1152)

@@ -136,6 +136,11 @@ int score_ld(int t_last, int ratio) {
     return ((nv > 0 ? nv : 1) + 3) / 4 * 4;
 }
 
+// Bytes of one row of kv_raw / kv_cmp in the handle's cache format.
+int kv_row_bytes_of(const ds4sp_config& c) {
+    return c.kv_format == 0 ? c.d_qk * 2 : quant_row_bytes(c.kv_format, c.d_qk);
+}
+
 float scale_of(const ds4sp_config& c) {
     return c.softmax_scale > 0.f ? c.softmax_scale : 1.0f / std::sqrt((float)c.d_qk);
 }
@@ -434,12 +439,15 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
                          const void* prefetch = nullptr, size_t prefetch_bytes = 0) {
     const int smem = attn::smem_bytes(h->cfg.top_k);
     if (!h->smem_set[kAttn]) {
-        // Every instantiation (fast or precise exponentials x fp16 or fp32-staged P),
-        // once per handle.
-        const void* fns[4] = {reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false>),
-                              reinterpret_cast<const void*>(sparse_attn_mma_kernel<true, false>),
-                              reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, true>),
-                              reinterpret_cast<const void*>(sparse_attn_mma_kernel<true, true>)};
+        // Every instantiation (fast or precise exponentials x fp16 or fp32-staged P, and
+        // the two quantized-cache forms), once per handle.
+        const void* fns[6] = {
+            reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtF16>),
+            reinterpret_cast<const void*>(sparse_attn_mma_kernel<true, false, kFmtF16>),
+            reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, true, kFmtF16>),
+            reinterpret_cast<const void*>(sparse_attn_mma_kernel<true, true, kFmtF16>),
+            reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtQ8>),
+            reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtQ4>)};
         for (const void* fn : fns) {
             const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                        attn::smem_bytes(attn::MAX_TOPK));
@@ -470,6 +478,7 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
     p.vis_mask = h->mask;
     p.mask_ld = h->mask_cols;
     p.mask_cols = h->mask ? std::min(h->mask_cols, nvis(t0 + n_q - 1, h->cfg.ratio)) : 0;
+    p.kv_row_bytes = kv_row_bytes_of(h->cfg);
     // Few tokens: one work item per 32-row unit, then a merge per token. The decision
     // and each token's units depend only on the token, so a token's result is the same
     // in every call that takes this path.
@@ -507,11 +516,17 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
         // persistent: one CTA per SM, each walking its share of the work items
         const int grid = std::min(p.n_items, h->sm_count);
         const dim3 g(grid), b(attn::THREADS);
-        switch (2 * h->cfg.pv_mode + h->cfg.exp_mode) {
-            case 0: sparse_attn_mma_kernel<false, false><<<g, b, smem, stream>>>(p); break;
-            case 1: sparse_attn_mma_kernel<true, false><<<g, b, smem, stream>>>(p); break;
-            case 2: sparse_attn_mma_kernel<false, true><<<g, b, smem, stream>>>(p); break;
-            default: sparse_attn_mma_kernel<true, true><<<g, b, smem, stream>>>(p); break;
+        if (h->cfg.kv_format == kFmtQ8) {
+            sparse_attn_mma_kernel<false, false, kFmtQ8><<<g, b, smem, stream>>>(p);
+        } else if (h->cfg.kv_format == kFmtQ4) {
+            sparse_attn_mma_kernel<false, false, kFmtQ4><<<g, b, smem, stream>>>(p);
+        } else {
+            switch (2 * h->cfg.pv_mode + h->cfg.exp_mode) {
+                case 0: sparse_attn_mma_kernel<false, false, kFmtF16><<<g, b, smem, stream>>>(p); break;
+                case 1: sparse_attn_mma_kernel<true, false, kFmtF16><<<g, b, smem, stream>>>(p); break;
+                case 2: sparse_attn_mma_kernel<false, true, kFmtF16><<<g, b, smem, stream>>>(p); break;
+                default: sparse_attn_mma_kernel<true, true, kFmtF16><<<g, b, smem, stream>>>(p); break;
+            }
         }
         if (p.split) attn_merge_kernel<<<n_q * attn::H, 128, 0, stream>>>(mp);
     });
@@ -647,6 +662,10 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
         return fail(DS4SP_ERR_INVALID_ARG, "pv_mode %d (0 = fp16 P, 1 = fp32-staged P)", c.pv_mode);
     if (c.topk_mode != 0 && c.topk_mode != 1)
         return fail(DS4SP_ERR_INVALID_ARG, "topk_mode %d (0 = separate top-k, 1 = fused)", c.topk_mode);
+    if (c.kv_format < 0 || c.kv_format > 2)
+        return fail(DS4SP_ERR_INVALID_ARG, "kv_format %d (0 = fp16, 1 = Q8_0, 2 = Q4_0)", c.kv_format);
+    if (c.kv_format != 0 && (c.exp_mode != 0 || c.pv_mode != 0))
+        return fail(DS4SP_ERR_UNSUPPORTED, "a quantized cache runs with exp_mode 0 and pv_mode 0");
     ds4sp_handle* h = new (std::nothrow) ds4sp_handle();
     if (!h) return fail(DS4SP_ERR_INVALID_ARG, "out of host memory");
     h->cfg = c;
@@ -851,7 +870,7 @@ ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* h
     if (e != cudaSuccess) return cuda_fail(e, "ds4sp_prefill_host: ordering");
 
     const size_t q_row = (size_t)c.n_heads * c.d_qk * 2, qi_row = (size_t)c.n_idx_heads * c.d_idx * 2;
-    const size_t w_row = (size_t)c.n_idx_heads * 4, kv_row = (size_t)c.d_qk * 2;
+    const size_t w_row = (size_t)c.n_idx_heads * 4, kv_row = (size_t)kv_row_bytes_of(c);
     const size_t ki_row = (size_t)c.d_idx * 2, o_row = (size_t)c.n_heads * c.d_v * 4;
     const size_t tk_row = (size_t)c.top_k * 4;
     auto h2d = [&](const void* dst, const void* src, size_t off, size_t bytes) {
@@ -985,6 +1004,33 @@ ds4sp_status ds4sp_debug_set_mask(ds4sp_handle* h, const uint8_t* mask, int rows
     h->mask_rows = rows;
     h->mask_cols = cols;
     return DS4SP_OK;
+}
+
+int ds4sp_kv_row_bytes(int kv_format, int dims) {
+    if ((kv_format != kFmtQ8 && kv_format != kFmtQ4) || dims < kQBlock || dims % kQBlock || dims > 4096)
+        return 0;
+    return quant_row_bytes(kv_format, dims);
+}
+
+ds4sp_status ds4sp_quantize_kv(const void* x, int rows, int dims, int kv_format, void* out,
+                               void* stream) {
+    const TraceRange trace("ds4sp_quantize_kv");
+    const int rb = ds4sp_kv_row_bytes(kv_format, dims);
+    if (rb == 0)
+        return fail(DS4SP_ERR_INVALID_ARG, "kv_format %d with %d dims (1 = Q8_0 or 2 = Q4_0, "
+                    "dims a multiple of 32 up to 4096)", kv_format, dims);
+    if (rows < 0) return fail(DS4SP_ERR_INVALID_ARG, "rows %d", rows);
+    if (rows == 0) return DS4SP_OK;
+    DS4SP_TRY(check_ptr(x, "x"));
+    DS4SP_TRY(check_ptr(out, "out"));
+    const long long n = (long long)rows * (dims / kQBlock);
+    const int threads = 256;
+    const long long grid = (n + threads - 1) / threads;
+    if (grid > 0x7fffffffLL) return fail(DS4SP_ERR_INVALID_ARG, "%d rows is too many", rows);
+    quantize_rows_kernel<<<(unsigned)grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __half*>(x), rows, dims, kv_format, static_cast<uint8_t*>(out));
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? DS4SP_OK : cuda_fail(e, "quantize launch");
 }
 
 ds4sp_status ds4sp_probe_gather(const void* table, int table_rows, int row_bytes,

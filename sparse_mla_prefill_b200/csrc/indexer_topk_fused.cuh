@@ -18,8 +18,8 @@
 // Per unit: the epilogue warps turn each tile's accumulator into order-preserving keys
 // of the scores (the top-k kernel's mapping) in a shared-memory key buffer [tokens of
 // the block][128 x tiles]; after the last tile the same warps run the radix select of
-// topk_radix.cuh on each token's row, 256 threads synchronised by a named barrier, and
-// write the token's indices. Meanwhile the q_idx loader brings the next unit's block
+// topk_radix.cuh, four groups of two warps on four tokens at once (each group with its
+// own named barrier), and write the tokens' indices. Meanwhile the q_idx loader brings the next unit's block
 // into the (single) B buffer as soon as this unit's MMAs have read it, and the MMA warp
 // runs ahead by the two TMEM accumulators.
 // Roles and pipelines are those of indexer_tcgen05_kernel (warp 0 streams k_idx tiles,
@@ -51,17 +51,21 @@ struct FusedTile {
     static constexpr int OFF_KEYS = OFF_A + A_STAGES * A_STAGE;
     static constexpr int OFF_W = OFF_KEYS + KEY_BYTES;            // two w buffers
     static constexpr int OFF_SEL = OFF_W + 2 * BN * 4;            // select scratch
-    // hist[256], w_or/w_and/w_cnt[8], s_digit, s_above, abort flag, pad, warp_tot[8]
-    // (8-byte aligned)
-    static constexpr int SEL_BYTES = 256 * 4 + 3 * 8 * 4 + 4 * 4 + 8 * 8;
-    static constexpr int SEL_ABORT = 256 * 4 + 3 * 8 * 4 + 2 * 4;   // byte offset of the flag
+    // The select runs on SEL_GROUPS groups of SEL_THREADS epilogue threads, one token per
+    // group at a time; per group: hist[256], w_or/w_and/w_cnt[2], s_digit, s_above,
+    // warp_tot[2] (8-byte aligned); after the groups, the abort flag.
+    static constexpr int SEL_GROUPS = 4, SEL_THREADS = EPI_THREADS / SEL_GROUPS;
+    static constexpr int GROUP_SEL = 256 * 4 + 3 * 2 * 4 + 2 * 4 + 2 * 8;
+    static constexpr int SEL_ABORT = SEL_GROUPS * GROUP_SEL;      // byte offset of the flag
+    static constexpr int SEL_BYTES = SEL_ABORT + 16;
     static constexpr int OFF_BAR = OFF_SEL + SEL_BYTES;
     // afull[A_STAGES], aempty[A_STAGES], bfull, bempty, tempty[2], done
     static constexpr int N_BARS = 2 * A_STAGES + 1 + 1 + 2 + 1;
     static constexpr int OFF_TMEM_PTR = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;   // + alignment slack
     static constexpr uint32_t IDESC = T::IDESC;
-    static_assert(SEL_BYTES % 8 == 0 && OFF_SEL % 8 == 0, "8-byte aligned select scratch");
+    static_assert(GROUP_SEL % 8 == 0 && OFF_SEL % 8 == 0, "8-byte aligned select scratch");
+    static_assert(SEL_THREADS == 64, "two warps per select group");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -78,24 +82,25 @@ struct FusedParams {
     uint16_t blk[kFusedMaxBlocks];
 };
 
-// Named barrier of the epilogue warps (they also run the select).
-struct EpiSync {
-    __device__ __forceinline__ void operator()() const { named_barrier(1, 8 * 32); }
+// Named barrier of one select group: two epilogue warps, barrier id 2 + group.
+struct GroupSync {
+    int id;
+    __device__ __forceinline__ void operator()() const { named_barrier(id, 64); }
 };
 
-// Top-k of one token's key row (n candidates, n > k) by the 256 epilogue threads: the
-// radix select and compaction of topk_radix_kernel on keys already in shared memory.
+// Top-k of one token's key row (n candidates, n > k) by one select group of 64 threads:
+// the radix select and compaction of topk_radix_kernel on keys already in shared memory.
+// `sel` is the group's scratch; `tid` the thread's index in the group.
 __device__ __forceinline__ void fused_select_row(const uint32_t* keys, int n, int k, int32_t* out,
-                                                 uint8_t* sel, int tid) {
-    constexpr int NT = 256;
+                                                 uint8_t* sel, int tid, GroupSync sync) {
+    constexpr int NT = 64;
     uint32_t* hist = reinterpret_cast<uint32_t*>(sel);
     uint32_t* w_or = hist + 256;
-    uint32_t* w_and = w_or + 8;
-    uint32_t* w_cnt = w_and + 8;
-    uint32_t* s_digit = w_cnt + 8;
+    uint32_t* w_and = w_or + 2;
+    uint32_t* w_cnt = w_and + 2;
+    uint32_t* s_digit = w_cnt + 2;
     uint32_t* s_above = s_digit + 1;
-    unsigned long long* warp_tot = reinterpret_cast<unsigned long long*>(s_digit + 4);
-    const EpiSync sync{};
+    unsigned long long* warp_tot = reinterpret_cast<unsigned long long*>(s_above + 1);
     uint32_t kor = 0u, kand = 0xffffffffu, cand = 0u;
     for (int j = tid; j < n; j += NT) {
         const uint32_t key = keys[j];
@@ -105,7 +110,7 @@ __device__ __forceinline__ void fused_select_row(const uint32_t* keys, int n, in
     }
     uint32_t all_or, all_and, n_cand;
     block_key_stats<NT>(kor, kand, cand, w_or, w_and, w_cnt, all_or, all_and, n_cand, tid, sync);
-    RadixSelect<EpiSync> rs(all_or, all_and, (uint32_t)k, tid, sync);
+    RadixSelect<GroupSync> rs(all_or, all_and, (uint32_t)k, tid, sync);
     while (rs.active) {
         rs.clear(hist, NT);
         for (int j = tid; j < n; j += NT) {
@@ -307,6 +312,14 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 tc_fence_after();
                 const int j = it * C::BM + quarter * 32 + lane;
                 const int tl_first = half * (128 / H_I);
+                // rows past the last visible row of every token of this warp: skip
+                const int t_warp_last = min(tok0 + tl_first + 128 / H_I, tok_end) - 1;
+                if (p.ratio * (it * C::BM + quarter * 32 + 1) > t_warp_last + 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tempty(buf));
+                    continue;
+                }
                 epilogue_tile<H_I>(
                     lane_addr + buf * C::BN, wh,
                     [&] {
@@ -324,14 +337,17 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
             // A warp that gave up a wait skipped tiles; then no warp runs the select (its
             // barriers need all eight), and the launch ends with its outputs undefined.
             if (*sel_abort) continue;
-            for (int tl = 0; tl < tok_end - tok0; ++tl) {
+            // The block's tokens, one per select group at a time (the groups run at once).
+            const int g = etid / C::SEL_THREADS, gtid = etid % C::SEL_THREADS;
+            for (int tl = g; tl < tok_end - tok0; tl += C::SEL_GROUPS) {
                 const int t = tok0 + tl, n = n_vis(t, p.ratio);
                 int32_t* out = p.topk + (size_t)(t - p.t0) * p.k;
                 if (n <= p.k) {                     // every visible row is kept
-                    for (int s = etid; s < p.k; s += C::EPI_THREADS) out[s] = s < n ? s : -1;
+                    for (int s = gtid; s < p.k; s += C::SEL_THREADS) out[s] = s < n ? s : -1;
                     continue;
                 }
-                fused_select_row(keys + tl * p.kld, n, p.k, out, sel, etid);
+                fused_select_row(keys + tl * p.kld, n, p.k, out, sel + g * C::GROUP_SEL, gtid,
+                                 GroupSync{2 + g});
             }
         }
     }

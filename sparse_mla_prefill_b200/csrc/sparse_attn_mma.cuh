@@ -42,6 +42,7 @@
 #pragma once
 
 #include "device_common.cuh"
+#include "quant_kv.cuh"
 
 namespace ds4sp {
 namespace attn {
@@ -137,6 +138,9 @@ struct AttnParams {
     const uint8_t* vis_mask;
     long long mask_ld;
     int mask_cols;
+    // Quantized cache (kernel instantiations with KVF != 0): kv_raw and kv_cmp hold rows
+    // of quant_row_bytes(KVF, 576) bytes, which the producers dequantize into the ring.
+    int kv_row_bytes;
 };
 
 // A work item: the token (i, t and its rows) and the run of its 32-row units it covers,
@@ -226,8 +230,63 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-// PRECISE selects exp2f for the softmax exponentials instead of ex2.approx.
-template <bool PRECISE, bool PSPLIT>
+// Producer side of a quantized cache: this lane's blocks of one row (lane l of the row's
+// four takes blocks l, l+4, l+8, ...), loaded as 16-byte words, dequantized to fp16 and
+// stored into the ring row as four 16-byte chunks per block; a masked row stores zeros.
+template <int KVF>
+__device__ __forceinline__ void dequant_row_to_ring(const uint8_t* rowq, bool ok, uint32_t dst,
+                                                    int r, int sub) {
+    using namespace attn;
+    constexpr int NB = DQK / kQBlock;                    // 18 blocks
+    constexpr int CB = quant_code_bytes(KVF, DQK);
+    constexpr int W = KVF == kFmtQ8 ? 2 : 1;             // 16-byte words per block
+    constexpr int BATCH = KVF == kFmtQ8 ? 2 : 3;         // blocks whose loads fly together
+    if (!ok) {
+        for (int m = sub; m < NB; m += 4)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) st_shared_v4(chunk_addr(dst, r, 4 * m + k), make_uint4(0, 0, 0, 0));
+        return;
+    }
+    for (int m0 = sub; m0 < NB; m0 += 4 * BATCH) {
+        uint4 c[BATCH][W];
+        __half2 d2[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+            const int m = m0 + 4 * i;
+            if (m < NB) {
+                const uint4* src = reinterpret_cast<const uint4*>(rowq + m * 16 * W);
+#pragma unroll
+                for (int h = 0; h < W; ++h) c[i][h] = __ldg(src + h);
+                d2[i] = __half2half2(*reinterpret_cast<const __half*>(rowq + CB + 2 * m));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+            const int m = m0 + 4 * i;
+            if (m >= NB) continue;
+            if constexpr (KVF == kFmtQ8) {
+                st_shared_v4(chunk_addr(dst, r, 4 * m + 0), dequant_q8_chunk(c[i][0].x, c[i][0].y, d2[i]));
+                st_shared_v4(chunk_addr(dst, r, 4 * m + 1), dequant_q8_chunk(c[i][0].z, c[i][0].w, d2[i]));
+                st_shared_v4(chunk_addr(dst, r, 4 * m + 2), dequant_q8_chunk(c[i][1].x, c[i][1].y, d2[i]));
+                st_shared_v4(chunk_addr(dst, r, 4 * m + 3), dequant_q8_chunk(c[i][1].z, c[i][1].w, d2[i]));
+            } else {
+                const uint4 w = c[i][0];
+                const uint32_t M = 0x0F0F0F0Fu;
+                st_shared_v4(chunk_addr(dst, r, 4 * m + 0), dequant_q4_chunk(w.x & M, w.y & M, d2[i]));
+                st_shared_v4(chunk_addr(dst, r, 4 * m + 1), dequant_q4_chunk(w.z & M, w.w & M, d2[i]));
+                st_shared_v4(chunk_addr(dst, r, 4 * m + 2),
+                             dequant_q4_chunk((w.x >> 4) & M, (w.y >> 4) & M, d2[i]));
+                st_shared_v4(chunk_addr(dst, r, 4 * m + 3),
+                             dequant_q4_chunk((w.z >> 4) & M, (w.w >> 4) & M, d2[i]));
+            }
+        }
+    }
+}
+
+// PRECISE selects exp2f for the softmax exponentials instead of ex2.approx; PSPLIT the
+// fp32-staged probabilities; KVF the cache format (kFmtF16, or a quantized one whose rows
+// the producers dequantize).
+template <bool PRECISE, bool PSPLIT, int KVF>
 __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnParams p) {
     using namespace attn;
     auto exp2_ = [](float x) { return PRECISE ? exp2f(x) : fast_exp2(x); };
@@ -313,35 +372,45 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
             const int* tk = reinterpret_cast<const int*>(smem + idx_buf(mc.turn, cu.m));
             const int r = 8 * pw + (lane >> 2);   // this lane's row of the unit
             const int gr = (cu.tr.u0 + cu.u - 1) * BR + r;
-            const __half* row = p.kv_raw + (size_t)cu.tr.t * DQK;   // valid stand-in
-            bool ok = false;
+            // the row's index: a compressed row (>= 0 from the top-k) or a raw row (-1 - s)
+            long long src_row = 0;
+            bool ok = false, cmp = false;
             if (gr < cu.tr.nsel) {
                 const int j = tk[gr];
                 if (p.vis_mask == nullptr) {
                     if (j >= 0 && j < cu.tr.nv) {
-                        row = p.kv_cmp + (size_t)j * DQK;
-                        ok = true;
+                        src_row = j;
+                        ok = cmp = true;
                     } else if ((lane & 3) == 0) {
                         record_status(p.wc.status, kStatusBounds);
                     }
                 } else if (j >= 0 && j < p.mask_cols) {
                     if (p.vis_mask[(size_t)cu.tr.t * p.mask_ld + j] != 0) {
-                        row = p.kv_cmp + (size_t)j * DQK;
-                        ok = true;
+                        src_row = j;
+                        ok = cmp = true;
                     }
                 } else if (j != -1 && (lane & 3) == 0) {
                     record_status(p.wc.status, kStatusBounds);
                 }
             } else if (gr < cu.tr.nrows) {
-                row = p.kv_raw + (size_t)(cu.tr.s_lo + gr - cu.tr.nsel) * DQK;
+                src_row = cu.tr.s_lo + gr - cu.tr.nsel;
                 ok = true;
             }
+            if constexpr (KVF == kFmtF16) {
+                const __half* row = ok ? (cmp ? p.kv_cmp : p.kv_raw) + (size_t)src_row * DQK
+                                       : p.kv_raw + (size_t)cu.tr.t * DQK;   // valid stand-in
 #pragma unroll
-            for (int m = 0; m < 18; ++m) {
-                const int ch = (lane & 3) + 4 * m;
-                cp_async_16(chunk_addr(dst, r, ch), row + ch * 8, ok);   // zero-filled if masked
+                for (int m = 0; m < 18; ++m) {
+                    const int ch = (lane & 3) + 4 * m;
+                    cp_async_16(chunk_addr(dst, r, ch), row + ch * 8, ok);   // zero-filled if masked
+                }
+                cp_async_arrive_noinc(full_bar(s));
+            } else {
+                const uint8_t* base_q = reinterpret_cast<const uint8_t*>(cmp ? p.kv_cmp : p.kv_raw);
+                dequant_row_to_ring<KVF>(base_q + (size_t)src_row * p.kv_row_bytes, ok, dst, r,
+                                         lane & 3);
+                mbar_arrive(full_bar(s));          // release: this thread's stores are visible
             }
-            cp_async_arrive_noinc(full_bar(s));
             const uint32_t bits = __ballot_sync(0xffffffffu, ok && (lane & 3) == 0);
             if (lane == 0) {
                 uint32_t m8 = 0;

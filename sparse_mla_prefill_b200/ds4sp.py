@@ -33,7 +33,7 @@ class ds4sp_config(ctypes.Structure):
                 ("top_k", ctypes.c_int), ("n_swa", ctypes.c_int), ("band", ctypes.c_int),
                 ("max_tokens", ctypes.c_int), ("softmax_scale", ctypes.c_float),
                 ("exp_mode", ctypes.c_int), ("pv_mode", ctypes.c_int),
-                ("topk_mode", ctypes.c_int)]
+                ("topk_mode", ctypes.c_int), ("kv_format", ctypes.c_int)]
 
 
 class ds4sp_io(ctypes.Structure):
@@ -65,6 +65,8 @@ _SIGS = {
     "ds4sp_debug_set_wait_limit_ns": (_i32, [_vp, ctypes.c_longlong]),
     "ds4sp_indexer_topk_noalloc": (_i32, [ctypes.POINTER(ds4sp_config), _vp, _vp, _vp, _i32,
                                           _i32, _vp, _vp]),
+    "ds4sp_kv_row_bytes": (_i32, [_i32, _i32]),
+    "ds4sp_quantize_kv": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "ds4sp_probe_gather": (_i32, [_vp, _i32, _i32, _vp, _i32, _vp, _i32, _vp]),
     "ds4sp_status_string": (ctypes.c_char_p, [_i32]),
     "ds4sp_last_error": (ctypes.c_char_p, []),
@@ -116,6 +118,11 @@ def _ptr(t: Optional[torch.Tensor], name: str, dtype=None) -> Optional[int]:
     return t.data_ptr()
 
 
+def _kv_dtype(t) -> torch.dtype:
+    """KV tensors are fp16 rows, or uint8 rows of a quantized cache (kv_format 1, 2)."""
+    return torch.uint8 if t is not None and t.dtype == torch.uint8 else torch.float16
+
+
 def _stream(stream=None) -> int:
     s = torch.cuda.current_stream() if stream is None else stream
     return s.cuda_stream
@@ -148,13 +155,14 @@ class Handle:
 def make_config(n_idx_heads: int, d_idx: int, top_k: int, n_swa: int, max_tokens: int,
                 band: int = 2048, softmax_scale: float = 0.0, n_heads: int = 16, d_qk: int = 576,
                 d_v: int = 512, ratio: int = 4, exp_mode: int = 0,
-                pv_mode: int = 0, topk_mode: int = 0) -> ds4sp_config:
+                pv_mode: int = 0, topk_mode: int = 0, kv_format: int = 0) -> ds4sp_config:
     """A ds4sp_config in field order. exp_mode: 0 = ex2.approx, 1 = exp2f for the
     softmax; pv_mode: 0 = fp16 probabilities in P . V, 1 = fp32-staged (hi + lo fp16);
     topk_mode: 0 = scores in the workspace and a separate top-k kernel, 1 = fused
-    indexer + top-k where the call qualifies."""
+    indexer + top-k where the call qualifies; kv_format: 0 = fp16 KV rows, 1 = Q8_0,
+    2 = Q4_0 quantized rows (ds4sp_quantize_kv)."""
     return ds4sp_config(n_heads, d_qk, d_v, ratio, n_idx_heads, d_idx, top_k, n_swa, band,
-                        max_tokens, softmax_scale, exp_mode, pv_mode, topk_mode)
+                        max_tokens, softmax_scale, exp_mode, pv_mode, topk_mode, kv_format)
 
 
 def ds4sp_create(cfg: ds4sp_config) -> Handle:
@@ -200,8 +208,8 @@ def ds4sp_indexer_topk_noalloc(cfg: ds4sp_config, q_idx, k_idx, w, t0: int, n_q:
 def ds4sp_sparse_attn(h: Handle, q, kv_raw, kv_cmp, topk, t0: int, n_q: int, out, stream=None):
     lib = load_library()
     _check(lib.ds4sp_sparse_attn(h.ptr, _ptr(q, "q", torch.float16),
-                                 _ptr(kv_raw, "kv_raw", torch.float16),
-                                 _ptr(kv_cmp, "kv_cmp", torch.float16),
+                                 _ptr(kv_raw, "kv_raw", _kv_dtype(kv_raw)),
+                                 _ptr(kv_cmp, "kv_cmp", _kv_dtype(kv_cmp)),
                                  _ptr(topk, "topk", torch.int32), t0, n_q,
                                  _ptr(out, "out", torch.float32), _stream(stream)),
            "ds4sp_sparse_attn")
@@ -213,8 +221,8 @@ def ds4sp_prefill_band(h: Handle, b: int, n_tokens: int, q, q_idx, w, kv_raw, kv
     _check(lib.ds4sp_prefill_band(h.ptr, b, n_tokens, _ptr(q, "q", torch.float16),
                                   _ptr(q_idx, "q_idx", torch.float16),
                                   _ptr(w, "w", torch.float32),
-                                  _ptr(kv_raw, "kv_raw", torch.float16),
-                                  _ptr(kv_cmp, "kv_cmp", torch.float16),
+                                  _ptr(kv_raw, "kv_raw", _kv_dtype(kv_raw)),
+                                  _ptr(kv_cmp, "kv_cmp", _kv_dtype(kv_cmp)),
                                   _ptr(k_idx, "k_idx", torch.float16),
                                   _ptr(topk, "topk", torch.int32),
                                   _ptr(out, "out", torch.float32), _ptr(ws, "ws"),
@@ -277,6 +285,23 @@ def ds4sp_debug_set_mask(h: Handle, mask: Optional[torch.Tensor]) -> None:
     h.mask = mask
 
 
+def ds4sp_kv_row_bytes(kv_format: int, dims: int) -> int:
+    return int(load_library().ds4sp_kv_row_bytes(kv_format, dims))
+
+
+def ds4sp_quantize_kv(x, kv_format: int, out=None, stream=None):
+    """Quantize fp16 rows x [rows, dims] (device) into the stored row layout; returns
+    ``out`` (uint8 [rows, ds4sp_kv_row_bytes(kv_format, dims)], allocated if None)."""
+    rows, dims = x.shape
+    rb = ds4sp_kv_row_bytes(kv_format, dims)
+    if out is None:
+        out = torch.empty((rows, max(rb, 16)), dtype=torch.uint8, device=x.device)
+    _check(load_library().ds4sp_quantize_kv(_ptr(x, "x", torch.float16), rows, dims, kv_format,
+                                            _ptr(out, "out", torch.uint8), _stream(stream)),
+           "ds4sp_quantize_kv")
+    return out
+
+
 def ds4sp_probe_gather(table, idx, sink, grid: int, stream=None) -> None:
     """Row-gather bandwidth probe (measurement helper): reads table[idx[i]] for every i
     (table [rows, row_bytes/2] fp16 or any 2-D tensor with 16-byte-multiple rows) and
@@ -329,8 +354,9 @@ def _io(t: Dict[str, torch.Tensor], topk: Optional[torch.Tensor], out: torch.Ten
             raise ValueError(f"{name}: expected a contiguous {dtype} tensor")
         return x.data_ptr()
     f16, f32, i32 = torch.float16, torch.float32, torch.int32
+    kvt = t["kv_raw"].dtype if t["kv_raw"].dtype == torch.uint8 else f16   # quantized rows
     return ds4sp_io(ptr("q", t["q"], f16), ptr("q_idx", t["q_idx"], f16), ptr("w", t["w"], f32),
-                    ptr("kv_raw", t["kv_raw"], f16), ptr("kv_cmp", t.get("kv_cmp"), f16),
+                    ptr("kv_raw", t["kv_raw"], kvt), ptr("kv_cmp", t.get("kv_cmp"), kvt),
                     ptr("k_idx", t.get("k_idx"), f16), ptr("topk", topk, i32), ptr("out", out, f32))
 
 
