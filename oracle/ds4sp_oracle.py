@@ -42,8 +42,12 @@ or reordering. A reader can check each function against its definition:
   with value d*q, d = max|x|/127; Q4_0 stores n in [0, 15] with value d*(n-8), d =
   m/-8 where m is the block's first value of largest magnitude. Codes are decided in
   fp32 (x / d rounded half to even), the value is d*q exactly. One latent row serves as
-  key and value, so a quantized cache stores each 576-wide row once
-  (``quantize_rows``, ``dequantize_rows``, ``prefill_tokens_quant``).
+  key and value, so a Q8_0 or Q4_0 cache stores each 576-wide row once
+  (``quantize_rows``, ``dequantize_rows``, ``prefill_tokens_quant``). The "Q8 K / Q4 V"
+  form keeps keys and values at different precisions: a stored row is the Q8_0 row of
+  all 576 values (the key) followed by the Q4_0 row of its first 512 (the value), and
+  attention takes logits from the first and values from the second
+  (``attention_token_kv``).
 
 Parity pins (tests/test_oracle_*.py) tie each function to something other than
 itself: an explicit mask, exact int64 arithmetic, the ReLU identities
@@ -238,7 +242,7 @@ def sparse_mla_attention(q: np.ndarray, kv_raw: np.ndarray, kv_cmp: np.ndarray,
 # --------------------------------------------------------------------------
 
 QBLOCK = 32
-Q8_0, Q4_0 = 1, 2
+Q8_0, Q4_0, Q8K_Q4V = 1, 2, 3
 
 
 def quantize_block_q8_0(x: np.ndarray):
@@ -291,7 +295,10 @@ def dequantize_rows(codes: np.ndarray, scales: np.ndarray, fmt: int) -> np.ndarr
 
 
 def quant_row_bytes(fmt: int, dims: int) -> int:
-    """Bytes of one stored row: codes, then the fp16 scales, padded to 16 bytes."""
+    """Bytes of one stored row: codes, then the fp16 scales, padded to 16 bytes (for
+    Q8K_Q4V: the Q8_0 row of the `dims` values, then the Q4_0 row of the first 512)."""
+    if fmt == Q8K_Q4V:
+        return quant_row_bytes(Q8_0, dims) + quant_row_bytes(Q4_0, 512)
     code_bytes = dims if fmt == Q8_0 else dims // 2
     raw = code_bytes + 2 * (dims // QBLOCK)
     return (raw + 15) // 16 * 16
@@ -331,17 +338,52 @@ def unpack_rows(packed: np.ndarray, fmt: int, dims: int):
     return codes, scales
 
 
+def kv_values(rows: np.ndarray, fmt: int, d_v: int = 512):
+    """(key rows [R, 576], value rows [R, d_v]) in float64 as a cache of format `fmt`
+    holds them: Q8_0 / Q4_0 dequantize one row that serves as both; Q8K_Q4V takes the key
+    from the Q8_0 row and the value from the Q4_0 row of the first d_v values."""
+    if fmt == Q8K_Q4V:
+        k = dequantize_rows(*quantize_rows(rows, Q8_0), Q8_0)
+        v = dequantize_rows(*quantize_rows(np.asarray(rows)[:, :d_v], Q4_0), Q4_0)
+        return k, v
+    deq = dequantize_rows(*quantize_rows(rows, fmt), fmt)
+    return deq, deq[:, :d_v]
+
+
+def attention_token_kv(q_t: np.ndarray, krows: np.ndarray, vrows: np.ndarray,
+                       scale: float) -> np.ndarray:
+    """Softmax attention of 16 heads over shared rows with separate keys and values,
+    float64: logits = scale * q_t @ krows^T, stable softmax over the rows, P @ vrows."""
+    q = np.asarray(q_t, dtype=np.float64)
+    logits = scale * (q @ np.asarray(krows, np.float64).T)
+    logits = logits - logits.max(axis=1, keepdims=True)
+    p = np.exp(logits)
+    p = p / p.sum(axis=1, keepdims=True)
+    return p @ np.asarray(vrows, np.float64)
+
+
 def prefill_tokens_quant(inputs: Dict[str, np.ndarray], tokens: Iterable[int], top_k: int,
                          n_swa: int, fmt: int, q_start: int = 0, scale: Optional[float] = None,
                          d_v: int = 512, ratio: int = RATIO) -> Dict[str, np.ndarray]:
     """The whole path with a quantized KV cache: kv_raw and kv_cmp are quantized row by
-    row (quantize_rows) and attention reads their dequantized values; the indexer keys
-    are unchanged. Equals prefill_tokens on the dequantized cache."""
-    deq = dict(inputs)
-    for name in ("kv_raw", "kv_cmp"):
-        codes, scales = quantize_rows(inputs[name], fmt)
-        deq[name] = dequantize_rows(codes, scales, fmt)
-    return prefill_tokens(deq, tokens, top_k, n_swa, q_start, scale, d_v, ratio)
+    row and attention reads the values the cache holds (kv_values); the indexer keys
+    are unchanged. Per token: indexer scores -> top-k -> the attended key rows and value
+    rows (selected compressed rows, then the window) -> attention_token_kv."""
+    tokens = list(tokens)
+    q, q_idx, w = inputs["q"], inputs["q_idx"], inputs["w"]
+    k_raw, v_raw = kv_values(inputs["kv_raw"], fmt, d_v)
+    k_cmp, v_cmp = kv_values(inputs["kv_cmp"], fmt, d_v)
+    sc = default_scale(q.shape[2]) if scale is None else scale
+    idx = np.zeros((len(tokens), top_k), dtype=np.int32)
+    out = np.zeros((len(tokens), q.shape[1], d_v), dtype=np.float64)
+    for n, t in enumerate(tokens):
+        i = t - q_start
+        s_t = indexer_scores_token(q_idx[i], inputs["k_idx"], w[i], t, ratio)
+        idx[n] = topk_row(s_t, top_k)
+        krows = attended_rows(t, idx[n], k_raw, k_cmp, n_swa)
+        vrows = attended_rows(t, idx[n], v_raw, v_cmp, n_swa)
+        out[n] = attention_token_kv(q[i], krows, vrows, sc)
+    return {"tokens": np.asarray(tokens, dtype=np.int64), "topk": idx, "out": out}
 
 
 # --------------------------------------------------------------------------

@@ -436,6 +436,48 @@ def pin_quant_path_reduces_to_fp16(o, T: int = 64):
         assert np.array_equal(a["topk"], b["topk"]) and np.array_equal(a["out"], b["out"]), fmt
 
 
+def _sdpa_rows(q_t, krows, vrows, scale):
+    """torch scaled_dot_product_attention in float64: 16 heads over one set of rows."""
+    Q = torch.from_numpy(np.asarray(q_t, np.float64))[None, :, None, :]          # [1,16,1,576]
+    K = torch.from_numpy(np.asarray(krows, np.float64))[None, None].expand(1, 16, -1, -1)
+    V = torch.from_numpy(np.asarray(vrows, np.float64))[None, None].expand(1, 16, -1, -1)
+    return torch.nn.functional.scaled_dot_product_attention(Q, K, V, scale=scale)[0, :, 0].numpy()
+
+
+def pin_attention_kv_sdpa(o):
+    """Separate keys and values: attention_token_kv equals torch SDPA with distinct K and V,
+    and with V = the keys' first 512 values it equals attention_token."""
+    q, kv_raw, kv_cmp = _attn_case(40, seed=26)
+    rng = np.random.default_rng(3)
+    krows = kv_raw[:37]
+    vrows = rng.standard_normal((37, 512))
+    got = o.attention_token_kv(q[5], krows, vrows, 0.06)
+    assert np.abs(got - _sdpa_rows(q[5], krows, vrows, 0.06)).max() < 1e-12
+    same = o.attention_token_kv(q[6], krows, krows[:, :512], 1.0 / 24.0)
+    assert np.abs(same - o.attention_token(q[6], krows, 1.0 / 24.0, 512)).max() < 1e-13
+
+
+def pin_quant_kv_split_composition(o, T: int = 48):
+    """The Q8 K / Q4 V path for every token equals, built here step by step: keys from
+    the Q8_0 rows, values from the Q4_0 rows of the first 512 values, the token's
+    selected compressed rows then its window, and torch SDPA over them."""
+    inp = _np(generate_small(T, 4, 64, seed=43))
+    k, n_swa = 5, 7
+    got = o.prefill_tokens_quant(inp, range(T), top_k=k, n_swa=n_swa, fmt=o.Q8K_Q4V)
+    kq = {n: o.dequantize_rows(*o.quantize_rows(inp[n], o.Q8_0), o.Q8_0) for n in ("kv_raw", "kv_cmp")}
+    vq = {n: o.dequantize_rows(*o.quantize_rows(inp[n][:, :512], o.Q4_0), o.Q4_0)
+          for n in ("kv_raw", "kv_cmp")}
+    for t in range(T):
+        idx = o.topk_row(o.indexer_scores_token(inp["q_idx"][t], inp["k_idx"], inp["w"][t], t), k)
+        assert np.array_equal(got["topk"][t], idx), t
+        sel = [j for j in idx if j >= 0]
+        win = list(range(max(0, t - n_swa + 1), t + 1))
+        krows = np.concatenate([kq["kv_cmp"][sel], kq["kv_raw"][win]])
+        vrows = np.concatenate([vq["kv_cmp"][sel], vq["kv_raw"][win]])
+        want = _sdpa_rows(inp["q"][t], krows, vrows, 1.0 / 24.0)
+        assert np.abs(got["out"][t] - want).max() < 1e-12, t
+
+
 ALL_PINS = [
     pin_visibility_mask, pin_visibility_golden,
     pin_scores_exact, pin_scores_relu_identities, pin_scores_bruteforce,
@@ -444,7 +486,7 @@ ALL_PINS = [
     pin_attention_bruteforce, pin_attention_closed_forms,
     pin_bands_equal_oneshot, pin_prefill_tokens_composition,
     pin_quant_golden, pin_quant_dequant_bruteforce, pin_quant_properties,
-    pin_quant_path_reduces_to_fp16,
+    pin_quant_path_reduces_to_fp16, pin_attention_kv_sdpa, pin_quant_kv_split_composition,
 ]
 
 

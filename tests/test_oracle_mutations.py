@@ -201,6 +201,19 @@ def _mut_q4_no_offset(o):
     o.dequantize_rows = f
 
 
+def _mut_split_values_from_keys(o):
+    # The Q8 K / Q4 V cache read with the values taken from the Q8_0 key rows.
+    orig = o.kv_values
+    def f(rows, fmt, d_v=512):
+        k, v = orig(rows, fmt, d_v)
+        return (k, k[:, :d_v]) if fmt == o.Q8K_Q4V else (k, v)
+    o.kv_values = f
+
+
+def _mut_kv_attention_values_from_keys(o):
+    o.attention_token_kv = lambda q_t, krows, vrows, scale: o.attention_token(q_t, krows, scale, 512)
+
+
 MUTATIONS = [
     (_mut_visibility_first_token, [P.pin_visibility_mask, P.pin_visibility_golden]),
     (_mut_no_relu, [P.pin_scores_exact, P.pin_scores_relu_identities, P.pin_scores_bruteforce]),
@@ -222,6 +235,8 @@ MUTATIONS = [
     (_mut_q4_adjacent_nibbles, [P.pin_quant_golden, P.pin_quant_dequant_bruteforce]),
     (_mut_q4_no_offset, [P.pin_quant_dequant_bruteforce, P.pin_quant_properties,
                          P.pin_quant_path_reduces_to_fp16]),
+    (_mut_split_values_from_keys, [P.pin_quant_kv_split_composition]),
+    (_mut_kv_attention_values_from_keys, [P.pin_attention_kv_sdpa]),
 ]
 
 
