@@ -585,6 +585,7 @@ VARIANTS = [
     ("fp32_staged_pv_exp2f", dict(pv_mode=1, exp_mode=1)),
     ("q8_0_cache", dict(kv_format=1)),
     ("q4_0_cache", dict(kv_format=2)),
+    ("q8k_q4v_cache", dict(kv_format=3)),
 ]
 
 

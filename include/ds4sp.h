@@ -96,17 +96,20 @@ typedef struct {
                             the same bits either way. Other values are
                             DS4SP_ERR_INVALID_ARG */
     int kv_format;       /* storage of kv_raw and kv_cmp: 0 = fp16 rows of 576 values
-                            (1152 bytes); 1 = Q8_0 and 2 = Q4_0 quantized rows of
-                            ds4sp_kv_row_bytes(kv_format, 576) bytes (624 and 336), as
-                            ds4sp_quantize_kv writes them. The attention dequantizes the
-                            rows it gathers (value d*q or d*(n-8), rounded once to fp16)
-                            and otherwise computes as for fp16 rows; the indexer keys
-                            (k_idx) stay fp16. Quantized formats need exp_mode 0 and
-                            pv_mode 0 (else DS4SP_ERR_UNSUPPORTED); other values are
-                            DS4SP_ERR_INVALID_ARG ("Q4_0 K/V cache" and "Q8 K / Q4 V",
-                            "perf(ds4): extend sparse prefill scheduling to 10K",
-                            Production workflow and the clean-head validation; the pages
-                            name the formats without defining them) */
+                            (1152 bytes); 1 = Q8_0 and 2 = Q4_0 quantized rows (one row
+                            is key and value), 3 = "Q8 K / Q4 V" rows (the Q8_0 row of the
+                            576 values is the key, the Q4_0 row of the first 512 the
+                            value), of ds4sp_kv_row_bytes(kv_format, 576) bytes (624, 336,
+                            912), as ds4sp_quantize_kv writes them. The attention
+                            dequantizes the rows it gathers (value d*q or d*(n-8), rounded
+                            once to fp16) and otherwise computes as for fp16 rows; the
+                            indexer keys (k_idx) stay fp16. Quantized formats need
+                            exp_mode 0 and pv_mode 0, and format 3 top_k <= 824 (else
+                            DS4SP_ERR_UNSUPPORTED); other values are DS4SP_ERR_INVALID_ARG
+                            ("Q4_0 K/V cache" and "Q8 K / Q4 V", "perf(ds4): extend sparse
+                            prefill scheduling to 10K", Production workflow and the
+                            clean-head validation; the pages name the formats without
+                            defining them) */
 } ds4sp_config;
 
 /* Validate cfg and create a handle bound to the current CUDA device. The handle owns
@@ -293,11 +296,12 @@ ds4sp_status ds4sp_indexer_topk_noalloc(const ds4sp_config* cfg, const void* q_i
  * Codes are decided in fp32 (x / d, IEEE division, rounded half to even, clamped). A row
  * is stored as its codes (Q8_0: one byte each; Q4_0: byte b of a block holds value b in
  * the low nibble and value b+16 in the high nibble), then its fp16 scales, then zeros up
- * to a multiple of 16 bytes. One latent row is key and value, so a cache stores each
- * 576-wide row once.
+ * to a multiple of 16 bytes. In formats 1 and 2 one latent row is key and value, so a
+ * cache stores each 576-wide row once; format 3 ("Q8 K / Q4 V") stores the Q8_0 row of
+ * the 576 values (the key) followed by the Q4_0 row of its first 512 (the value).
  *
  * ds4sp_kv_row_bytes: bytes of one stored row of `dims` values (a multiple of 32, at most
- * 4096) in kv_format 1 or 2, or 0 for anything else.
+ * 4096; at least 512 for format 3) in kv_format 1, 2 or 3, or 0 for anything else.
  * ds4sp_quantize_kv: quantize x [rows, dims] fp16 (device) into out [rows,
  * ds4sp_kv_row_bytes(kv_format, dims)] bytes (device, caller-owned). Asynchronous on
  * `stream`; argument errors are returned before the launch. */

@@ -338,6 +338,17 @@ def unpack_rows(packed: np.ndarray, fmt: int, dims: int):
     return codes, scales
 
 
+def cache_rows(rows: np.ndarray, fmt: int, d_v: int = 512) -> np.ndarray:
+    """The stored bytes of rows [R, dims] in cache format `fmt`: pack_rows of the
+    quantized rows (Q8_0, Q4_0), or for Q8K_Q4V the Q8_0 row of all values followed by
+    the Q4_0 row of the first d_v."""
+    rows = np.asarray(rows)
+    if fmt == Q8K_Q4V:
+        return np.concatenate([pack_rows(*quantize_rows(rows, Q8_0), Q8_0),
+                               pack_rows(*quantize_rows(rows[:, :d_v], Q4_0), Q4_0)], axis=1)
+    return pack_rows(*quantize_rows(rows, fmt), fmt)
+
+
 def kv_values(rows: np.ndarray, fmt: int, d_v: int = 512):
     """(key rows [R, 576], value rows [R, d_v]) in float64 as a cache of format `fmt`
     holds them: Q8_0 / Q4_0 dequantize one row that serves as both; Q8K_Q4V takes the key

@@ -437,20 +437,26 @@ ds4sp_status launch_topk(ds4sp_handle* h, const float* scores, int ld, int t0, i
 ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, const void* kv_cmp,
                          const int32_t* topk, int t0, int n_q, float* out, cudaStream_t stream,
                          const void* prefetch = nullptr, size_t prefetch_bytes = 0) {
-    const int smem = attn::smem_bytes(h->cfg.top_k);
+    const int kvf = h->cfg.kv_format;
+    const int smem = kvf == kFmtQ8Q4 ? attn::RingLayout<kFmtQ8Q4>::smem_bytes(h->cfg.top_k)
+                                     : attn::smem_bytes(h->cfg.top_k);
     if (!h->smem_set[kAttn]) {
         // Every instantiation (fast or precise exponentials x fp16 or fp32-staged P, and
         // the two quantized-cache forms), once per handle.
-        const void* fns[6] = {
+        const void* fns[7] = {
             reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtF16>),
             reinterpret_cast<const void*>(sparse_attn_mma_kernel<true, false, kFmtF16>),
             reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, true, kFmtF16>),
             reinterpret_cast<const void*>(sparse_attn_mma_kernel<true, true, kFmtF16>),
             reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtQ8>),
-            reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtQ4>)};
+            reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtQ4>),
+            reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtQ8Q4>)};
         for (const void* fn : fns) {
+            const int max_smem = fn == fns[6] ? attn::RingLayout<kFmtQ8Q4>::smem_bytes(
+                                                    attn::RingLayout<kFmtQ8Q4>::MAX_K)
+                                              : attn::smem_bytes(attn::MAX_TOPK);
             const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       attn::smem_bytes(attn::MAX_TOPK));
+                                                       max_smem);
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention)");
             cudaFuncAttributes fa;
             const cudaError_t ea = cudaFuncGetAttributes(&fa, fn);
@@ -520,6 +526,8 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
             sparse_attn_mma_kernel<false, false, kFmtQ8><<<g, b, smem, stream>>>(p);
         } else if (h->cfg.kv_format == kFmtQ4) {
             sparse_attn_mma_kernel<false, false, kFmtQ4><<<g, b, smem, stream>>>(p);
+        } else if (h->cfg.kv_format == kFmtQ8Q4) {
+            sparse_attn_mma_kernel<false, false, kFmtQ8Q4><<<g, b, smem, stream>>>(p);
         } else {
             switch (2 * h->cfg.pv_mode + h->cfg.exp_mode) {
                 case 0: sparse_attn_mma_kernel<false, false, kFmtF16><<<g, b, smem, stream>>>(p); break;
@@ -662,8 +670,12 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
         return fail(DS4SP_ERR_INVALID_ARG, "pv_mode %d (0 = fp16 P, 1 = fp32-staged P)", c.pv_mode);
     if (c.topk_mode != 0 && c.topk_mode != 1)
         return fail(DS4SP_ERR_INVALID_ARG, "topk_mode %d (0 = separate top-k, 1 = fused)", c.topk_mode);
-    if (c.kv_format < 0 || c.kv_format > 2)
-        return fail(DS4SP_ERR_INVALID_ARG, "kv_format %d (0 = fp16, 1 = Q8_0, 2 = Q4_0)", c.kv_format);
+    if (c.kv_format < 0 || c.kv_format > 3)
+        return fail(DS4SP_ERR_INVALID_ARG, "kv_format %d (0 = fp16, 1 = Q8_0, 2 = Q4_0, 3 = Q8 K / Q4 V)",
+                    c.kv_format);
+    if (c.kv_format == kFmtQ8Q4 && c.top_k > attn::RingLayout<kFmtQ8Q4>::MAX_K)
+        return fail(DS4SP_ERR_UNSUPPORTED, "kv_format 3 supports top_k up to %d",
+                    attn::RingLayout<kFmtQ8Q4>::MAX_K);
     if (c.kv_format != 0 && (c.exp_mode != 0 || c.pv_mode != 0))
         return fail(DS4SP_ERR_UNSUPPORTED, "a quantized cache runs with exp_mode 0 and pv_mode 0");
     ds4sp_handle* h = new (std::nothrow) ds4sp_handle();
@@ -1007,8 +1019,9 @@ ds4sp_status ds4sp_debug_set_mask(ds4sp_handle* h, const uint8_t* mask, int rows
 }
 
 int ds4sp_kv_row_bytes(int kv_format, int dims) {
-    if ((kv_format != kFmtQ8 && kv_format != kFmtQ4) || dims < kQBlock || dims % kQBlock || dims > 4096)
+    if (kv_format < kFmtQ8 || kv_format > kFmtQ8Q4 || dims < kQBlock || dims % kQBlock || dims > 4096)
         return 0;
+    if (kv_format == kFmtQ8Q4 && dims < kValueDims) return 0;
     return quant_row_bytes(kv_format, dims);
 }
 
@@ -1023,14 +1036,28 @@ ds4sp_status ds4sp_quantize_kv(const void* x, int rows, int dims, int kv_format,
     if (rows == 0) return DS4SP_OK;
     DS4SP_TRY(check_ptr(x, "x"));
     DS4SP_TRY(check_ptr(out, "out"));
-    const long long n = (long long)rows * (dims / kQBlock);
-    const int threads = 256;
-    const long long grid = (n + threads - 1) / threads;
-    if (grid > 0x7fffffffLL) return fail(DS4SP_ERR_INVALID_ARG, "%d rows is too many", rows);
-    quantize_rows_kernel<<<(unsigned)grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const __half*>(x), rows, dims, kv_format, static_cast<uint8_t*>(out));
-    const cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? DS4SP_OK : cuda_fail(e, "quantize launch");
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // (format, values, byte offset) of each part of a stored row
+    struct Part { int fmt, dims, off; };
+    Part parts[2] = {{kv_format, dims, 0}, {0, 0, 0}};
+    int n_parts = 1;
+    if (kv_format == kFmtQ8Q4) {
+        parts[0] = {kFmtQ8, dims, 0};
+        parts[1] = {kFmtQ4, kValueDims, quant_row_bytes(kFmtQ8, dims)};
+        n_parts = 2;
+    }
+    for (int i = 0; i < n_parts; ++i) {
+        const long long n = (long long)rows * (parts[i].dims / kQBlock);
+        const int threads = 256;
+        const long long grid = (n + threads - 1) / threads;
+        if (grid > 0x7fffffffLL) return fail(DS4SP_ERR_INVALID_ARG, "%d rows is too many", rows);
+        quantize_rows_kernel<<<(unsigned)grid, threads, 0, st>>>(
+            static_cast<const __half*>(x), dims, rows, parts[i].dims, parts[i].fmt,
+            static_cast<uint8_t*>(out), rb, parts[i].off);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+    }
+    return DS4SP_OK;
 }
 
 ds4sp_status ds4sp_probe_gather(const void* table, int table_rows, int row_bytes,

@@ -22,26 +22,33 @@
 namespace ds4sp {
 
 constexpr int kQBlock = 32;
-constexpr int kFmtF16 = 0, kFmtQ8 = 1, kFmtQ4 = 2;
+// kFmtQ8Q4 ("Q8 K / Q4 V"): keys and values at different precisions. A stored row is the
+// Q8_0 row of all the latent values (the key) followed by the Q4_0 row of the first 512
+// (the value).
+constexpr int kFmtF16 = 0, kFmtQ8 = 1, kFmtQ4 = 2, kFmtQ8Q4 = 3;
+constexpr int kValueDims = 512;
 
 __host__ __device__ constexpr int quant_code_bytes(int fmt, int dims) {
     return fmt == kFmtQ8 ? dims : dims / 2;
 }
 __host__ __device__ constexpr int quant_row_bytes(int fmt, int dims) {
-    return (quant_code_bytes(fmt, dims) + 2 * (dims / kQBlock) + 15) / 16 * 16;
+    return fmt == kFmtQ8Q4 ? quant_row_bytes(kFmtQ8, dims) + quant_row_bytes(kFmtQ4, kValueDims)
+                           : (quant_code_bytes(fmt, dims) + 2 * (dims / kQBlock) + 15) / 16 * 16;
 }
 
-// One thread per (row, block): quantize 32 fp16 values and store codes and scale.
+// One thread per (row, block): quantize 32 fp16 values of row r (values dims, stride
+// x_ld) in format fmt (Q8_0 or Q4_0) into the part of an output row of out_ld bytes that
+// starts at byte out_off: codes, fp16 scales, zero padding to a multiple of 16 bytes.
 __global__ void __launch_bounds__(256)
-quantize_rows_kernel(const __half* __restrict__ x, int rows, int dims, int fmt,
-                     uint8_t* __restrict__ out) {
+quantize_rows_kernel(const __half* __restrict__ x, int x_ld, int rows, int dims, int fmt,
+                     uint8_t* __restrict__ out, int out_ld, int out_off) {
     const int nb = dims / kQBlock;
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= (long long)rows * nb) return;
     const int r = (int)(gid / nb), b = (int)(gid % nb);
-    const __half* src = x + (size_t)r * dims + b * kQBlock;
+    const __half* src = x + (size_t)r * x_ld + b * kQBlock;
     const int rb = quant_row_bytes(fmt, dims), cb = quant_code_bytes(fmt, dims);
-    uint8_t* row = out + (size_t)r * rb;
+    uint8_t* row = out + (size_t)r * out_ld + out_off;
     float v[kQBlock];
 #pragma unroll
     for (int i = 0; i < kQBlock; ++i) v[i] = __half2float(src[i]);
@@ -50,7 +57,7 @@ quantize_rows_kernel(const __half* __restrict__ x, int rows, int dims, int fmt,
         float amax = 0.f;
 #pragma unroll
         for (int i = 0; i < kQBlock; ++i) amax = fmaxf(amax, fabsf(v[i]));
-        d16 = __float2half_rn(amax / 127.f);
+        d16 = __float2half_rn(amax / 127.f);               // >= +0
         const float d = __half2float(d16);
 #pragma unroll
         for (int i = 0; i < kQBlock; ++i) {
@@ -66,6 +73,7 @@ quantize_rows_kernel(const __half* __restrict__ x, int rows, int dims, int fmt,
                 m = v[i];
             }
         d16 = __float2half_rn(m / -8.f);
+        if (__half2float(d16) == 0.f) d16 = __float2half_rn(0.f);   // +0 for an all-zero block
         const float d = __half2float(d16);
         uint8_t n[kQBlock];
 #pragma unroll

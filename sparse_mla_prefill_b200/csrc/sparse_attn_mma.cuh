@@ -86,19 +86,41 @@ constexpr int FLAG_BYTES = 16;                // raised[2], abort, pad
 constexpr int G_BYTES = 2 * P_BYTES + X_BYTES + REF_BYTES + RED_BYTES + FLAG_BYTES;
 constexpr int G_P = 0, G_PLO = P_BYTES, G_X = 2 * P_BYTES, G_REF = G_X + X_BYTES,
               G_RED = G_REF + REF_BYTES, G_FLAGS = G_RED + RED_BYTES;
-constexpr int OFF_RING = 0;
-constexpr int OFF_GROUP = OFF_RING + NS * SLOT;
-constexpr int OFF_MASK = OFF_GROUP + GROUPS * G_BYTES;   // row-validity bits per slot
-constexpr int OFF_BAR = OFF_MASK + 32;                   // full[NS], empty[NS]
-constexpr int OFF_IDX = OFF_BAR + 2 * NS * 8;
 constexpr int MAX_TOPK = 2048;
-__host__ __device__ constexpr int smem_bytes(int k) {
-    return OFF_IDX + GROUPS * IDX_BUFS * ((k + 3) / 4 * 4) * 4;
-}
+constexpr int SMEM_LIMIT = 227 * 1024;
+constexpr int ROWV = DV * 2;                  // 1024 bytes: a separate value row
+
+// Shared-memory layout of the kernel for a cache format: NS ring slots of BR rows, each
+// row 1152 bytes (key = the row's 576 values; value = its first 512), or, for the
+// "Q8 K / Q4 V" format whose keys and values differ, a 1152-byte key row plus a
+// 1024-byte value row (the value rows of a slot follow its key rows); then the groups'
+// areas, the row-validity bits, the barriers and the staged top-k rows.
+template <int KVF>
+struct RingLayout {
+    static constexpr bool SPLIT = KVF == kFmtQ8Q4;
+    static constexpr int NS_ = SPLIT ? 3 : NS;
+    static constexpr int VOFF = BR * ROW;                   // value rows within a slot
+    static constexpr int SLOT_ = SPLIT ? BR * (ROW + ROWV) : SLOT;
+    static constexpr int OFF_RING = 0;
+    static constexpr int OFF_GROUP = OFF_RING + NS_ * SLOT_;
+    static constexpr int OFF_MASK = OFF_GROUP + GROUPS * G_BYTES;   // row-validity bits per slot
+    static constexpr int OFF_BAR = OFF_MASK + 32;                   // full[NS_], empty[NS_]
+    static constexpr int OFF_IDX = OFF_BAR + 2 * NS_ * 8;
+    __host__ __device__ static constexpr int smem_bytes(int k) {
+        return OFF_IDX + GROUPS * IDX_BUFS * ((k + 3) / 4 * 4) * 4;
+    }
+    // the largest top_k whose staged rows fit
+    static constexpr int MAX_K = (SMEM_LIMIT - OFF_IDX) / (GROUPS * IDX_BUFS * 4) / 4 * 4 < MAX_TOPK
+                                     ? (SMEM_LIMIT - OFF_IDX) / (GROUPS * IDX_BUFS * 4) / 4 * 4
+                                     : MAX_TOPK;
+    static_assert(NS_ <= 8, "row-validity bytes for at most 8 slots");
+    static_assert(G_BYTES % 16 == 0 && OFF_GROUP % 16 == 0, "16-byte aligned group areas");
+    static_assert(smem_bytes(MAX_K) <= SMEM_LIMIT, "shared memory budget");
+};
+__host__ __device__ constexpr int smem_bytes(int k) { return RingLayout<kFmtF16>::smem_bytes(k); }
 static_assert(DV == GWARPS * 128, "each group warp owns 128 value dims");
 static_assert(CH % 8 == 0 && BR * CH == PTHREADS * 18, "producer chunk split");
-static_assert(G_BYTES % 16 == 0 && OFF_GROUP % 16 == 0, "16-byte aligned group areas");
-static_assert(smem_bytes(MAX_TOPK) <= 227 * 1024, "shared memory budget");
+static_assert(RingLayout<kFmtF16>::MAX_K == MAX_TOPK, "fp16 ring holds top_k up to 2048");
 
 // 16-byte chunk swizzle: eight consecutive rows put one chunk in eight different bank
 // groups (ldmatrix), and rows 2m, 2m+1 put an aligned group of four chunks in
@@ -106,6 +128,10 @@ static_assert(smem_bytes(MAX_TOPK) <= 227 * 1024, "shared memory budget");
 __device__ __forceinline__ int swz(int row) { return ((row & 1) << 2) | ((row >> 1) & 3); }
 __device__ __forceinline__ uint32_t chunk_addr(uint32_t slot, int row, int chunk) {
     return slot + row * ROW + ((chunk ^ swz(row)) << 4);
+}
+// The same swizzle for rows of `pitch` bytes (a multiple of 128) from `base`.
+__device__ __forceinline__ uint32_t chunk_addr_p(uint32_t base, int row, int chunk, int pitch) {
+    return base + row * pitch + ((chunk ^ swz(row)) << 4);
 }
 
 }  // namespace attn
@@ -230,21 +256,21 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-// Producer side of a quantized cache: this lane's blocks of one row (lane l of the row's
-// four takes blocks l, l+4, l+8, ...), loaded as 16-byte words, dequantized to fp16 and
-// stored into the ring row as four 16-byte chunks per block; a masked row stores zeros.
-template <int KVF>
-__device__ __forceinline__ void dequant_row_to_ring(const uint8_t* rowq, bool ok, uint32_t dst,
-                                                    int r, int sub) {
-    using namespace attn;
-    constexpr int NB = DQK / kQBlock;                    // 18 blocks
-    constexpr int CB = quant_code_bytes(KVF, DQK);
-    constexpr int W = KVF == kFmtQ8 ? 2 : 1;             // 16-byte words per block
-    constexpr int BATCH = KVF == kFmtQ8 ? 2 : 3;         // blocks whose loads fly together
+// Producer side of a quantized cache: this lane's blocks of one stored row part (lane l
+// of the row's four takes blocks l, l+4, l+8, ...), loaded as 16-byte words, dequantized
+// to fp16 and stored as four 16-byte chunks per block into ring row r of `pitch` bytes
+// from `base`; a masked row stores zeros. FMT is Q8_0 or Q4_0 and NB the part's blocks.
+template <int FMT, int NB>
+__device__ __forceinline__ void dequant_part_to_ring(const uint8_t* rowq, bool ok, uint32_t base,
+                                                     int pitch, int r, int sub) {
+    using attn::chunk_addr_p;
+    constexpr int CB = quant_code_bytes(FMT, NB * kQBlock);
+    constexpr int W = FMT == kFmtQ8 ? 2 : 1;             // 16-byte words per block
+    constexpr int BATCH = FMT == kFmtQ8 ? 2 : 3;         // blocks whose loads fly together
     if (!ok) {
         for (int m = sub; m < NB; m += 4)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) st_shared_v4(chunk_addr(dst, r, 4 * m + k), make_uint4(0, 0, 0, 0));
+            for (int k = 0; k < 4; ++k) st_shared_v4(chunk_addr_p(base, r, 4 * m + k, pitch), make_uint4(0, 0, 0, 0));
         return;
     }
     for (int m0 = sub; m0 < NB; m0 += 4 * BATCH) {
@@ -264,22 +290,37 @@ __device__ __forceinline__ void dequant_row_to_ring(const uint8_t* rowq, bool ok
         for (int i = 0; i < BATCH; ++i) {
             const int m = m0 + 4 * i;
             if (m >= NB) continue;
-            if constexpr (KVF == kFmtQ8) {
-                st_shared_v4(chunk_addr(dst, r, 4 * m + 0), dequant_q8_chunk(c[i][0].x, c[i][0].y, d2[i]));
-                st_shared_v4(chunk_addr(dst, r, 4 * m + 1), dequant_q8_chunk(c[i][0].z, c[i][0].w, d2[i]));
-                st_shared_v4(chunk_addr(dst, r, 4 * m + 2), dequant_q8_chunk(c[i][1].x, c[i][1].y, d2[i]));
-                st_shared_v4(chunk_addr(dst, r, 4 * m + 3), dequant_q8_chunk(c[i][1].z, c[i][1].w, d2[i]));
+            if constexpr (FMT == kFmtQ8) {
+                st_shared_v4(chunk_addr_p(base, r, 4 * m + 0, pitch), dequant_q8_chunk(c[i][0].x, c[i][0].y, d2[i]));
+                st_shared_v4(chunk_addr_p(base, r, 4 * m + 1, pitch), dequant_q8_chunk(c[i][0].z, c[i][0].w, d2[i]));
+                st_shared_v4(chunk_addr_p(base, r, 4 * m + 2, pitch), dequant_q8_chunk(c[i][1].x, c[i][1].y, d2[i]));
+                st_shared_v4(chunk_addr_p(base, r, 4 * m + 3, pitch), dequant_q8_chunk(c[i][1].z, c[i][1].w, d2[i]));
             } else {
                 const uint4 w = c[i][0];
                 const uint32_t M = 0x0F0F0F0Fu;
-                st_shared_v4(chunk_addr(dst, r, 4 * m + 0), dequant_q4_chunk(w.x & M, w.y & M, d2[i]));
-                st_shared_v4(chunk_addr(dst, r, 4 * m + 1), dequant_q4_chunk(w.z & M, w.w & M, d2[i]));
-                st_shared_v4(chunk_addr(dst, r, 4 * m + 2),
+                st_shared_v4(chunk_addr_p(base, r, 4 * m + 0, pitch), dequant_q4_chunk(w.x & M, w.y & M, d2[i]));
+                st_shared_v4(chunk_addr_p(base, r, 4 * m + 1, pitch), dequant_q4_chunk(w.z & M, w.w & M, d2[i]));
+                st_shared_v4(chunk_addr_p(base, r, 4 * m + 2, pitch),
                              dequant_q4_chunk((w.x >> 4) & M, (w.y >> 4) & M, d2[i]));
-                st_shared_v4(chunk_addr(dst, r, 4 * m + 3),
+                st_shared_v4(chunk_addr_p(base, r, 4 * m + 3, pitch),
                              dequant_q4_chunk((w.z >> 4) & M, (w.w >> 4) & M, d2[i]));
             }
         }
+    }
+}
+
+// A stored row of the cache format into ring row r of the slot at `dst`.
+template <int KVF>
+__device__ __forceinline__ void dequant_row_to_ring(const uint8_t* rowq, bool ok, uint32_t dst,
+                                                    int r, int sub) {
+    using namespace attn;
+    constexpr int NB = DQK / kQBlock;                        // 18 key blocks
+    if constexpr (KVF == kFmtQ8Q4) {
+        dequant_part_to_ring<kFmtQ8, NB>(rowq, ok, dst, ROW, r, sub);
+        dequant_part_to_ring<kFmtQ4, DV / kQBlock>(rowq + quant_row_bytes(kFmtQ8, DQK), ok,
+                                                   dst + RingLayout<KVF>::VOFF, ROWV, r, sub);
+    } else {
+        dequant_part_to_ring<KVF, NB>(rowq, ok, dst, ROW, r, sub);
     }
 }
 
@@ -289,23 +330,24 @@ __device__ __forceinline__ void dequant_row_to_ring(const uint8_t* rowq, bool ok
 template <bool PRECISE, bool PSPLIT, int KVF>
 __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnParams p) {
     using namespace attn;
+    using L = RingLayout<KVF>;
     auto exp2_ = [](float x) { return PRECISE ? exp2f(x) : fast_exp2(x); };
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int kpad = (p.k + 3) / 4 * 4;
-    volatile uint32_t* rowmask = reinterpret_cast<volatile uint32_t*>(smem + OFF_MASK);
-    const uint32_t bar0 = sbase + OFF_BAR;
+    volatile uint32_t* rowmask = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MASK);
+    const uint32_t bar0 = sbase + L::OFF_BAR;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (L::NS_ + s); };
 
     if (tid == 0) {
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < L::NS_; ++s) {
             mbar_init(full_bar(s), PTHREADS + PWARPS);   // noinc copy arrivals + mask writers
             mbar_init(empty_bar(s), GWARPS);             // the owning group's warps
         }
         for (int g = 0; g < GROUPS; ++g) {
-            volatile int* f = reinterpret_cast<volatile int*>(smem + OFF_GROUP + g * G_BYTES + G_FLAGS);
+            volatile int* f = reinterpret_cast<volatile int*>(smem + L::OFF_GROUP + g * G_BYTES + G_FLAGS);
             f[0] = f[1] = f[2] = 0;
         }
         fence_mbar_init();
@@ -317,7 +359,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         // ================================================================ producers
         regs_decrease<PRODUCER_REGS>();
         const int ptid = tid - CTHREADS, pw = warp - CWARPS;
-        auto idx_buf = [&](int g, int m) { return OFF_IDX + (g * IDX_BUFS + (m & 1)) * kpad * 4; };
+        auto idx_buf = [&](int g, int m) { return L::OFF_IDX + (g * IDX_BUFS + (m & 1)) * kpad * 4; };
         auto stage_idx = [&](int g, int m) {      // top-k row of group g's m-th token
             const int idx = blockIdx.x + (g + GROUPS * m) * gridDim.x;
             if (idx >= p.n_items) return;
@@ -340,11 +382,11 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         // (its waits then return at once), so that it still meets every producer barrier
         // that the other producer warps reach.
         for (int uc = 0; mc.valid(); ++uc, mc.advance(p)) {
-            const int s = uc % NS;
+            const int s = uc % L::NS_;
             if (!abort &&
-                !__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ((uc / NS) & 1) ^ 1, p.wc, abort)))
+                !__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ((uc / L::NS_) & 1) ^ 1, p.wc, abort)))
                 abort = true;                      // the whole warp gives up together
-            const uint32_t dst = sbase + OFF_RING + s * SLOT;
+            const uint32_t dst = sbase + L::OFF_RING + s * L::SLOT_;
             const GroupCursor cu = mc.group(mc.turn);
             if (cu.u == 0) {
                 if (!abort) {
@@ -436,9 +478,9 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         regs_increase<CONSUMER_REGS>();
         const int grp = warp / GWARPS, gw = warp % GWARPS;
         const int gbar = GROUP_BAR + grp;
-        uint8_t* garea = smem + OFF_GROUP + grp * G_BYTES;
-        const uint32_t pbase = sbase + OFF_GROUP + grp * G_BYTES + G_P;
-        const uint32_t plobase = sbase + OFF_GROUP + grp * G_BYTES + G_PLO;
+        uint8_t* garea = smem + L::OFF_GROUP + grp * G_BYTES;
+        const uint32_t pbase = sbase + L::OFF_GROUP + grp * G_BYTES + G_P;
+        const uint32_t plobase = sbase + L::OFF_GROUP + grp * G_BYTES + G_PLO;
         float4* xbuf = reinterpret_cast<float4*>(garea + G_X);
         float* ref_tile = reinterpret_cast<float*>(garea + G_REF);
         float* red_sum = reinterpret_cast<float*>(garea + G_RED);
@@ -455,7 +497,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         float m_g = -INFINITY, m_g8 = -INFINITY; // reference max, heads g and g+8 (log2 units)
         float l_g = 0.f, l_g8 = 0.f;             // this warp's share of the softmax sums
         auto wait_full = [&](int q) {
-            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(q % NS), (q / NS) & 1, p.wc, abort)))
+            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(q % L::NS_), (q / L::NS_) & 1, p.wc, abort)))
                 flags[2] = 1;
         };
         MergedCursor mc;
@@ -464,7 +506,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         for (int q = 0; mc.valid(); ++q, mc.advance(p)) {
             if (mc.turn != grp) continue;         // the other group's unit
             const GroupCursor cu = mc.group(grp);
-            const uint32_t slot = sbase + OFF_RING + (q % NS) * SLOT;
+            const uint32_t slot = sbase + L::OFF_RING + (q % L::NS_) * L::SLOT_;
             wait_full(q);
             if (cu.u == 0) {
 #pragma unroll
@@ -476,7 +518,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                 m_g = m_g8 = -INFINITY;
                 l_g = l_g8 = 0.f;
                 __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(q % NS));
+                if (lane == 0) mbar_arrive(empty_bar(q % L::NS_));
                 continue;
             }
 
@@ -505,7 +547,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
 
             {
                 const float4 u = xbuf[own * 32 + lane];
-                const uint32_t mk = rowmask[q % NS];
+                const uint32_t mk = rowmask[q % L::NS_];
                 const bool v0 = (mk >> r0) & 1u, v1 = (mk >> (r0 + 1)) & 1u;
                 s4[0] = v0 ? (s4[0] + u.x) * p.scale_log2 : -INFINITY;
                 s4[1] = v1 ? (s4[1] + u.y) * p.scale_log2 : -INFINITY;
@@ -598,7 +640,10 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
 #pragma unroll
                 for (int np = 0; np < 8; ++np) {
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4_trans(chunk_addr(slot, vr, 16 * gw + 2 * np + hi), b0, b1, b2, b3);
+                    const int vch = 16 * gw + 2 * np + hi;
+                    const uint32_t vaddr = L::SPLIT ? chunk_addr_p(slot + L::VOFF, vr, vch, ROWV)
+                                                    : chunk_addr(slot, vr, vch);
+                    ldsm_x4_trans(vaddr, b0, b1, b2, b3);
                     if constexpr (PSPLIT) {
                         mma_16816(o[2 * np], al, b0, b1);
                         mma_16816(o[2 * np + 1], al, b2, b3);
@@ -608,7 +653,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(empty_bar(q % NS));
+            if (lane == 0) mbar_arrive(empty_bar(q % L::NS_));
 
             if (cu.u == cu.tr.nblk) {
                 // ---- last unit of the token: normalise and store

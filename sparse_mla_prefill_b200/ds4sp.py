@@ -160,7 +160,7 @@ def make_config(n_idx_heads: int, d_idx: int, top_k: int, n_swa: int, max_tokens
     softmax; pv_mode: 0 = fp16 probabilities in P . V, 1 = fp32-staged (hi + lo fp16);
     topk_mode: 0 = scores in the workspace and a separate top-k kernel, 1 = fused
     indexer + top-k where the call qualifies; kv_format: 0 = fp16 KV rows, 1 = Q8_0,
-    2 = Q4_0 quantized rows (ds4sp_quantize_kv)."""
+    2 = Q4_0, 3 = Q8 K / Q4 V quantized rows (ds4sp_quantize_kv)."""
     return ds4sp_config(n_heads, d_qk, d_v, ratio, n_idx_heads, d_idx, top_k, n_swa, band,
                         max_tokens, softmax_scale, exp_mode, pv_mode, topk_mode, kv_format)
 

@@ -478,6 +478,26 @@ def pin_quant_kv_split_composition(o, T: int = 48):
         assert np.abs(got["out"][t] - want).max() < 1e-12, t
 
 
+def pin_cache_rows_layout(o):
+    """The stored row of each cache format read back part by part (unpack_rows at the
+    part's byte offset, dequantize_rows) gives the key and value rows kv_values uses, and
+    its length is quant_row_bytes."""
+    rng = np.random.default_rng(15)
+    x = (rng.standard_normal((5, 576)) * 2).astype(np.float16)
+    for fmt in (o.Q8_0, o.Q4_0, o.Q8K_Q4V):
+        packed = o.cache_rows(x, fmt)
+        assert packed.shape == (5, o.quant_row_bytes(fmt, 576)), fmt
+        k, v = o.kv_values(x, fmt)
+        if fmt == o.Q8K_Q4V:
+            kb = o.quant_row_bytes(o.Q8_0, 576)
+            k2 = o.dequantize_rows(*o.unpack_rows(packed[:, :kb], o.Q8_0, 576), o.Q8_0)
+            v2 = o.dequantize_rows(*o.unpack_rows(packed[:, kb:], o.Q4_0, 512), o.Q4_0)
+        else:
+            k2 = o.dequantize_rows(*o.unpack_rows(packed, fmt, 576), fmt)
+            v2 = k2[:, :512]
+        assert np.array_equal(k, k2) and np.array_equal(v, v2), fmt
+
+
 ALL_PINS = [
     pin_visibility_mask, pin_visibility_golden,
     pin_scores_exact, pin_scores_relu_identities, pin_scores_bruteforce,
@@ -487,6 +507,7 @@ ALL_PINS = [
     pin_bands_equal_oneshot, pin_prefill_tokens_composition,
     pin_quant_golden, pin_quant_dequant_bruteforce, pin_quant_properties,
     pin_quant_path_reduces_to_fp16, pin_attention_kv_sdpa, pin_quant_kv_split_composition,
+    pin_cache_rows_layout,
 ]
 
 

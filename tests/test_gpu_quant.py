@@ -1,4 +1,4 @@
-"""Quantized KV cache (kv_format 1 = Q8_0, 2 = Q4_0) through the C ABI.
+"""Quantized KV cache (kv_format 1 = Q8_0, 2 = Q4_0, 3 = Q8 K / Q4 V) through the C ABI.
 
 ds4sp_quantize_kv must write the oracle's bytes exactly: codes are decided in fp32 on
 both sides (IEEE division, half-to-even rounding, the first extreme of Q4_0), and the
@@ -41,13 +41,13 @@ def _special_rows():
     return r.astype(np.float16)
 
 
-@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("fmt", [1, 2, 3])
 @pytest.mark.parametrize("dims", [576, 512])
 def test_quantize_bytes_match_oracle(fmt, dims):
     x = np.concatenate([_special_rows()[:, :dims],
                         generate(workload("band"))["kv_raw"].numpy()[:300, :dims]])
     got = D.ds4sp_quantize_kv(torch.from_numpy(x).cuda(), fmt).cpu().numpy()
-    want = oracle.pack_rows(*oracle.quantize_rows(x, fmt), fmt)
+    want = oracle.cache_rows(x, fmt)
     assert got.shape == want.shape == (x.shape[0], oracle.quant_row_bytes(fmt, dims))
     if not np.array_equal(got, want):
         bad = np.argwhere(got != want)
@@ -61,7 +61,7 @@ def _quantized(dev, fmt):
     return q
 
 
-@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("fmt", [1, 2, 3])
 @pytest.mark.parametrize("name", ["tiny", "band"])
 def test_quantized_cache_parity(name, fmt):
     wl = workload(name)
@@ -115,8 +115,26 @@ def test_quantized_cache_host_path_equals_device_path():
     assert torch.equal(out_h, out_d.cpu())
 
 
-def test_quantized_format_needs_default_modes():
+def test_quantized_cache_10k_sampled_split_format():
+    """Q8 K / Q4 V on the 10K prefill (its 3-slot ring): sampled tokens against the oracle."""
+    wl = workload("10k")
+    inp = generate(wl)
+    dev = _quantized(to_device(inp), 3)
+    with handle_for(wl, kv_format=3) as h:
+        topk, out = run_prefill(h, dev, wl.T, wl.top_k)
+    toks = sample_tokens(wl.T, wl.band, 16, seed=33)
+    npi = {k: v.numpy() for k, v in inp.items()}
+    ref = oracle.prefill_tokens_quant(npi, toks, wl.top_k, wl.n_swa, 3)
+    assert np.array_equal(topk.cpu().numpy()[toks], ref["topk"])
+    assert_attention_close(out.cpu().numpy()[toks], ref["out"], "10k Q8 K / Q4 V")
+
+
+def test_quantized_format_limits():
     wl = workload("tiny")
     with pytest.raises(D.Ds4spError) as e:
         handle_for(wl, kv_format=1, pv_mode=1)
     assert e.value.status == D.ERR_UNSUPPORTED
+    with pytest.raises(D.Ds4spError) as e:
+        handle_for(workload("tiny", top_k=1000), kv_format=3)
+    assert e.value.status == D.ERR_UNSUPPORTED
+    assert D.ds4sp_kv_row_bytes(3, 576) == 912 and D.ds4sp_kv_row_bytes(3, 256) == 0
