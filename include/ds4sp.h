@@ -110,6 +110,13 @@ typedef struct {
                             prefill scheduling to 10K", Production workflow and the
                             clean-head validation; the pages name the formats without
                             defining them) */
+    int dependent_launch; /* 1 = launch each kernel as a programmatic dependent of the
+                            kernel before it on the stream: its launch and prologue
+                            (barrier set-up, tensor-memory allocation) overlap that
+                            kernel's last wave, and it touches global memory only once
+                            that kernel has completed, so results are the same bits.
+                            0 = plain stream order. Other values are
+                            DS4SP_ERR_INVALID_ARG */
 } ds4sp_config;
 
 /* Validate cfg and create a handle bound to the current CUDA device. The handle owns

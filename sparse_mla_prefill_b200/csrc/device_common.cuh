@@ -122,6 +122,22 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, c
     return false;
 }
 
+// ---------------------------------------------------------------- dependent launch
+
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization may start while the kernel before it on the stream is finishing; it must
+// not touch global memory that kernel (or any earlier work) writes or reads until
+// grid_dependency_wait() returns, which happens once that kernel has completed and its
+// memory operations are visible. After the wait, grid_dependents_launch() lets the next
+// kernel of the stream start its own prologue. Without the launch attribute both are
+// no-ops, and the kernels run in plain stream order.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- cp.async
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, bool valid) {

@@ -14,6 +14,7 @@
 #include <mutex>
 #include <new>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "ds4sp.h"
@@ -187,6 +188,26 @@ ds4sp_status launch(ds4sp_handle* h, int kind, cudaStream_t stream, F&& f) {
     return DS4SP_OK;
 }
 
+// A kernel launch on `stream`, as a programmatic dependent of the previous kernel when
+// `dependent` is set (the kernels wait for that kernel before touching global memory,
+// so only their launch and prologue overlap its tail). Launch errors are also left for
+// cudaGetLastError.
+template <class... KArgs, class... Args>
+void launch_k(bool dependent, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+              cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = dependent ? 1 : 0;
+    cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------- TMA descriptors
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -300,7 +321,8 @@ ds4sp_status launch_indexer(ds4sp_handle* h, const void* q_idx, const void* k_id
         if (b != grid - 1) return fail(DS4SP_ERR_CUDA, "indexer partition: %d of %d shares", b + 1, grid);
     }
     return launch(h, kIndexer, stream, [&] {
-        indexer_tcgen05_kernel<D_I, H_I><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tq, p);
+        launch_k(h->cfg.dependent_launch != 0, indexer_tcgen05_kernel<D_I, H_I>, grid, C::THREADS,
+                 C::SMEM_BYTES, stream, tk, tq, p);
     });
 }
 
@@ -387,7 +409,8 @@ ds4sp_status launch_fused(ds4sp_handle* h, const void* q_idx, const void* k_idx,
     }
     p.first[grid] = (uint16_t)u;
     return launch(h, kIndexer, stream, [&] {
-        indexer_topk_fused_kernel<D_I, H_I><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tq, p);
+        launch_k(h->cfg.dependent_launch != 0, indexer_topk_fused_kernel<D_I, H_I>, grid, C::THREADS,
+                 C::SMEM_BYTES, stream, tk, tq, p);
     });
 }
 
@@ -424,13 +447,14 @@ ds4sp_status launch_topk(ds4sp_handle* h, const float* scores, int ld, int t0, i
         h->smem_set[kTopk] = true;
     }
     const size_t smem = (size_t)ld * 4;
+    const bool pdl = h->cfg.dependent_launch != 0;
     return launch(h, kTopk, stream, [&] {
         if (big)
-            topk_radix_kernel<1024><<<n_q, 1024, smem, stream>>>(scores, ld, t0, n_q, k, ratio,
-                                                                 vm, mld, mcols, topk);
+            launch_k(pdl, topk_radix_kernel<1024>, n_q, 1024, smem, stream, scores, ld, t0, n_q, k,
+                     ratio, vm, mld, mcols, topk);
         else
-            topk_radix_kernel<256><<<n_q, 256, smem, stream>>>(scores, ld, t0, n_q, k, ratio,
-                                                               vm, mld, mcols, topk);
+            launch_k(pdl, topk_radix_kernel<256>, n_q, 256, smem, stream, scores, ld, t0, n_q, k,
+                     ratio, vm, mld, mcols, topk);
     });
 }
 
@@ -522,21 +546,22 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
         // persistent: one CTA per SM, each walking its share of the work items
         const int grid = std::min(p.n_items, h->sm_count);
         const dim3 g(grid), b(attn::THREADS);
+        const bool pdl = h->cfg.dependent_launch != 0;
         if (h->cfg.kv_format == kFmtQ8) {
-            sparse_attn_mma_kernel<false, false, kFmtQ8><<<g, b, smem, stream>>>(p);
+            launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ8>, g, b, smem, stream, p);
         } else if (h->cfg.kv_format == kFmtQ4) {
-            sparse_attn_mma_kernel<false, false, kFmtQ4><<<g, b, smem, stream>>>(p);
+            launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ4>, g, b, smem, stream, p);
         } else if (h->cfg.kv_format == kFmtQ8Q4) {
-            sparse_attn_mma_kernel<false, false, kFmtQ8Q4><<<g, b, smem, stream>>>(p);
+            launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ8Q4>, g, b, smem, stream, p);
         } else {
             switch (2 * h->cfg.pv_mode + h->cfg.exp_mode) {
-                case 0: sparse_attn_mma_kernel<false, false, kFmtF16><<<g, b, smem, stream>>>(p); break;
-                case 1: sparse_attn_mma_kernel<true, false, kFmtF16><<<g, b, smem, stream>>>(p); break;
-                case 2: sparse_attn_mma_kernel<false, true, kFmtF16><<<g, b, smem, stream>>>(p); break;
-                default: sparse_attn_mma_kernel<true, true, kFmtF16><<<g, b, smem, stream>>>(p); break;
+                case 0: launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtF16>, g, b, smem, stream, p); break;
+                case 1: launch_k(pdl, sparse_attn_mma_kernel<true, false, kFmtF16>, g, b, smem, stream, p); break;
+                case 2: launch_k(pdl, sparse_attn_mma_kernel<false, true, kFmtF16>, g, b, smem, stream, p); break;
+                default: launch_k(pdl, sparse_attn_mma_kernel<true, true, kFmtF16>, g, b, smem, stream, p); break;
             }
         }
-        if (p.split) attn_merge_kernel<<<n_q * attn::H, 128, 0, stream>>>(mp);
+        if (p.split) launch_k(pdl, attn_merge_kernel, n_q * attn::H, 128, 0, stream, mp);
     });
 }
 
@@ -670,6 +695,8 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
         return fail(DS4SP_ERR_INVALID_ARG, "pv_mode %d (0 = fp16 P, 1 = fp32-staged P)", c.pv_mode);
     if (c.topk_mode != 0 && c.topk_mode != 1)
         return fail(DS4SP_ERR_INVALID_ARG, "topk_mode %d (0 = separate top-k, 1 = fused)", c.topk_mode);
+    if (c.dependent_launch != 0 && c.dependent_launch != 1)
+        return fail(DS4SP_ERR_INVALID_ARG, "dependent_launch %d (0 or 1)", c.dependent_launch);
     if (c.kv_format < 0 || c.kv_format > 3)
         return fail(DS4SP_ERR_INVALID_ARG, "kv_format %d (0 = fp16, 1 = Q8_0, 2 = Q4_0, 3 = Q8 K / Q4 V)",
                     c.kv_format);

@@ -232,6 +232,10 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_ptr;
+    // The prologue above (barriers, TMEM, descriptors) may overlap the previous kernel;
+    // inputs are read and outputs written only after it has completed.
+    grid_dependency_wait();
+    grid_dependents_launch();
     // This CTA's share, as the host cut it.
     const IndexerWalk walk0{p.start_tb[b], p.start_jt[b], p.count[b]};
 
@@ -365,15 +369,6 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 tc_fence_after();
                 const int j = w.jt(it) * C::BM + quarter * 32 + lane;
                 const int t_first = w.tok0 + half * (128 / H_I);
-                // Rows of the tile past the last visible row of every token of this warp:
-                // nothing to compute or store; release the accumulator unread.
-                const int t_warp_last = min(t_first + 128 / H_I, w.tok_end) - 1;
-                if (p.ratio * (w.jt(it) * C::BM + quarter * 32 + 1) > t_warp_last + 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(tempty(buf));
-                    continue;
-                }
                 epilogue_tile<H_I>(
                     lane_addr + buf * C::BN, wh,
                     [&] {

@@ -200,6 +200,10 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_ptr;
+    // The prologue above (barriers, TMEM, descriptors) may overlap the previous kernel;
+    // inputs are read and outputs written only after it has completed.
+    grid_dependency_wait();
+    grid_dependents_launch();
 
     bool abort = false;
     if (warp == C::B_WARP || warp == 0) {
@@ -312,14 +316,6 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 tc_fence_after();
                 const int j = it * C::BM + quarter * 32 + lane;
                 const int tl_first = half * (128 / H_I);
-                // rows past the last visible row of every token of this warp: skip
-                const int t_warp_last = min(tok0 + tl_first + 128 / H_I, tok_end) - 1;
-                if (p.ratio * (it * C::BM + quarter * 32 + 1) > t_warp_last + 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(tempty(buf));
-                    continue;
-                }
                 epilogue_tile<H_I>(
                     lane_addr + buf * C::BN, wh,
                     [&] {

@@ -353,6 +353,10 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         fence_mbar_init();
     }
     __syncthreads();
+    // Global memory only after the previous kernel of the stream has completed (the
+    // prologue above may overlap it when launched as a programmatic dependent).
+    grid_dependency_wait();
+    grid_dependents_launch();
 
     bool abort = false;
     if (warp >= CWARPS) {
@@ -731,6 +735,8 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const MergeParams mp) {
     __shared__ float wgt[SPLIT_MAX_UNITS];      // per unit: 2^(m - M) / L for this head
     __shared__ float red[2][4];
     const int i = blockIdx.x / H, h = blockIdx.x % H;
+    grid_dependency_wait();                      // the partial results are complete
+    grid_dependents_launch();
     if (i >= mp.n_q) return;
     const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
     const int first = mp.first[i], cnt = min(mp.first[i + 1] - first, SPLIT_MAX_UNITS);

@@ -189,6 +189,8 @@ topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int
 
     const int i = blockIdx.x;
     const int t = t0 + i;
+    grid_dependency_wait();                      // the scores are complete
+    grid_dependents_launch();
     int32_t* out = topk + (size_t)i * k;
     const int tid = threadIdx.x;
     const float* row = scores + (size_t)i * ld;

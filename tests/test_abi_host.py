@@ -58,6 +58,11 @@ def _cfg(**kw):
     (dict(exp_mode=2), D.ERR_INVALID_ARG),
     (dict(pv_mode=2), D.ERR_INVALID_ARG),
     (dict(pv_mode=-1), D.ERR_INVALID_ARG),
+    (dict(topk_mode=2), D.ERR_INVALID_ARG),
+    (dict(kv_format=4), D.ERR_INVALID_ARG),
+    (dict(kv_format=1, exp_mode=1), D.ERR_UNSUPPORTED),
+    (dict(kv_format=3, top_k=900), D.ERR_UNSUPPORTED),
+    (dict(dependent_launch=2), D.ERR_INVALID_ARG),
 ])
 def test_create_rejects_bad_config_before_touching_the_device(lib, kw, status):
     out = ctypes.c_void_p(123)
