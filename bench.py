@@ -361,8 +361,15 @@ def run_ours(args, rank, world, local_rank):
     host = generate(wl)
     inputs = {k: v.to(dev) for k, v in host.items()}
     cfg = D.make_config(n_idx_heads=wl.H_i, d_idx=wl.D_i, top_k=wl.top_k, n_swa=wl.n_swa,
-                        max_tokens=wl.T, band=wl.band)
+                        max_tokens=wl.T, band=wl.band, topk_mode=args.topk_mode,
+                        kv_format=args.kv_format)
     h = D.ds4sp_create(cfg)
+    if args.kv_format:
+        # a quantized cache of the same rows, made on the device before any timing
+        for kv in ("kv_raw", "kv_cmp"):
+            inputs[kv] = D.ds4sp_quantize_kv(inputs[kv], args.kv_format)
+    # the tensors the end-to-end pass copies in (the quantized cache, if any)
+    host_io = dict(host, kv_raw=inputs["kv_raw"].cpu(), kv_cmp=inputs["kv_cmp"].cpu())
     topk = torch.empty((wl.T, wl.top_k), dtype=torch.int32, device=dev)
     out = torch.empty((wl.T, 16, 512), dtype=torch.float32, device=dev)
     ws = D.band_workspace(h, wl.T, dev)
@@ -418,7 +425,7 @@ def run_ours(args, rank, world, local_rank):
     ms_prof_max = max_over_ranks(ms_prof, world, dev)
 
     # end to end through the public API: pinned host inputs -> device, prefill, out -> host
-    pinned = {k: v.pin_memory() for k, v in host.items()}
+    pinned = {k: v.pin_memory() for k, v in host_io.items()}
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
     d2h = out.numel() * out.element_size()
@@ -511,7 +518,7 @@ def run_ours(args, rank, world, local_rank):
         l2 = gather_ceiling(dev, stream)
 
     cpu_base = parity = None
-    if solo and not args.no_cpu_baseline:
+    if solo and not args.no_cpu_baseline and not args.kv_format:
         cpu_base, ref = cpu_oracle_sample(wl, args.cpu_sample,
                                           {k: v.numpy() for k, v in host.items()},
                                           return_result=True)
@@ -605,6 +612,12 @@ def main():
                     help="skip the band and 8K prefill lines (and the 8K parity check)")
     ap.add_argument("--soak", type=float, default=1.5,
                     help="seconds of extra steps under the clock sampler")
+    ap.add_argument("--topk-mode", type=int, default=0, choices=[0, 1],
+                    help="the headline step's top-k form (1 = fused indexer + top-k; for "
+                         "profiling that kernel; the default line uses 0)")
+    ap.add_argument("--kv-format", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="the headline step's cache format (1 = Q8_0, 2 = Q4_0, 3 = Q8 K / "
+                         "Q4 V; for profiling; the default line uses fp16 rows)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
