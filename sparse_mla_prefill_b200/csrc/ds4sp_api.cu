@@ -22,6 +22,7 @@
 #include "indexer_topk_fused.cuh"
 #include "probe_gather.cuh"
 #include "sparse_attn_mma.cuh"
+#include "sparse_attn_tc.cuh"
 #include "topk_radix.cuh"
 
 using namespace ds4sp;
@@ -462,8 +463,10 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
                          const int32_t* topk, int t0, int n_q, float* out, cudaStream_t stream,
                          const void* prefetch = nullptr, size_t prefetch_bytes = 0) {
     const int kvf = h->cfg.kv_format;
-    const int smem = kvf == kFmtQ8Q4 ? attn::RingLayout<kFmtQ8Q4>::smem_bytes(h->cfg.top_k)
-                                     : attn::smem_bytes(h->cfg.top_k);
+    const bool tc = h->cfg.attn_kernel == 1;
+    const int smem = tc ? tcattn::smem_bytes(h->cfg.top_k)
+                        : kvf == kFmtQ8Q4 ? attn::RingLayout<kFmtQ8Q4>::smem_bytes(h->cfg.top_k)
+                                          : attn::smem_bytes(h->cfg.top_k);
     if (!h->smem_set[kAttn]) {
         // Every instantiation (fast or precise exponentials x fp16 or fp32-staged P, and
         // the two quantized-cache forms), once per handle.
@@ -489,6 +492,10 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
                 return fail(DS4SP_ERR_UNSUPPORTED, "attention kernel built with %d registers, not %d",
                             fa.numRegs, attn::LAUNCH_REGS);
         }
+        const cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   tcattn::smem_bytes(attn::MAX_TOPK));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention, tcgen05)");
         h->smem_set[kAttn] = true;
     }
     AttnParams p;
@@ -515,7 +522,7 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
     MergeParams mp{};
     p.split = 0;
     p.n_items = n_q;
-    if (n_q <= attn::SPLIT_MAX_TOKENS && h->split_cap > 0) {
+    if (!tc && n_q <= attn::SPLIT_MAX_TOKENS && h->split_cap > 0) {
         int items = 0;
         bool fits = true;
         for (int i = 0; i < n_q; ++i) {
@@ -547,7 +554,9 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
         const int grid = std::min(p.n_items, h->sm_count);
         const dim3 g(grid), b(attn::THREADS);
         const bool pdl = h->cfg.dependent_launch != 0;
-        if (h->cfg.kv_format == kFmtQ8) {
+        if (tc) {
+            launch_k(pdl, sparse_attn_tc_kernel, g, dim3(tcattn::THREADS), smem, stream, p);
+        } else if (h->cfg.kv_format == kFmtQ8) {
             launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ8>, g, b, smem, stream, p);
         } else if (h->cfg.kv_format == kFmtQ4) {
             launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ4>, g, b, smem, stream, p);
@@ -695,6 +704,11 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
         return fail(DS4SP_ERR_INVALID_ARG, "pv_mode %d (0 = fp16 P, 1 = fp32-staged P)", c.pv_mode);
     if (c.topk_mode != 0 && c.topk_mode != 1)
         return fail(DS4SP_ERR_INVALID_ARG, "topk_mode %d (0 = separate top-k, 1 = fused)", c.topk_mode);
+    if (c.attn_kernel != 0 && c.attn_kernel != 1)
+        return fail(DS4SP_ERR_INVALID_ARG, "attn_kernel %d (0 = mma.sync streaming, 1 = tcgen05 logits)",
+                    c.attn_kernel);
+    if (c.attn_kernel == 1 && (c.kv_format != 0 || c.exp_mode != 0 || c.pv_mode != 0))
+        return fail(DS4SP_ERR_UNSUPPORTED, "attn_kernel 1 runs fp16 rows with exp_mode 0 and pv_mode 0");
     if (c.dependent_launch != 0 && c.dependent_launch != 1)
         return fail(DS4SP_ERR_INVALID_ARG, "dependent_launch %d (0 or 1)", c.dependent_launch);
     if (c.kv_format < 0 || c.kv_format > 3)
