@@ -362,7 +362,7 @@ def run_ours(args, rank, world, local_rank):
     inputs = {k: v.to(dev) for k, v in host.items()}
     cfg = D.make_config(n_idx_heads=wl.H_i, d_idx=wl.D_i, top_k=wl.top_k, n_swa=wl.n_swa,
                         max_tokens=wl.T, band=wl.band, topk_mode=args.topk_mode,
-                        kv_format=args.kv_format)
+                        kv_format=args.kv_format, attn_kernel=args.attn_kernel)
     h = D.ds4sp_create(cfg)
     if args.kv_format:
         # a quantized cache of the same rows, made on the device before any timing
@@ -562,8 +562,10 @@ def run_ours(args, rank, world, local_rank):
                             "TFLOPs": idx_achieved,
                             "frac_tensor": idx_achieved / pk["bf16_tflops"],
                             "alg_flops_per_step": alg["indexer_flops"]},
+                # (with the fused top-k the select runs inside the indexer's launches)
                 "topk": {"ms_per_step": topk_ms / steps, "launches": topk_n,
-                         "alg_GBps": alg["topk_bytes"] * steps / (topk_ms / 1e3) / 1e9},
+                         "alg_GBps": (alg["topk_bytes"] * steps / (topk_ms / 1e3) / 1e9
+                                      if topk_ms > 0 else None)},
             },
             "gpu_launches": attn_n + idx_n + topk_n,
             "kernel_timing": {"steps": steps, "ms_per_step": ms_prof_max / steps,
@@ -616,6 +618,9 @@ def main():
     ap.add_argument("--topk-mode", type=int, default=0, choices=[0, 1],
                     help="the headline step's top-k form (1 = fused indexer + top-k; for "
                          "profiling that kernel; the default line uses 0)")
+    ap.add_argument("--attn-kernel", type=int, default=0, choices=[0, 1],
+                    help="the headline step's attention kernel (1 = logits on tcgen05; for "
+                         "profiling; the default line uses 0)")
     ap.add_argument("--kv-format", type=int, default=0, choices=[0, 1, 2, 3],
                     help="the headline step's cache format (1 = Q8_0, 2 = Q4_0, 3 = Q8 K / "
                          "Q4 V; for profiling; the default line uses fp16 rows)")
