@@ -104,8 +104,8 @@ typedef struct {
                             dequantizes the rows it gathers (value d*q or d*(n-8), rounded
                             once to fp16) and otherwise computes as for fp16 rows; the
                             indexer keys (k_idx) stay fp16. Quantized formats need
-                            exp_mode 0 and pv_mode 0, and format 3 top_k <= 824 (else
-                            DS4SP_ERR_UNSUPPORTED); other values are DS4SP_ERR_INVALID_ARG
+                            exp_mode 0 and pv_mode 0, and top_k <= 1012 (format 2) or
+                            824 (format 3) (else DS4SP_ERR_UNSUPPORTED); other values are DS4SP_ERR_INVALID_ARG
                             ("Q4_0 K/V cache" and "Q8 K / Q4 V", "perf(ds4): extend sparse
                             prefill scheduling to 10K", Production workflow and the
                             clean-head validation; the pages name the formats without

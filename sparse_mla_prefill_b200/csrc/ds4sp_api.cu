@@ -138,6 +138,25 @@ int score_ld(int t_last, int ratio) {
     return ((nv > 0 ? nv : 1) + 3) / 4 * 4;
 }
 
+// Shared memory of the streaming attention kernel for a cache format and top_k, and the
+// largest top_k that format's layout holds.
+int attn_smem_bytes(int kvf, int k) {
+    switch (kvf) {
+        case kFmtQ8: return attn::RingLayout<kFmtQ8>::smem_bytes(k);
+        case kFmtQ4: return attn::RingLayout<kFmtQ4>::smem_bytes(k);
+        case kFmtQ8Q4: return attn::RingLayout<kFmtQ8Q4>::smem_bytes(k);
+        default: return attn::RingLayout<kFmtF16>::smem_bytes(k);
+    }
+}
+int attn_max_topk(int kvf) {
+    switch (kvf) {
+        case kFmtQ8: return attn::RingLayout<kFmtQ8>::MAX_K;
+        case kFmtQ4: return attn::RingLayout<kFmtQ4>::MAX_K;
+        case kFmtQ8Q4: return attn::RingLayout<kFmtQ8Q4>::MAX_K;
+        default: return attn::RingLayout<kFmtF16>::MAX_K;
+    }
+}
+
 // Bytes of one row of kv_raw / kv_cmp in the handle's cache format.
 int kv_row_bytes_of(const ds4sp_config& c) {
     return c.kv_format == 0 ? c.d_qk * 2 : quant_row_bytes(c.kv_format, c.d_qk);
@@ -464,9 +483,7 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
                          const void* prefetch = nullptr, size_t prefetch_bytes = 0) {
     const int kvf = h->cfg.kv_format;
     const bool tc = h->cfg.attn_kernel == 1;
-    const int smem = tc ? tcattn::smem_bytes(h->cfg.top_k)
-                        : kvf == kFmtQ8Q4 ? attn::RingLayout<kFmtQ8Q4>::smem_bytes(h->cfg.top_k)
-                                          : attn::smem_bytes(h->cfg.top_k);
+    const int smem = tc ? tcattn::smem_bytes(h->cfg.top_k) : attn_smem_bytes(kvf, h->cfg.top_k);
     if (!h->smem_set[kAttn]) {
         // Every instantiation (fast or precise exponentials x fp16 or fp32-staged P, and
         // the two quantized-cache forms), once per handle.
@@ -478,10 +495,10 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
             reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtQ8>),
             reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtQ4>),
             reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtQ8Q4>)};
-        for (const void* fn : fns) {
-            const int max_smem = fn == fns[6] ? attn::RingLayout<kFmtQ8Q4>::smem_bytes(
-                                                    attn::RingLayout<kFmtQ8Q4>::MAX_K)
-                                              : attn::smem_bytes(attn::MAX_TOPK);
+        const int fmt_of[7] = {kFmtF16, kFmtF16, kFmtF16, kFmtF16, kFmtQ8, kFmtQ4, kFmtQ8Q4};
+        for (int fi = 0; fi < 7; ++fi) {
+            const void* fn = fns[fi];
+            const int max_smem = attn_smem_bytes(fmt_of[fi], attn_max_topk(fmt_of[fi]));
             const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                        max_smem);
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention)");
@@ -714,9 +731,9 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
     if (c.kv_format < 0 || c.kv_format > 3)
         return fail(DS4SP_ERR_INVALID_ARG, "kv_format %d (0 = fp16, 1 = Q8_0, 2 = Q4_0, 3 = Q8 K / Q4 V)",
                     c.kv_format);
-    if (c.kv_format == kFmtQ8Q4 && c.top_k > attn::RingLayout<kFmtQ8Q4>::MAX_K)
-        return fail(DS4SP_ERR_UNSUPPORTED, "kv_format 3 supports top_k up to %d",
-                    attn::RingLayout<kFmtQ8Q4>::MAX_K);
+    if (c.kv_format >= 1 && c.kv_format <= 3 && c.top_k > attn_max_topk(c.kv_format))
+        return fail(DS4SP_ERR_UNSUPPORTED, "kv_format %d supports top_k up to %d", c.kv_format,
+                    attn_max_topk(c.kv_format));
     if (c.kv_format != 0 && (c.exp_mode != 0 || c.pv_mode != 0))
         return fail(DS4SP_ERR_UNSUPPORTED, "a quantized cache runs with exp_mode 0 and pv_mode 0");
     ds4sp_handle* h = new (std::nothrow) ds4sp_handle();

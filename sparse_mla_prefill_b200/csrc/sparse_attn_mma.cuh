@@ -98,14 +98,20 @@ constexpr int ROWV = DV * 2;                  // 1024 bytes: a separate value ro
 template <int KVF>
 struct RingLayout {
     static constexpr bool SPLIT = KVF == kFmtQ8Q4;
-    static constexpr int NS_ = SPLIT ? 3 : NS;
+    // Q8_0 and Q4_0 rows are staged: the producers copy a unit's quantized rows into one
+    // of two staging buffers a unit ahead and dequantize from there into the ring.
+    static constexpr bool STAGED = KVF == kFmtQ8 || KVF == kFmtQ4;
+    static constexpr int NS_ = SPLIT ? 3 : KVF == kFmtQ8 ? 4 : NS;
     static constexpr int VOFF = BR * ROW;                   // value rows within a slot
     static constexpr int SLOT_ = SPLIT ? BR * (ROW + ROWV) : SLOT;
+    static constexpr int QROW = STAGED ? quant_row_bytes(KVF, DQK) : 0;   // a stored row
+    static constexpr int STAGE = BR * QROW;                 // one staging buffer
     static constexpr int OFF_RING = 0;
     static constexpr int OFF_GROUP = OFF_RING + NS_ * SLOT_;
     static constexpr int OFF_MASK = OFF_GROUP + GROUPS * G_BYTES;   // row-validity bits per slot
     static constexpr int OFF_BAR = OFF_MASK + 32;                   // full[NS_], empty[NS_]
-    static constexpr int OFF_IDX = OFF_BAR + 2 * NS_ * 8;
+    static constexpr int OFF_STAGE = OFF_BAR + 2 * NS_ * 8;
+    static constexpr int OFF_IDX = OFF_STAGE + 2 * STAGE;
     __host__ __device__ static constexpr int smem_bytes(int k) {
         return OFF_IDX + GROUPS * IDX_BUFS * ((k + 3) / 4 * 4) * 4;
     }
@@ -309,6 +315,66 @@ __device__ __forceinline__ void dequant_part_to_ring(const uint8_t* rowq, bool o
     }
 }
 
+// Staged quantized rows (Q8_0, Q4_0). Lane `sub` of a row's four copies the code bytes of
+// blocks sub, sub+4, ... and, for sub < 3, one 16-byte piece of the scales, to the same
+// byte offsets of a staging row; it later dequantizes the same blocks (its own copies,
+// plus the scales its row's lanes copied, once the warp has synchronised).
+template <int FMT>
+__device__ __forceinline__ void stage_row_copy(const uint8_t* rowq, uint32_t srow, int sub) {
+    constexpr int NB = attn::DQK / kQBlock;
+    constexpr int CB = quant_code_bytes(FMT, attn::DQK);
+    constexpr int W = FMT == kFmtQ8 ? 2 : 1;
+    for (int m = sub; m < NB; m += 4)
+#pragma unroll
+        for (int h = 0; h < W; ++h) cp_async_16(srow + (m * W + h) * 16, rowq + (m * W + h) * 16, true);
+    if (sub < 3) cp_async_16(srow + CB + 16 * sub, rowq + CB + 16 * sub, true);
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+
+template <int FMT>
+__device__ __forceinline__ void dequant_staged_to_ring(uint32_t srow, bool ok, uint32_t dst, int r,
+                                                       int sub) {
+    using attn::chunk_addr;
+    constexpr int NB = attn::DQK / kQBlock;
+    constexpr int CB = quant_code_bytes(FMT, attn::DQK);
+    for (int m = sub; m < NB; m += 4) {
+        if (!ok) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) st_shared_v4(chunk_addr(dst, r, 4 * m + k), make_uint4(0, 0, 0, 0));
+            continue;
+        }
+        const unsigned short dbits = (unsigned short)ld_shared_u16(srow + CB + 2 * m);
+        const __half2 d2 = __half2half2(__ushort_as_half(dbits));
+        if constexpr (FMT == kFmtQ8) {
+            const uint4 c0 = ld_shared_v4(srow + 32 * m), c1 = ld_shared_v4(srow + 32 * m + 16);
+            st_shared_v4(chunk_addr(dst, r, 4 * m + 0), dequant_q8_chunk(c0.x, c0.y, d2));
+            st_shared_v4(chunk_addr(dst, r, 4 * m + 1), dequant_q8_chunk(c0.z, c0.w, d2));
+            st_shared_v4(chunk_addr(dst, r, 4 * m + 2), dequant_q8_chunk(c1.x, c1.y, d2));
+            st_shared_v4(chunk_addr(dst, r, 4 * m + 3), dequant_q8_chunk(c1.z, c1.w, d2));
+        } else {
+            const uint4 w = ld_shared_v4(srow + 16 * m);
+            const uint32_t M = 0x0F0F0F0Fu;
+            st_shared_v4(chunk_addr(dst, r, 4 * m + 0), dequant_q4_chunk(w.x & M, w.y & M, d2));
+            st_shared_v4(chunk_addr(dst, r, 4 * m + 1), dequant_q4_chunk(w.z & M, w.w & M, d2));
+            st_shared_v4(chunk_addr(dst, r, 4 * m + 2), dequant_q4_chunk((w.x >> 4) & M, (w.y >> 4) & M, d2));
+            st_shared_v4(chunk_addr(dst, r, 4 * m + 3), dequant_q4_chunk((w.z >> 4) & M, (w.w >> 4) & M, d2));
+        }
+    }
+}
+
 // A stored row of the cache format into ring row r of the slot at `dst`.
 template <int KVF>
 __device__ __forceinline__ void dequant_row_to_ring(const uint8_t* rowq, bool ok, uint32_t dst,
@@ -380,6 +446,64 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         cp_async_commit();
         cp_async_wait<0>();
         named_barrier(PRODUCER_BAR, PTHREADS);
+        // Row r of group g's current unit: a selected compressed row (index checked; with
+        // `report`, an out-of-range entry sets the status word) or a window row.
+        auto resolve_row = [&](int g, const GroupCursor& cu, int r, long long& src_row, bool& cmp,
+                               bool report) {
+            const int* tk = reinterpret_cast<const int*>(smem + idx_buf(g, cu.m));
+            const int gr = (cu.tr.u0 + cu.u - 1) * BR + r;
+            src_row = 0;
+            cmp = false;
+            if (gr < cu.tr.nsel) {
+                const int j = tk[gr];
+                if (p.vis_mask == nullptr) {
+                    if (j >= 0 && j < cu.tr.nv) {
+                        src_row = j;
+                        cmp = true;
+                        return true;
+                    }
+                    if (report && (lane & 3) == 0) record_status(p.wc.status, kStatusBounds);
+                    return false;
+                }
+                if (j >= 0 && j < p.mask_cols) {
+                    if (p.vis_mask[(size_t)cu.tr.t * p.mask_ld + j] != 0) {
+                        src_row = j;
+                        cmp = true;
+                        return true;
+                    }
+                    return false;
+                }
+                if (j != -1 && report && (lane & 3) == 0) record_status(p.wc.status, kStatusBounds);
+                return false;
+            }
+            if (gr < cu.tr.nrows) {
+                src_row = cu.tr.s_lo + gr - cu.tr.nsel;
+                return true;
+            }
+            return false;
+        };
+        auto stage_buf = [&](int uc) { return sbase + L::OFF_STAGE + (uc & 1) * L::STAGE; };
+        // Staged formats: copy the rows of the unit after `uc` (if it is a row unit) into
+        // the other staging buffer; this lane's row and blocks only.
+        auto stage_next = [&](const MergedCursor& at, int uc) {
+            MergedCursor nx = at;
+            nx.advance(p);
+            if (nx.valid()) {
+                const GroupCursor cn = nx.group(nx.turn);
+                if (cn.u != 0) {
+                    const int r = 8 * pw + (lane >> 2);
+                    long long src_row;
+                    bool cmp;
+                    if (resolve_row(nx.turn, cn, r, src_row, cmp, false)) {
+                        const uint8_t* base_q = reinterpret_cast<const uint8_t*>(cmp ? p.kv_cmp : p.kv_raw);
+                        stage_row_copy<KVF == kFmtQ8 ? kFmtQ8 : kFmtQ4>(
+                            base_q + (size_t)src_row * p.kv_row_bytes, stage_buf(uc + 1) + r * L::QROW,
+                            lane & 3);
+                    }
+                }
+            }
+            cp_async_commit();
+        };
         MergedCursor mc;
         mc.start(p);
         // A producer warp whose wait gives up stops copying but keeps walking the units
@@ -412,37 +536,24 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                     cp_async_wait<1>();
                 }
                 named_barrier(PRODUCER_BAR, PTHREADS);
+                if constexpr (L::STAGED)
+                    if (!abort) stage_next(mc, uc);   // the top-k rows it needs are in place
                 continue;
             }
             if (abort) continue;
-            const int* tk = reinterpret_cast<const int*>(smem + idx_buf(mc.turn, cu.m));
             const int r = 8 * pw + (lane >> 2);   // this lane's row of the unit
-            const int gr = (cu.tr.u0 + cu.u - 1) * BR + r;
-            // the row's index: a compressed row (>= 0 from the top-k) or a raw row (-1 - s)
             long long src_row = 0;
-            bool ok = false, cmp = false;
-            if (gr < cu.tr.nsel) {
-                const int j = tk[gr];
-                if (p.vis_mask == nullptr) {
-                    if (j >= 0 && j < cu.tr.nv) {
-                        src_row = j;
-                        ok = cmp = true;
-                    } else if ((lane & 3) == 0) {
-                        record_status(p.wc.status, kStatusBounds);
-                    }
-                } else if (j >= 0 && j < p.mask_cols) {
-                    if (p.vis_mask[(size_t)cu.tr.t * p.mask_ld + j] != 0) {
-                        src_row = j;
-                        ok = cmp = true;
-                    }
-                } else if (j != -1 && (lane & 3) == 0) {
-                    record_status(p.wc.status, kStatusBounds);
-                }
-            } else if (gr < cu.tr.nrows) {
-                src_row = cu.tr.s_lo + gr - cu.tr.nsel;
-                ok = true;
-            }
-            if constexpr (KVF == kFmtF16) {
+            bool cmp = false;
+            const bool ok = resolve_row(mc.turn, cu, r, src_row, cmp, true);
+            if constexpr (L::STAGED) {
+                // this unit's rows were copied to staging[uc & 1] one unit ago; copy the next
+                // unit's rows to the other buffer, then dequantize this one into the slot
+                cp_async_wait<0>();
+                __syncwarp();
+                stage_next(mc, uc);
+                dequant_staged_to_ring<KVF>(stage_buf(uc) + r * L::QROW, ok, dst, r, lane & 3);
+                mbar_arrive(full_bar(s));          // release: this thread's stores are visible
+            } else if constexpr (KVF == kFmtF16) {
                 const __half* row = ok ? (cmp ? p.kv_cmp : p.kv_raw) + (size_t)src_row * DQK
                                        : p.kv_raw + (size_t)cu.tr.t * DQK;   // valid stand-in
 #pragma unroll
@@ -465,6 +576,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                 reinterpret_cast<volatile uint8_t*>(rowmask + s)[pw] = (uint8_t)m8;
                 mbar_arrive(full_bar(s));         // release: the mask byte is visible with the slot
             }
+            if constexpr (L::STAGED) __syncwarp();   // staging[uc & 1] is read before its reuse
         }
         if (p.prefetch_bytes > 0 && !abort) {
             // This CTA's slice of the region, in 16-byte-aligned pieces of up to 32 KB,
