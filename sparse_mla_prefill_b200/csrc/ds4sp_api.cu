@@ -112,7 +112,8 @@ constexpr int kMaxDevices = 64;
 
 // cudaFuncSetAttribute(kernel, max dynamic shared memory) once per (device, kernel): the
 // attribute belongs to the device's copy of the function.
-ds4sp_status set_smem_once(ds4sp_handle* h, const void* fn, int bytes, int slot, const char* what) {
+ds4sp_status set_smem_once(ds4sp_handle* h, const void* fn, int bytes, int slot, const char* what,
+                           int launch_regs = 0) {
     static std::mutex mu;
     static bool done[kMaxDevices][32] = {};
     if (h->device < 0 || h->device >= kMaxDevices || slot < 0 || slot >= 32)
@@ -121,6 +122,14 @@ ds4sp_status set_smem_once(ds4sp_handle* h, const void* fn, int bytes, int slot,
     if (done[h->device][slot]) return DS4SP_OK;
     const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return cuda_fail(e, what);
+    if (launch_regs) {   // a setmaxnreg split that assumes this launch register count
+        cudaFuncAttributes fa;
+        const cudaError_t ea = cudaFuncGetAttributes(&fa, fn);
+        if (ea != cudaSuccess) return cuda_fail(ea, what);
+        if (fa.numRegs != launch_regs)
+            return fail(DS4SP_ERR_UNSUPPORTED, "%s: kernel built with %d registers, not %d", what,
+                        fa.numRegs, launch_regs);
+    }
     done[h->device][slot] = true;
     return DS4SP_OK;
 }
@@ -362,7 +371,8 @@ ds4sp_status dispatch_indexer_h(ds4sp_handle* h, const void* q_idx, const void* 
 
 // Indexer and top-k in one launch (indexer_topk_fused_kernel), when the call qualifies:
 // no explicit mask, some token sees a compressed row, the key rows of a token block fit
-// the kernel's 64 KB key buffer and the launch has at most kFusedMaxBlocks token blocks.
+// one of the kernel's two 40 KB key buffers (2,560 rows, a 10,240-token context, at 64
+// index heads) and the launch has at most kFusedMaxBlocks token blocks.
 // Returns DS4SP_ERR_UNSUPPORTED (with nothing launched) when it does not qualify.
 template <int D_I, int H_I>
 ds4sp_status launch_fused(ds4sp_handle* h, const void* q_idx, const void* k_idx, const float* w,
@@ -382,7 +392,7 @@ ds4sp_status launch_fused(ds4sp_handle* h, const void* q_idx, const void* k_idx,
         return fail(DS4SP_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     DS4SP_TRY(set_smem_once(h, reinterpret_cast<const void*>(indexer_topk_fused_kernel<D_I, H_I>),
                             C::SMEM_BYTES, fused_slot(D_I, H_I),
-                            "cudaFuncSetAttribute(fused indexer)"));
+                            "cudaFuncSetAttribute(fused indexer)", C::LAUNCH_REGS));
     FusedParams p;
     p.w = w;
     p.topk = topk;

@@ -16,15 +16,16 @@
 // assigns the launch's token blocks to the persistent CTAs by longest-processing-time
 // on their cost (tiles, plus the select), heaviest first.
 // Per unit: the epilogue warps turn each tile's accumulator into order-preserving keys
-// of the scores (the top-k kernel's mapping) in a shared-memory key buffer [tokens of
-// the block][128 x tiles]; after the last tile the same warps run the radix select of
-// topk_radix.cuh, four groups of two warps on four tokens at once (each group with its
-// own named barrier), and write the tokens' indices. Meanwhile the q_idx loader brings the next unit's block
-// into the (single) B buffer as soon as this unit's MMAs have read it, and the MMA warp
-// runs ahead by the two TMEM accumulators.
-// Roles and pipelines are those of indexer_tcgen05_kernel (warp 0 streams k_idx tiles,
-// warp 10 loads q_idx blocks, warp 1 issues the MMAs, warps 2-9 run the epilogue and the
-// select); every wait is bounded (device_common.cuh).
+// of the scores (the top-k kernel's mapping) in one of two shared-memory key buffers
+// [tokens of the block][128 x tiles]; when the unit's last tile is done they hand the
+// buffer to eight select warps and go on with the next unit's tiles. The select warps
+// run the radix select of topk_radix.cuh, four groups of two warps on four tokens at
+// once (each group with its own named barrier), write the tokens' indices and hand the
+// buffer back. So the select of one unit overlaps the tensor-core work of the next.
+// Warps: 0 streams k_idx tiles (TMA), 1 owns TMEM and issues the MMAs, 2 loads q_idx
+// blocks into the single B buffer as soon as the previous unit's MMAs have read it, 3 is
+// idle, 4-11 run the epilogue, 12-19 the select. setmaxnreg gives the epilogue warps
+// most of the registers. Every wait is bounded (device_common.cuh).
 #pragma once
 
 #include <cuda.h>
@@ -41,29 +42,35 @@ struct FusedTile {
     static constexpr int BM = T::BM, BN = T::BN, TB = T::TB, KSUB = T::KSUB;
     static constexpr int A_SUB = T::A_SUB, A_STAGE = T::A_STAGE, B_SUB = T::B_SUB;
     static constexpr int B_BYTES = T::B_BYTES, A_STAGES = T::A_STAGES;
-    static constexpr int EPI_WARPS = 8, EPI_THREADS = EPI_WARPS * 32;
-    static constexpr int B_WARP = 2 + EPI_WARPS;
-    static constexpr int THREADS = (3 + EPI_WARPS) * 32;
+    static constexpr int A_WARP = 0, MMA_WARP = 1, B_WARP = 2;
+    static constexpr int EPI_WARP0 = 4, EPI_WARPS = 8, EPI_THREADS = EPI_WARPS * 32;
+    static constexpr int SEL_WARP0 = 12, SEL_WARPS = 8, SEL_ALL = SEL_WARPS * 32;
+    static constexpr int THREADS = (SEL_WARP0 + SEL_WARPS) * 32;  // 640
+    // Registers per thread: the launch's (THREADS x LAUNCH_REGS) is split by setmaxnreg
+    // between the warpgroups; the host checks the built count before the first launch.
+    static constexpr int LAUNCH_REGS = 96, CTRL_REGS = 40, EPI_REGS = 152, SEL_REGS = 64;
+    static_assert(4 * 32 * CTRL_REGS + EPI_THREADS * EPI_REGS + SEL_ALL * SEL_REGS <=
+                      THREADS * LAUNCH_REGS, "register split must fit the launch's registers");
     static constexpr int TMEM_COLS = 2 * BN;
-    static constexpr int KEY_BYTES = 64 * 1024;                   // [TB][kld] uint32 keys
+    static constexpr int KEY_BYTES = 40 * 1024;                   // one of two key buffers
     static constexpr int OFF_B = 0;                               // one B buffer
     static constexpr int OFF_A = B_BYTES;
     static constexpr int OFF_KEYS = OFF_A + A_STAGES * A_STAGE;
-    static constexpr int OFF_W = OFF_KEYS + KEY_BYTES;            // two w buffers
+    static constexpr int OFF_W = OFF_KEYS + 2 * KEY_BYTES;        // two w buffers
     static constexpr int OFF_SEL = OFF_W + 2 * BN * 4;            // select scratch
-    // The select runs on SEL_GROUPS groups of SEL_THREADS epilogue threads, one token per
-    // group at a time; per group: hist[256], w_or/w_and/w_cnt[2], s_digit, s_above,
-    // warp_tot[2] (8-byte aligned); after the groups, the abort flag.
-    static constexpr int SEL_GROUPS = 4, SEL_THREADS = EPI_THREADS / SEL_GROUPS;
+    // Per select group: hist[256], w_or/w_and/w_cnt[2], s_digit, s_above, warp_tot[2]
+    // (8-byte aligned); after the groups, the abort flag.
+    static constexpr int SEL_GROUPS = 4, SEL_THREADS = SEL_ALL / SEL_GROUPS;
     static constexpr int GROUP_SEL = 256 * 4 + 3 * 2 * 4 + 2 * 4 + 2 * 8;
     static constexpr int SEL_ABORT = SEL_GROUPS * GROUP_SEL;      // byte offset of the flag
     static constexpr int SEL_BYTES = SEL_ABORT + 16;
     static constexpr int OFF_BAR = OFF_SEL + SEL_BYTES;
-    // afull[A_STAGES], aempty[A_STAGES], bfull, bempty, tempty[2], done
-    static constexpr int N_BARS = 2 * A_STAGES + 1 + 1 + 2 + 1;
+    // afull[A_STAGES], aempty[A_STAGES], bfull, bempty, tempty[2], kfull[2], kempty[2], done
+    static constexpr int N_BARS = 2 * A_STAGES + 1 + 1 + 2 + 2 + 2 + 1;
     static constexpr int OFF_TMEM_PTR = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;   // + alignment slack
     static constexpr uint32_t IDESC = T::IDESC;
+    static constexpr int EPI_BAR = 1, SEL_BAR = 6;                // named barriers (2-5: groups)
     static_assert(GROUP_SEL % 8 == 0 && OFF_SEL % 8 == 0, "8-byte aligned select scratch");
     static_assert(SEL_THREADS == 64, "two warps per select group");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -82,7 +89,7 @@ struct FusedParams {
     uint16_t blk[kFusedMaxBlocks];
 };
 
-// Named barrier of one select group: two epilogue warps, barrier id 2 + group.
+// Named barrier of one select group: two select warps, barrier id 2 + group.
 struct GroupSync {
     int id;
     __device__ __forceinline__ void operator()() const { named_barrier(id, 64); }
@@ -158,15 +165,21 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t base = (raw_u32 + 1023u) & ~1023u;         // 128B-swizzle atoms need 1 KB alignment
     uint8_t* smem = smem_raw + (base - raw_u32);
-    uint32_t* keys = reinterpret_cast<uint32_t*>(smem + C::OFF_KEYS);
+    auto keys_of = [&](int ui) {
+        return reinterpret_cast<uint32_t*>(smem + C::OFF_KEYS + (ui & 1) * C::KEY_BYTES);
+    };
     float* sw = reinterpret_cast<float*>(smem + C::OFF_W);
+    uint8_t* sel = smem + C::OFF_SEL;
+    volatile uint32_t* sel_abort = reinterpret_cast<volatile uint32_t*>(sel + C::SEL_ABORT);
     const uint32_t bar0 = base + C::OFF_BAR;
     auto afull = [&](int s) { return bar0 + 8u * s; };
     auto aempty = [&](int s) { return bar0 + 8u * (C::A_STAGES + s); };
     const uint32_t bfull = bar0 + 8u * (2 * C::A_STAGES);
     const uint32_t bempty = bar0 + 8u * (2 * C::A_STAGES + 1);
     auto tempty = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + 2 + i); };
-    const uint32_t done_bar = bar0 + 8u * (2 * C::A_STAGES + 4);
+    auto kfull = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + 4 + i); };
+    auto kempty = [&](int i) { return bar0 + 8u * (2 * C::A_STAGES + 6 + i); };
+    const uint32_t done_bar = bar0 + 8u * (2 * C::A_STAGES + 8);
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_PTR);
 
     // Token block tb of the launch: tokens [tok0, tok_end), j-tiles 0 .. n_tiles-1.
@@ -185,14 +198,18 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         mbar_init(bfull, 1);
         mbar_init(bempty, 1);
-        for (int i = 0; i < 2; ++i) mbar_init(tempty(i), C::EPI_WARPS);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(tempty(i), C::EPI_WARPS);
+            mbar_init(kfull(i), C::EPI_WARPS);     // the epilogue warps hand a key buffer over
+            mbar_init(kempty(i), C::SEL_WARPS);    // the select warps hand it back
+        }
         mbar_init(done_bar, 1);
-        *reinterpret_cast<volatile uint32_t*>(smem + C::OFF_SEL + C::SEL_ABORT) = 0u;
+        *sel_abort = 0u;
         fence_mbar_init();
         prefetch_tmap(&tmap_k);
         prefetch_tmap(&tmap_q);
     }
-    if (warp == 1) {
+    if (warp == C::MMA_WARP) {
         tmem_alloc(smem_u32(tmem_ptr), C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -206,9 +223,10 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
     grid_dependents_launch();
 
     bool abort = false;
-    if (warp == C::B_WARP || warp == 0) {
-        // ------------------------------------------------------------ TMA producers
+    if (warp < C::EPI_WARP0) {
+        regs_decrease<C::CTRL_REGS>();
         if (warp == C::B_WARP && lane == 0) {
+            // ------------------------------------------------------------ q_idx loader
             int issued = 0;
             for (int u = u_begin; u < u_end && !abort; ++u) {
                 int tok0, tok_end, n_tiles;
@@ -223,7 +241,8 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             // Every bulk copy this CTA started must land before the CTA exits.
             if (issued) mbar_wait_drain(bfull, (issued - 1) & 1, p.wc);
-        } else if (warp == 0 && lane == 0) {
+        } else if (warp == C::A_WARP && lane == 0) {
+            // ------------------------------------------------------------ k_idx loader
             int a_it = 0;
             int a_issued[C::A_STAGES] = {};
             for (int u = u_begin; u < u_end && !abort; ++u) {
@@ -242,11 +261,8 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             for (int s = 0; s < C::A_STAGES; ++s)
                 if (a_issued[s]) mbar_wait_drain(afull(s), (a_issued[s] - 1) & 1, p.wc);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        } else if (warp == C::MMA_WARP && lane == 0) {
+            // ------------------------------------------------------------ MMA issuer
             const uint64_t a_desc0 = umma_desc_sw128(base + C::OFF_A);
             const uint64_t b_desc = umma_desc_sw128(base + C::OFF_B);
             int tc = 0;
@@ -276,10 +292,10 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
             mbar_wait_drain(done_bar, 0, p.wc);
         }
         __syncwarp();
-    } else {
-        // ------------------------------------------------------------ epilogue + select
-        const int e = warp - 2;                      // 0..7
-        const int etid = threadIdx.x - 64;           // 0..255
+    } else if (warp < C::SEL_WARP0) {
+        // ------------------------------------------------------------ epilogue
+        regs_increase<C::EPI_REGS>();
+        const int e = warp - C::EPI_WARP0;           // 0..7
         const int quarter = warp & 3;                // TMEM lanes 32*quarter .. +31
         const int half = e / 4;                      // columns 128*half .. +127
         const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + half * 128;
@@ -290,27 +306,31 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int tl = col / H_I;
             return (tok0 + tl < tok_end) ? p.w[(size_t)(tok0 - p.t0 + tl) * H_I + (col % H_I)] : 0.f;
         };
-        uint8_t* sel = smem + C::OFF_SEL;
-        volatile uint32_t* sel_abort = reinterpret_cast<volatile uint32_t*>(sel + C::SEL_ABORT);
         int tc = 0;
         float w_next = u_begin < u_end ? unit_weight(u_begin) : 0.f;
         for (int u = u_begin; u < u_end; ++u) {
+            const int ui = u - u_begin;
             int tok0, tok_end, n_tiles;
             unit_of(u, tok0, tok_end, n_tiles);
             const float w_this = w_next;
             w_next = u + 1 < u_end ? unit_weight(u + 1) : 0.f;
-            float* swb = sw + ((u - u_begin) & 1) * C::BN;
+            float* swb = sw + (ui & 1) * C::BN;
             swb[col] = 0.5f * w_this;                // halved: see epilogue_half
-            // also orders the previous unit's select (key reads) before this unit's key writes
-            named_barrier(1, C::EPI_THREADS);
+            named_barrier(C::EPI_BAR, C::EPI_THREADS);
             const float* wh = swb + half * 128;
+            uint32_t* keys = keys_of(ui);
+            // this key buffer's previous unit (ui - 2) must be selected before it is rewritten
+            if (!__all_sync(0xffffffffu, mbar_wait(kempty(ui & 1), ((ui >> 1) & 1) ^ 1, p.wc, abort))) {
+                abort = true;
+                *sel_abort = 1u;
+            }
             for (int it = 0; it < n_tiles; ++it, ++tc) {
                 const int buf = tc & 1;
                 const bool ready = mbar_wait(aempty(tc % C::A_STAGES), (tc / C::A_STAGES) & 1,
                                              p.wc, abort);
                 if (!__all_sync(0xffffffffu, ready)) {           // warp-uniform skip
                     abort = true;
-                    *sel_abort = 1u;                             // read by all after the barrier
+                    *sel_abort = 1u;
                     continue;
                 }
                 tc_fence_after();
@@ -329,12 +349,26 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
                             keys[tl * p.kld + j] = order_key(score);
                     });
             }
-            named_barrier(1, C::EPI_THREADS);       // every key of the unit is in place
-            // A warp that gave up a wait skipped tiles; then no warp runs the select (its
-            // barriers need all eight), and the launch ends with its outputs undefined.
-            if (*sel_abort) continue;
+            // hand the unit's keys to the select warps (also after a give-up, so that they
+            // are not left waiting; they read the abort flag first)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(kfull(ui & 1));
+        }
+    } else {
+        // ------------------------------------------------------------ select
+        regs_decrease<C::SEL_REGS>();
+        const int stid = threadIdx.x - C::SEL_WARP0 * 32;   // 0..255
+        const int g = stid / C::SEL_THREADS, gtid = stid % C::SEL_THREADS;
+        for (int u = u_begin; u < u_end; ++u) {
+            const int ui = u - u_begin;
+            int tok0, tok_end, n_tiles;
+            unit_of(u, tok0, tok_end, n_tiles);
+            const bool ready = mbar_wait(kfull(ui & 1), (ui >> 1) & 1, p.wc, abort);
+            // The epilogue may raise the flag at any time: one reduction gives every select
+            // warp the same answer, so that none is left alone at a group barrier.
+            if (named_barrier_or(C::SEL_BAR, C::SEL_ALL, !ready || *sel_abort != 0u)) break;
+            const uint32_t* keys = keys_of(ui);
             // The block's tokens, one per select group at a time (the groups run at once).
-            const int g = etid / C::SEL_THREADS, gtid = etid % C::SEL_THREADS;
             for (int tl = g; tl < tok_end - tok0; tl += C::SEL_GROUPS) {
                 const int t = tok0 + tl, n = n_vis(t, p.ratio);
                 int32_t* out = p.topk + (size_t)(t - p.t0) * p.k;
@@ -345,13 +379,15 @@ indexer_topk_fused_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 fused_select_row(keys + tl * p.kld, n, p.k, out, sel + g * C::GROUP_SEL, gtid,
                                  GroupSync{2 + g});
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(kempty(ui & 1));     // the buffer may be rewritten
         }
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if (warp == C::MMA_WARP) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
 }  // namespace ds4sp

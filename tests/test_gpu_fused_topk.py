@@ -86,7 +86,7 @@ def test_edge_cases_fused(T, H_i, D_i, k, n_swa, band):
 
 def test_all_scores_equal_fused():
     """Zero index weights: every key equal, the k lowest rows win (ties to the lower j)."""
-    T, k = 600, 16
+    T, k = 512, 16                   # 128 rows at most: inside the fused kernel's key buffer
     wl = Workload("ties", T=T, H_i=4, D_i=64, top_k=k, n_swa=16, seed=T, band=256)
     inp = generate_small(T, 4, 64, seed=T + 2, weight_max=0)
     res = _both(wl, to_device(inp))
