@@ -48,6 +48,7 @@ ds4sp_status cuda_fail(cudaError_t e, const char* what) {
 
 constexpr int kMaxTopkCandidates = 51200;  // top-k keeps a token's row in shared memory
 constexpr int kHostStep = 1024;            // ds4sp_prefill_host: tokens per copy/compute step
+constexpr int kHostTail = 256;             // ds4sp_prefill_host: tokens of the last step at most
 
 enum Kind { kIndexer = 0, kTopk = 1, kAttn = 2 };
 
@@ -919,6 +920,13 @@ ds4sp_status ds4sp_prefill_host(ds4sp_handle* h, int n_tokens, const ds4sp_io* h
             steps.push_back({b, u, n});
             u += n;
         }
+    }
+    // Only the last step's compute and copy out trail the copies in (the link is the
+    // bound): cut the last kHostTail tokens into a step of their own.
+    if (steps.back().n - kHostTail > attn::SPLIT_MAX_TOKENS) {
+        Step& last = steps.back();
+        last.n -= kHostTail;
+        steps.push_back({last.band, last.t0 + last.n, kHostTail});
     }
     const int n_steps = (int)steps.size();
 
