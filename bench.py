@@ -281,6 +281,22 @@ def verify_latency(dev, reps: int = 50):
             e1.record()
             torch.cuda.synchronize()
             res[f"q{q}"] = round(e0.elapsed_time(e1) / reps * 1e3, 1)
+            # The same step captured once into a CUDA graph and replayed: the launches'
+            # host cost (argument checks, schedules, three to four launches) leaves the
+            # step's latency.
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                call()
+            for _ in range(5):
+                g.replay()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            res[f"graph_q{q}"] = round(e0.elapsed_time(e1) / reps * 1e3, 1)
+            del g
         st, bits = D.ds4sp_device_status(h)
         if st != D.OK:
             raise RuntimeError(f"device status {bits:#x} after verify timing")
@@ -288,7 +304,8 @@ def verify_latency(dev, reps: int = 50):
         D.ds4sp_destroy(h)
     return {"workload": "verify: 122,880-token context, the last q = 1..5 tokens, top_k 512, "
                         "n_swa 128, indexer 64x128, seed 4",
-            "unit": "us per step (indexer + top-k + attention)", **res}
+            "unit": "us per step (indexer + top-k + attention); q<n>: launched from the host "
+                    "each step, graph_q<n>: one captured CUDA graph replayed", **res}
 
 
 def config_throughput(name, dev, steps, stream):

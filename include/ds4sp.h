@@ -229,7 +229,15 @@ int ds4sp_next_band(const ds4sp_handle* h);
 /* Synchronise `stream`, then read and clear the handle's device status word:
  * DS4SP_OK, or DS4SP_ERR_DEVICE_BOUNDS if a kernel skipped an out-of-range index or
  * gave up a bounded wait since the last read. *bits (may be NULL) receives the raw
- * word: bit 0 = index out of range, bit 1 = wait gave up. */
+ * word: bit 0 = index out of range, bit 1 = wait gave up. It also clears the word
+ * through which the CTAs of a launch that gave up tell one another.
+ *
+ * CUDA graphs: ds4sp_indexer_topk, ds4sp_sparse_attn and ds4sp_prefill_band may be
+ * captured into a graph (stream capture) once each has run outside the capture with
+ * the same configuration (the first call sets kernel attributes). A replay launches
+ * the captured kernels with their captured arguments; after a replay that gave up a
+ * wait, call this function before the next replay. ds4sp_destroy does not wait for
+ * replays: finish them (synchronise their stream) before destroying the handle. */
 ds4sp_status ds4sp_device_status(ds4sp_handle* h, void* stream, uint32_t* bits);
 
 /* Per-kernel timing. When enabled, the handle records CUDA events around each of its

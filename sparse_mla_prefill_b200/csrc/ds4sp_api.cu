@@ -625,6 +625,13 @@ ds4sp_status check_ptr(const void* p, const char* name) {
 
 
 ds4sp_status record_last(ds4sp_handle* h, cudaStream_t stream) {
+    // Not while the stream is being captured into a graph: the record would belong to
+    // the graph, and ds4sp_destroy could not wait on it (replays are the caller's to
+    // finish before destroy).
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess)
+        return cuda_fail(cudaGetLastError(), "cudaStreamIsCapturing");
+    if (cs != cudaStreamCaptureStatusNone) return DS4SP_OK;
     const cudaError_t e = cudaEventRecord(h->last, stream);
     return e == cudaSuccess ? DS4SP_OK : cuda_fail(e, "cudaEventRecord");
 }
@@ -1032,7 +1039,9 @@ ds4sp_status ds4sp_device_status(ds4sp_handle* h, void* stream, uint32_t* bits) 
     uint32_t word = 0;
     cudaError_t e = cudaStreamSynchronize(s);
     if (e == cudaSuccess) e = cudaMemcpy(&word, h->d_status, sizeof(word), cudaMemcpyDeviceToHost);
-    if (e == cudaSuccess) e = cudaMemset(h->d_status, 0, sizeof(uint32_t));
+    // Both words: the status and the launch give-up word (a replayed graph reuses its
+    // launches' epochs, which a stale give-up word would match).
+    if (e == cudaSuccess) e = cudaMemset(h->d_status, 0, 2 * sizeof(uint32_t));
     if (e != cudaSuccess) return cuda_fail(e, "ds4sp_device_status");
     if (bits) *bits = word;
     if (word) return fail(DS4SP_ERR_DEVICE_BOUNDS, "device status word 0x%x", word);
