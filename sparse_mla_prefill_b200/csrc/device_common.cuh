@@ -224,6 +224,29 @@ __device__ __forceinline__ bool named_barrier_or(int id, int count, bool pred) {
     return r != 0u;
 }
 
+// ---------------------------------------------------------------- thread-block clusters
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Every thread of every CTA of the cluster: shared-memory writes before it are visible
+// to the cluster's CTAs after it.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// A 32-bit word of CTA `rank`'s shared memory at the offset of local address `local`.
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t local, uint32_t rank) {
+    uint32_t a, v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local), "r"(rank));
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+
 // Ask L2 to fetch [src, src+bytes) from global memory (no destination, no completion
 // signal). bytes is a multiple of 16 and src 16-byte aligned.
 __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {

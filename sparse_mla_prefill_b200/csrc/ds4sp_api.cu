@@ -47,6 +47,7 @@ ds4sp_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 constexpr int kMaxTopkCandidates = 51200;  // top-k keeps a token's row in shared memory
+constexpr int kTopkCluster = 8;            // CTAs per token in topk_cluster_kernel
 constexpr int kHostStep = 1024;            // ds4sp_prefill_host: tokens per copy/compute step
 constexpr int kHostTail = 256;             // ds4sp_prefill_host: tokens of the last step at most
 
@@ -235,6 +236,27 @@ void launch_k(bool dependent, void (*kernel)(KArgs...), dim3 grid, dim3 block, s
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = dependent ? 1 : 0;
+    cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
+}
+
+// The same with thread-block clusters of `cluster` CTAs along x.
+template <class... KArgs, class... Args>
+void launch_k_cluster(bool dependent, int cluster, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                      size_t smem, cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = dependent ? 2 : 1;
     cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
 }
 
@@ -479,6 +501,17 @@ ds4sp_status launch_topk(ds4sp_handle* h, const float* scores, int ld, int t0, i
     }
     const size_t smem = (size_t)ld * 4;
     const bool pdl = h->cfg.dependent_launch != 0;
+    // A few tokens with long rows (the verify form): a cluster of kTopkCluster CTAs per
+    // token shares each row, so that the launch covers more than a handful of SMs.
+    const int n_max = nvis(t0 + n_q - 1, ratio);
+    if (!vm && n_max > 4096 && (long long)n_q * kTopkCluster <= 2LL * h->sm_count) {
+        const size_t csmem = (size_t)((n_max + kTopkCluster - 1) / kTopkCluster) * 4;
+        return launch(h, kTopk, stream, [&] {
+            launch_k_cluster(pdl, kTopkCluster, topk_cluster_kernel<kTopkCluster, 512>,
+                             n_q * kTopkCluster, 512, csmem, stream, scores, ld, t0, n_q, k, ratio,
+                             topk);
+        });
+    }
     return launch(h, kTopk, stream, [&] {
         if (big)
             launch_k(pdl, topk_radix_kernel<1024>, n_q, 1024, smem, stream, scores, ld, t0, n_q, k,

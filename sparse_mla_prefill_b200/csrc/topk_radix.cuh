@@ -271,4 +271,164 @@ topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int
     for (int s = keep + tid; s < k; s += THREADS) out[s] = -1;
 }
 
+// ---------------------------------------------------------------- a cluster per token
+//
+// The same selection for calls of a few tokens with long rows (the verify form: one to
+// five tokens, 30,720 candidates each), where one CTA per token would leave the GPU
+// idle: a cluster of CL CTAs per token, CTA r holding the keys of j in [r c, r c + c),
+// c = ceil(n / CL), in its shared memory. The OR/AND window, each radix pass's 256-bin
+// histogram and the compaction's counts are combined across the cluster through
+// distributed shared memory (each CTA reads its peers' words after a cluster barrier;
+// every CTA derives the same digits from the same sums). Histograms alternate between
+// two buffers, so one cluster barrier per pass suffices: a buffer is cleared only after
+// the barrier that follows every peer's reads of it. Analytic visibility only.
+template <int CL, int THREADS>
+__global__ void __launch_bounds__(THREADS)
+topk_cluster_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int k, int ratio,
+                    int32_t* __restrict__ topk) {
+    extern __shared__ uint32_t keys[];           // [c]
+    __shared__ uint32_t hist[2][256];
+    __shared__ uint32_t ghist[256];              // the cluster's sums of a pass
+    __shared__ uint32_t s_word[4];               // this CTA's OR, AND; kept > thr, == thr
+    __shared__ uint32_t s_all[4];                // the cluster's OR, AND; counts before this CTA
+    __shared__ uint32_t s_digit, s_above;
+    __shared__ uint32_t w_or[THREADS / 32], w_and[THREADS / 32], w_cnt[THREADS / 32];
+    __shared__ unsigned long long warp_tot[THREADS / 32];
+
+    const uint32_t rank = cluster_ctarank();
+    const int i = blockIdx.x / CL;               // the launch's token (grid = n_q x CL)
+    const int tid = threadIdx.x;
+    grid_dependency_wait();                      // the scores are complete
+    grid_dependents_launch();
+    const int t = t0 + i;
+    const int n = n_vis(t, ratio);
+    int32_t* out = topk + (size_t)i * k;
+    if (n <= k) {                                // the same in every CTA of the cluster
+        if (rank == 0)
+            for (int s = tid; s < k; s += THREADS) out[s] = s < n ? s : -1;
+        return;
+    }
+    const int c = (n + CL - 1) / CL;
+    const int jb = min(n, (int)rank * c), nl = min(n, jb + c) - jb;   // this CTA's keys
+    const float* row = scores + (size_t)i * ld + jb;
+    uint32_t kor = 0u, kand = 0xffffffffu, cand = 0u;
+    for (int x = tid; x < nl; x += THREADS) {
+        const uint32_t key = order_key(row[x]);
+        keys[x] = key;
+        kor |= key;
+        kand &= key;
+        ++cand;
+    }
+    uint32_t cta_or, cta_and, cta_cnt;
+    block_key_stats<THREADS>(kor, kand, cand, w_or, w_and, w_cnt, cta_or, cta_and, cta_cnt, tid,
+                             BlockSync{});
+    if (tid == 0) {
+        s_word[0] = cta_or;
+        s_word[1] = cta_and;
+    }
+    cluster_sync();
+    if (tid < 32) {
+        uint32_t o = 0u, a = 0xffffffffu;
+        if (tid < CL) {
+            o = ld_cluster_u32(smem_u32(&s_word[0]), tid);
+            a = ld_cluster_u32(smem_u32(&s_word[1]), tid);
+        }
+        o = __reduce_or_sync(0xffffffffu, o);
+        a = __reduce_and_sync(0xffffffffu, a);
+        if (tid == 0) {
+            s_all[0] = o;
+            s_all[1] = a;
+        }
+    }
+    __syncthreads();
+    const uint32_t all_or = s_all[0], all_and = s_all[1];
+
+    // Radix passes over the bits where the token's candidates differ (as RadixSelect).
+    uint32_t thr = all_or, need = (uint32_t)k;   // all candidates equal: the first k
+    const uint32_t diff = all_or ^ all_and;
+    if (diff != 0u) {
+        const int hi_bit = 31 - __clz(diff), lo_bit = __ffs(diff) - 1;
+        uint32_t digits = hi_bit < 31 ? ~((2u << hi_bit) - 1u) : 0u;
+        uint32_t prefix = all_or & digits, remaining = (uint32_t)k;
+        int shift = max(hi_bit - 7, 0);
+        for (int pass = 0;; ++pass) {
+            uint32_t* h = hist[pass & 1];
+            for (int b = tid; b < 256; b += THREADS) h[b] = 0u;
+            __syncthreads();
+            for (int x = tid; x < nl; x += THREADS) {
+                const uint32_t key = keys[x];
+                if ((key & digits) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+            }
+            cluster_sync();                      // every CTA's histogram of this pass
+            for (int b = tid; b < 256; b += THREADS) {
+                uint32_t sum = 0u;
+#pragma unroll
+                for (int r = 0; r < CL; ++r) sum += ld_cluster_u32(smem_u32(&h[b]), r);
+                ghist[b] = sum;
+            }
+            __syncthreads();
+            if (tid < 32) radix_find_digit(ghist, remaining, &s_digit, &s_above);
+            __syncthreads();
+            prefix |= s_digit << shift;
+            digits |= 255u << shift;
+            remaining -= s_above;
+            if (shift <= lo_bit) {
+                thr = prefix | (all_or & ((1u << shift) - 1u));
+                need = remaining;
+                break;
+            }
+            shift = max(shift - 8, 0);
+        }
+    }
+
+    // Compaction in ascending j: this CTA's keys > thr and its share of the first
+    // `need` keys == thr, after the counts of the CTAs before it.
+    const int per = (nl + THREADS - 1) / THREADS;
+    const int xb = min(nl, tid * per), xe = min(nl, xb + per);
+    uint32_t gt = 0, eq = 0;
+    for (int x = xb; x < xe; ++x) {
+        const uint32_t key = keys[x];
+        gt += key > thr;
+        eq += key == thr;
+    }
+    const unsigned long long v = ((unsigned long long)gt << 32) | eq;
+    const unsigned long long before = block_exclusive_scan<THREADS>(v, warp_tot, tid, BlockSync{});
+    if (tid == THREADS - 1) {
+        s_word[2] = (uint32_t)((before + v) >> 32);
+        s_word[3] = (uint32_t)(before + v);
+    }
+    cluster_sync();                              // every CTA's counts
+    if (tid < 32) {
+        uint32_t g = 0u, e = 0u;
+        if (tid < (int)rank) {
+            g = ld_cluster_u32(smem_u32(&s_word[2]), tid);
+            e = ld_cluster_u32(smem_u32(&s_word[3]), tid);
+        }
+        g = __reduce_add_sync(0xffffffffu, g);
+        e = __reduce_add_sync(0xffffffffu, e);
+        if (tid == 0) {
+            s_all[2] = g;
+            s_all[3] = e;
+        }
+    }
+    __syncthreads();
+    const uint32_t gt_before = s_all[2] + (uint32_t)(before >> 32);
+    const uint32_t eq_before = s_all[3] + (uint32_t)before;
+    uint32_t pos = gt_before + min(eq_before, need), eq_rank = eq_before;
+    for (int x = xb; x < xe; ++x) {
+        const uint32_t key = keys[x];
+        if (key > thr) {
+            if (pos < (uint32_t)k) out[pos] = jb + x;
+            ++pos;
+        } else if (key == thr) {
+            if (eq_rank < need) {
+                if (pos < (uint32_t)k) out[pos] = jb + x;
+                ++pos;
+            }
+            ++eq_rank;
+        }
+    }
+    cluster_sync();                              // no CTA leaves while a peer reads its words
+}
+
 }  // namespace ds4sp
