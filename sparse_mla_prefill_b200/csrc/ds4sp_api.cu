@@ -540,6 +540,12 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
             reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtQ4>),
             reinterpret_cast<const void*>(sparse_attn_mma_kernel<false, false, kFmtQ8Q4>)};
         const int fmt_of[7] = {kFmtF16, kFmtF16, kFmtF16, kFmtF16, kFmtQ8, kFmtQ4, kFmtQ8Q4};
+        auto launch_regs = [](int fmt) {
+            return fmt == kFmtQ8 ? attn::Roles<kFmtQ8>::LAUNCH_REGS
+                   : fmt == kFmtQ4 ? attn::Roles<kFmtQ4>::LAUNCH_REGS
+                   : fmt == kFmtQ8Q4 ? attn::Roles<kFmtQ8Q4>::LAUNCH_REGS
+                                     : attn::Roles<kFmtF16>::LAUNCH_REGS;
+        };
         for (int fi = 0; fi < 7; ++fi) {
             const void* fn = fns[fi];
             const int max_smem = attn_smem_bytes(fmt_of[fi], attn_max_topk(fmt_of[fi]));
@@ -549,9 +555,9 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
             cudaFuncAttributes fa;
             const cudaError_t ea = cudaFuncGetAttributes(&fa, fn);
             if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncGetAttributes(attention)");
-            if (fa.numRegs != attn::LAUNCH_REGS)   // the warp roles' register split assumes it
+            if (fa.numRegs != launch_regs(fmt_of[fi]))   // the warp roles' register split assumes it
                 return fail(DS4SP_ERR_UNSUPPORTED, "attention kernel built with %d registers, not %d",
-                            fa.numRegs, attn::LAUNCH_REGS);
+                            fa.numRegs, launch_regs(fmt_of[fi]));
         }
         const cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -613,14 +619,18 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
     return launch(h, kAttn, stream, [&] {
         // persistent: one CTA per SM, each walking its share of the work items
         const int grid = std::min(p.n_items, h->sm_count);
-        const dim3 g(grid), b(attn::THREADS);
+        const dim3 g(grid), b(attn::Roles<kFmtF16>::THREADS);
+        const dim3 bs(attn::Roles<kFmtQ8>::THREADS);   // the staged formats' eight producer warps
+        static_assert(attn::Roles<kFmtQ8>::THREADS == attn::Roles<kFmtQ4>::THREADS &&
+                          attn::Roles<kFmtQ8Q4>::THREADS == attn::Roles<kFmtF16>::THREADS,
+                      "block shapes per format");
         const bool pdl = h->cfg.dependent_launch != 0;
         if (tc) {
             launch_k(pdl, sparse_attn_tc_kernel, g, dim3(tcattn::THREADS), smem, stream, p);
         } else if (h->cfg.kv_format == kFmtQ8) {
-            launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ8>, g, b, smem, stream, p);
+            launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ8>, g, bs, smem, stream, p);
         } else if (h->cfg.kv_format == kFmtQ4) {
-            launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ4>, g, b, smem, stream, p);
+            launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ4>, g, bs, smem, stream, p);
         } else if (h->cfg.kv_format == kFmtQ8Q4) {
             launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ8Q4>, g, b, smem, stream, p);
         } else {

@@ -17,11 +17,12 @@
 // tensor-core work. The two groups' unit sequences are merged, one unit of each in
 // turn, into one stream through a 5-slot shared-memory ring with an mbarrier pair
 // per slot; producers and both groups walk the same merged order.
-//   * Warps 8-11 produce. They stage each token's top-k row in shared memory one
+//   * Warps 8-11 produce (8-15 for the staged Q8_0 / Q4_0 caches, whose dequantization
+//     needs the extra warps). They stage each token's top-k row in shared memory one
 //     token ahead per group, resolve and check every row, and copy it in 16-byte chunks
 //     with cp.async; cp.async.mbarrier.arrive.noinc lets the slot's barrier count the
 //     copies without the producer waiting for them. Each producer warp also publishes
-//     which of its 8 rows are valid. Producers never take part in the consumers'
+//     which of its rows are valid. Producers never take part in the consumers'
 //     barriers, and setmaxnreg moves most of their registers to the consumers.
 //   * Warps 4g .. 4g+3 form consumer group g, with the 16 heads as the M of
 //     mma.sync.m16n8k16. Group warp w (kh = w/2, rh = w%2) computes the partial
@@ -57,22 +58,14 @@ constexpr int NS = 5;                         // ring slots
 constexpr int GROUPS = 2;                     // consumer groups, each on its own token
 constexpr int GWARPS = 4;                     // warps per consumer group
 constexpr int CWARPS = GROUPS * GWARPS;       // consumer warps
-constexpr int PWARPS = 4;                     // producer warps
 constexpr int GTHREADS = GWARPS * 32;
 constexpr int CTHREADS = CWARPS * 32;
-constexpr int PTHREADS = PWARPS * 32;
-constexpr int THREADS = CTHREADS + PTHREADS;
 constexpr int PRODUCER_BAR = 1;               // named barriers; group g uses GROUP_BAR + g
 constexpr int GROUP_BAR = 2;
-// Registers per thread: the kernel is built for LAUNCH_REGS (one CTA of THREADS per
+// Registers per thread: the kernel is built for Roles<KVF>::LAUNCH_REGS (one CTA per
 // SM); producers hand part of theirs to the consumers with setmaxnreg. The host checks
 // the built count before the first launch: a split above the launch's total would
 // leave the consumers' setmaxnreg.inc waiting.
-constexpr int LAUNCH_REGS = 168;
-constexpr int CONSUMER_REGS = 224;
-constexpr int PRODUCER_REGS = 56;
-static_assert(CWARPS * 32 * CONSUMER_REGS + PWARPS * 32 * PRODUCER_REGS <= THREADS * LAUNCH_REGS,
-              "register split must fit the launch's registers");
 constexpr float HEADROOM = 8.f;               // log2 units a tile may exceed the reference
 constexpr int SLOT = BR * ROW;
 constexpr int P_PITCH = (BR + 8) * 2;         // fp16 probabilities of one unit, 80 B per head
@@ -108,8 +101,11 @@ struct RingLayout {
     static constexpr int STAGE = BR * QROW;                 // one staging buffer
     static constexpr int OFF_RING = 0;
     static constexpr int OFF_GROUP = OFF_RING + NS_ * SLOT_;
-    static constexpr int OFF_MASK = OFF_GROUP + GROUPS * G_BYTES;   // row-validity bits per slot
-    static constexpr int OFF_BAR = OFF_MASK + 32;                   // full[NS_], empty[NS_]
+    // Row-validity bytes per slot: one per producer warp (four, or eight for the staged
+    // formats' eight producer warps).
+    static constexpr int MASK_STRIDE = STAGED ? 8 : 4;
+    static constexpr int OFF_MASK = OFF_GROUP + GROUPS * G_BYTES;
+    static constexpr int OFF_BAR = OFF_MASK + 8 * MASK_STRIDE;      // full[NS_], empty[NS_]
     static constexpr int OFF_STAGE = OFF_BAR + 2 * NS_ * 8;
     static constexpr int OFF_IDX = OFF_STAGE + 2 * STAGE;
     __host__ __device__ static constexpr int smem_bytes(int k) {
@@ -124,8 +120,32 @@ struct RingLayout {
     static_assert(smem_bytes(MAX_K) <= SMEM_LIMIT, "shared memory budget");
 };
 __host__ __device__ constexpr int smem_bytes(int k) { return RingLayout<kFmtF16>::smem_bytes(k); }
+
+// Producer warps of a cache format: four (eight rows of the unit each, four lanes a row)
+// for fp16 rows and the split format; eight (four rows each, eight lanes a row) for the
+// staged Q8_0 / Q4_0 rows, whose dequantization is the producers' limit. The register
+// split keeps the launch's 64K registers: consumers 224 / producers 56 at 384 threads,
+// 200 / 56 at 512.
+template <int KVF>
+struct Roles {
+    static constexpr int PW = RingLayout<KVF>::STAGED ? 8 : 4;   // producer warps
+    static constexpr int PT = PW * 32;
+    static constexpr int THREADS = CTHREADS + PT;
+    static constexpr int RPW = BR / PW;          // rows per producer warp
+    static constexpr int LPR = 32 / RPW;         // lanes per row
+    static constexpr int LPR_LOG2 = LPR == 8 ? 3 : 2;
+    static constexpr int LAUNCH_REGS = 65536 / THREADS / 8 * 8;
+    static constexpr int PREGS = 56;
+    static constexpr int CREGS = (THREADS * LAUNCH_REGS - PT * PREGS) / CTHREADS / 8 * 8;
+    static_assert(CREGS <= 224 && CWARPS * 32 * CREGS + PT * PREGS <= THREADS * LAUNCH_REGS,
+                  "register split must fit the launch's registers");
+    static_assert(RPW * PW == BR && LPR * RPW == 32 && (1 << LPR_LOG2) == LPR,
+                  "whole rows per producer warp");
+    static_assert(CH % LPR == 0, "a row's chunks split evenly over its lanes");
+    static_assert(PW == RingLayout<KVF>::MASK_STRIDE, "one row-validity byte per producer warp");
+};
 static_assert(DV == GWARPS * 128, "each group warp owns 128 value dims");
-static_assert(CH % 8 == 0 && BR * CH == PTHREADS * 18, "producer chunk split");
+static_assert(CH % 8 == 0, "whole 128-byte swizzle groups per row");
 static_assert(RingLayout<kFmtF16>::MAX_K == MAX_TOPK, "fp16 ring holds top_k up to 2048");
 
 // 16-byte chunk swizzle: eight consecutive rows put one chunk in eight different bank
@@ -315,16 +335,16 @@ __device__ __forceinline__ void dequant_part_to_ring(const uint8_t* rowq, bool o
     }
 }
 
-// Staged quantized rows (Q8_0, Q4_0). Lane `sub` of a row's four copies the code bytes of
-// blocks sub, sub+4, ... and, for sub < 3, one 16-byte piece of the scales, to the same
+// Staged quantized rows (Q8_0, Q4_0). Lane `sub` of a row's LPR copies the code bytes of
+// blocks sub, sub+LPR, ... and, for sub < 3, one 16-byte piece of the scales, to the same
 // byte offsets of a staging row; it later dequantizes the same blocks (its own copies,
 // plus the scales its row's lanes copied, once the warp has synchronised).
-template <int FMT>
+template <int FMT, int LPR>
 __device__ __forceinline__ void stage_row_copy(const uint8_t* rowq, uint32_t srow, int sub) {
     constexpr int NB = attn::DQK / kQBlock;
     constexpr int CB = quant_code_bytes(FMT, attn::DQK);
     constexpr int W = FMT == kFmtQ8 ? 2 : 1;
-    for (int m = sub; m < NB; m += 4)
+    for (int m = sub; m < NB; m += LPR)
 #pragma unroll
         for (int h = 0; h < W; ++h) cp_async_16(srow + (m * W + h) * 16, rowq + (m * W + h) * 16, true);
     if (sub < 3) cp_async_16(srow + CB + 16 * sub, rowq + CB + 16 * sub, true);
@@ -344,13 +364,14 @@ __device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
     return v;
 }
 
-template <int FMT>
+// Lane `sub` of the row's LPR: blocks sub, sub+LPR, ... of the staged row into ring row r.
+template <int FMT, int LPR>
 __device__ __forceinline__ void dequant_staged_to_ring(uint32_t srow, bool ok, uint32_t dst, int r,
                                                        int sub) {
     using attn::chunk_addr;
     constexpr int NB = attn::DQK / kQBlock;
     constexpr int CB = quant_code_bytes(FMT, attn::DQK);
-    for (int m = sub; m < NB; m += 4) {
+    for (int m = sub; m < NB; m += LPR) {
         if (!ok) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) st_shared_v4(chunk_addr(dst, r, 4 * m + k), make_uint4(0, 0, 0, 0));
@@ -394,22 +415,25 @@ __device__ __forceinline__ void dequant_row_to_ring(const uint8_t* rowq, bool ok
 // fp32-staged probabilities; KVF the cache format (kFmtF16, or a quantized one whose rows
 // the producers dequantize).
 template <bool PRECISE, bool PSPLIT, int KVF>
-__global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnParams p) {
+__global__ void __launch_bounds__(attn::Roles<KVF>::THREADS, 1) sparse_attn_mma_kernel(AttnParams p) {
     using namespace attn;
     using L = RingLayout<KVF>;
+    using R = Roles<KVF>;
     auto exp2_ = [](float x) { return PRECISE ? exp2f(x) : fast_exp2(x); };
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int kpad = (p.k + 3) / 4 * 4;
-    volatile uint32_t* rowmask = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MASK);
+    // Row validity of each slot: byte w of the slot's MASK_STRIDE holds producer warp w's
+    // rows, row RPW*w + i in bit i (so with eight rows a warp, bit r of the slot's word).
+    volatile uint8_t* rowmask = reinterpret_cast<volatile uint8_t*>(smem + L::OFF_MASK);
     const uint32_t bar0 = sbase + L::OFF_BAR;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (L::NS_ + s); };
 
     if (tid == 0) {
         for (int s = 0; s < L::NS_; ++s) {
-            mbar_init(full_bar(s), PTHREADS + PWARPS);   // noinc copy arrivals + mask writers
+            mbar_init(full_bar(s), R::PT + R::PW);       // noinc copy arrivals + mask writers
             mbar_init(empty_bar(s), GWARPS);             // the owning group's warps
         }
         for (int g = 0; g < GROUPS; ++g) {
@@ -427,8 +451,9 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
     bool abort = false;
     if (warp >= CWARPS) {
         // ================================================================ producers
-        regs_decrease<PRODUCER_REGS>();
+        regs_decrease<R::PREGS>();
         const int ptid = tid - CTHREADS, pw = warp - CWARPS;
+        const int sub = lane & (R::LPR - 1);      // this lane's part of its row
         auto idx_buf = [&](int g, int m) { return L::OFF_IDX + (g * IDX_BUFS + (m & 1)) * kpad * 4; };
         auto stage_idx = [&](int g, int m) {      // top-k row of group g's m-th token
             const int idx = blockIdx.x + (g + GROUPS * m) * gridDim.x;
@@ -436,7 +461,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
             const TokenRows nx = token_rows(p, idx);
             const int32_t* src = p.topk + (size_t)nx.i * p.k;
             const uint32_t dst = sbase + idx_buf(g, m);
-            for (int e = ptid; e < nx.nsel; e += PTHREADS)
+            for (int e = ptid; e < nx.nsel; e += R::PT)
                 asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst + 4 * e),
                              "l"(src + e)
                              : "memory");
@@ -445,7 +470,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
         stage_idx(1, 0);
         cp_async_commit();
         cp_async_wait<0>();
-        named_barrier(PRODUCER_BAR, PTHREADS);
+        named_barrier(PRODUCER_BAR, R::PT);
         // Row r of group g's current unit: a selected compressed row (index checked; with
         // `report`, an out-of-range entry sets the status word) or a window row.
         auto resolve_row = [&](int g, const GroupCursor& cu, int r, long long& src_row, bool& cmp,
@@ -462,7 +487,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                         cmp = true;
                         return true;
                     }
-                    if (report && (lane & 3) == 0) record_status(p.wc.status, kStatusBounds);
+                    if (report && sub == 0) record_status(p.wc.status, kStatusBounds);
                     return false;
                 }
                 if (j >= 0 && j < p.mask_cols) {
@@ -473,7 +498,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                     }
                     return false;
                 }
-                if (j != -1 && report && (lane & 3) == 0) record_status(p.wc.status, kStatusBounds);
+                if (j != -1 && report && sub == 0) record_status(p.wc.status, kStatusBounds);
                 return false;
             }
             if (gr < cu.tr.nrows) {
@@ -491,14 +516,14 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
             if (nx.valid()) {
                 const GroupCursor cn = nx.group(nx.turn);
                 if (cn.u != 0) {
-                    const int r = 8 * pw + (lane >> 2);
+                    const int r = R::RPW * pw + (lane >> R::LPR_LOG2);
                     long long src_row;
                     bool cmp;
                     if (resolve_row(nx.turn, cn, r, src_row, cmp, false)) {
                         const uint8_t* base_q = reinterpret_cast<const uint8_t*>(cmp ? p.kv_cmp : p.kv_raw);
-                        stage_row_copy<KVF == kFmtQ8 ? kFmtQ8 : kFmtQ4>(
+                        stage_row_copy<KVF == kFmtQ8 ? kFmtQ8 : kFmtQ4, R::LPR>(
                             base_q + (size_t)src_row * p.kv_row_bytes, stage_buf(uc + 1) + r * L::QROW,
-                            lane & 3);
+                            sub);
                     }
                 }
             }
@@ -522,9 +547,10 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                     stage_idx(mc.turn, cu.m + 1);
                     const __half* qt = p.q + (size_t)cu.tr.i * H * DQK;
 #pragma unroll
-                    for (int m = 0; m < H * CH / PTHREADS; ++m) {
-                        const int e = ptid + m * PTHREADS, r = e / CH, ch = e % CH;
-                        cp_async_16(chunk_addr(dst, r, ch), qt + r * DQK + ch * 8, true);
+                    for (int m = 0; m < (H * CH + R::PT - 1) / R::PT; ++m) {
+                        const int e = ptid + m * R::PT, r = e / CH, ch = e % CH;
+                        if (H * CH % R::PT == 0 || e < H * CH)
+                            cp_async_16(chunk_addr(dst, r, ch), qt + r * DQK + ch * 8, true);
                     }
                     cp_async_commit();
                     cp_async_arrive_noinc(full_bar(s));
@@ -535,13 +561,13 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                     // thread, before its row units are resolved.
                     cp_async_wait<1>();
                 }
-                named_barrier(PRODUCER_BAR, PTHREADS);
+                named_barrier(PRODUCER_BAR, R::PT);
                 if constexpr (L::STAGED)
                     if (!abort) stage_next(mc, uc);   // the top-k rows it needs are in place
                 continue;
             }
             if (abort) continue;
-            const int r = 8 * pw + (lane >> 2);   // this lane's row of the unit
+            const int r = R::RPW * pw + (lane >> R::LPR_LOG2);   // this lane's row of the unit
             long long src_row = 0;
             bool cmp = false;
             const bool ok = resolve_row(mc.turn, cu, r, src_row, cmp, true);
@@ -551,29 +577,28 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
                 cp_async_wait<0>();
                 __syncwarp();
                 stage_next(mc, uc);
-                dequant_staged_to_ring<KVF>(stage_buf(uc) + r * L::QROW, ok, dst, r, lane & 3);
+                dequant_staged_to_ring<KVF, R::LPR>(stage_buf(uc) + r * L::QROW, ok, dst, r, sub);
                 mbar_arrive(full_bar(s));          // release: this thread's stores are visible
             } else if constexpr (KVF == kFmtF16) {
                 const __half* row = ok ? (cmp ? p.kv_cmp : p.kv_raw) + (size_t)src_row * DQK
                                        : p.kv_raw + (size_t)cu.tr.t * DQK;   // valid stand-in
 #pragma unroll
-                for (int m = 0; m < 18; ++m) {
-                    const int ch = (lane & 3) + 4 * m;
+                for (int m = 0; m < CH / R::LPR; ++m) {
+                    const int ch = sub + R::LPR * m;
                     cp_async_16(chunk_addr(dst, r, ch), row + ch * 8, ok);   // zero-filled if masked
                 }
                 cp_async_arrive_noinc(full_bar(s));
             } else {
                 const uint8_t* base_q = reinterpret_cast<const uint8_t*>(cmp ? p.kv_cmp : p.kv_raw);
-                dequant_row_to_ring<KVF>(base_q + (size_t)src_row * p.kv_row_bytes, ok, dst, r,
-                                         lane & 3);
+                dequant_row_to_ring<KVF>(base_q + (size_t)src_row * p.kv_row_bytes, ok, dst, r, sub);
                 mbar_arrive(full_bar(s));          // release: this thread's stores are visible
             }
-            const uint32_t bits = __ballot_sync(0xffffffffu, ok && (lane & 3) == 0);
+            const uint32_t bits = __ballot_sync(0xffffffffu, ok && sub == 0);
             if (lane == 0) {
                 uint32_t m8 = 0;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) m8 |= ((bits >> (4 * i)) & 1u) << i;
-                reinterpret_cast<volatile uint8_t*>(rowmask + s)[pw] = (uint8_t)m8;
+                for (int i = 0; i < R::RPW; ++i) m8 |= ((bits >> (R::LPR * i)) & 1u) << i;
+                rowmask[L::MASK_STRIDE * s + pw] = (uint8_t)m8;
                 mbar_arrive(full_bar(s));         // release: the mask byte is visible with the slot
             }
             if constexpr (L::STAGED) __syncwarp();   // staging[uc & 1] is read before its reuse
@@ -585,13 +610,13 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
             const long long lo = per * blockIdx.x;
             const long long hi = min(p.prefetch_bytes, lo + per);
             if (lane == 0)
-                for (long long off = lo + (long long)pw * 32768; off < hi; off += PWARPS * 32768LL)
+                for (long long off = lo + (long long)pw * 32768; off < hi; off += R::PW * 32768LL)
                     prefetch_l2(p.prefetch + off, (uint32_t)min(32768LL, hi - off));
         }
         cp_async_wait<0>();
     } else {
         // ================================================================ consumers
-        regs_increase<CONSUMER_REGS>();
+        regs_increase<R::CREGS>();
         const int grp = warp / GWARPS, gw = warp % GWARPS;
         const int gbar = GROUP_BAR + grp;
         uint8_t* garea = smem + L::OFF_GROUP + grp * G_BYTES;
@@ -663,8 +688,17 @@ __global__ void __launch_bounds__(attn::THREADS, 1) sparse_attn_mma_kernel(AttnP
 
             {
                 const float4 u = xbuf[own * 32 + lane];
-                const uint32_t mk = rowmask[q % L::NS_];
-                const bool v0 = (mk >> r0) & 1u, v1 = (mk >> (r0 + 1)) & 1u;
+                bool v0, v1;
+                if constexpr (R::RPW == 8) {
+                    const uint32_t mk =
+                        *reinterpret_cast<const volatile uint32_t*>(rowmask + 4 * (q % L::NS_));
+                    v0 = (mk >> r0) & 1u;
+                    v1 = (mk >> (r0 + 1)) & 1u;
+                } else {
+                    const volatile uint8_t* mb = rowmask + L::MASK_STRIDE * (q % L::NS_);
+                    v0 = (mb[r0 / R::RPW] >> (r0 % R::RPW)) & 1u;
+                    v1 = (mb[(r0 + 1) / R::RPW] >> ((r0 + 1) % R::RPW)) & 1u;
+                }
                 s4[0] = v0 ? (s4[0] + u.x) * p.scale_log2 : -INFINITY;
                 s4[1] = v1 ? (s4[1] + u.y) * p.scale_log2 : -INFINITY;
                 s4[2] = v0 ? (s4[2] + u.z) * p.scale_log2 : -INFINITY;
