@@ -181,7 +181,10 @@ __global__ void __launch_bounds__(THREADS)
 topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int k, int ratio,
                   const uint8_t* __restrict__ vis_mask, long long mask_ld, int mask_cols,
                   int32_t* __restrict__ topk) {
-    extern __shared__ uint32_t keys[];           // [ld]
+    // Keys are handled four at a time (16-byte loads and shared-memory accesses): the
+    // row and the key array are 16-byte aligned and ld is a multiple of 4, so the
+    // n4 = ceil(n/4) groups stay inside both; keys of j >= n are 0 (no candidate).
+    extern __shared__ uint4 keys4[];             // [ld / 4]
     __shared__ uint32_t hist[256];
     __shared__ uint32_t s_digit, s_above;
     __shared__ uint32_t w_or[THREADS / 32], w_and[THREADS / 32], w_cnt[THREADS / 32];
@@ -193,10 +196,15 @@ topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int
     grid_dependents_launch();
     int32_t* out = topk + (size_t)i * k;
     const int tid = threadIdx.x;
-    const float* row = scores + (size_t)i * ld;
+    const float4* row4 = reinterpret_cast<const float4*>(scores + (size_t)i * ld);
     int n;                                       // keys examined: j < n
     int keep = k;                                // slots filled; the rest hold -1
     uint32_t kor = 0u, kand = 0xffffffffu, cand = 0u;   // over this thread's candidates
+    auto take = [&](uint32_t key) {
+        kor |= key;
+        kand &= key;
+        ++cand;
+    };
 
     if (vis_mask == nullptr) {
         n = n_vis(t, ratio);
@@ -204,27 +212,40 @@ topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int
             for (int s = tid; s < k; s += THREADS) out[s] = s < n ? s : -1;
             return;
         }
-        for (int j = tid; j < n; j += THREADS) {
-            const uint32_t key = order_key(row[j]);
-            keys[j] = key;
-            kor |= key;
-            kand &= key;
-            ++cand;
+        const int n4 = (n + 3) / 4;
+        for (int x = tid; x < n4; x += THREADS) {
+            const float4 v = row4[x];
+            const int j = 4 * x;
+            uint4 kk;
+            kk.x = order_key(v.x);
+            kk.y = j + 1 < n ? order_key(v.y) : 0u;
+            kk.z = j + 2 < n ? order_key(v.z) : 0u;
+            kk.w = j + 3 < n ? order_key(v.w) : 0u;
+            keys4[x] = kk;
+            take(kk.x);
+            if (kk.y) take(kk.y);
+            if (kk.z) take(kk.z);
+            if (kk.w) take(kk.w);
         }
     } else {
         n = mask_cols;
         const uint8_t* mrow = vis_mask + (size_t)t * mask_ld;
-        for (int j = tid; j < n; j += THREADS) {
-            const bool v = mrow[j] != 0;
-            const uint32_t key = v ? order_key(row[j]) : 0u;
-            keys[j] = key;
-            if (v) {
-                kor |= key;
-                kand &= key;
-                ++cand;
+        const int n4 = (n + 3) / 4;
+        for (int x = tid; x < n4; x += THREADS) {
+            const float4 v = row4[x];
+            const float f[4] = {v.x, v.y, v.z, v.w};
+            uint32_t kk[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int j = 4 * x + c;
+                const bool vis = j < n && mrow[j] != 0;
+                kk[c] = vis ? order_key(f[c]) : 0u;
+                if (vis) take(kk[c]);
             }
+            keys4[x] = make_uint4(kk[0], kk[1], kk[2], kk[3]);
         }
     }
+    const int n4 = (n + 3) / 4;
     uint32_t all_or, all_and, n_cand;
     block_key_stats<THREADS>(kor, kand, cand, w_or, w_and, w_cnt, all_or, all_and, n_cand, tid,
                              BlockSync{});
@@ -236,10 +257,13 @@ topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int
         RadixSelect<BlockSync> rs(all_or, all_and, (uint32_t)k, tid, BlockSync{});
         while (rs.active) {
             rs.clear(hist, THREADS);
-            for (int j = tid; j < n; j += THREADS) {
-                const uint32_t key = keys[j];
-                if (key != 0u && (key & rs.digits) == rs.prefix)
-                    atomicAdd(&hist[(key >> rs.shift) & 255u], 1u);
+            for (int x = tid; x < n4; x += THREADS) {
+                const uint4 kk = keys4[x];
+                const uint32_t q[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (q[c] != 0u && (q[c] & rs.digits) == rs.prefix)
+                        atomicAdd(&hist[(q[c] >> rs.shift) & 255u], 1u);
             }
             rs.step(hist, &s_digit, &s_above);
         }
@@ -247,25 +271,30 @@ topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int
         need = rs.need;                          // keys == thr to keep, lowest j first
     }
 
-    const int per = (n + THREADS - 1) / THREADS;
-    const int jb = min(n, tid * per), je = min(n, jb + per);
+    // Each thread compacts a contiguous run of key groups, in ascending j.
+    const int per = (n4 + THREADS - 1) / THREADS;
+    const int xb = min(n4, tid * per), xe = min(n4, xb + per);
     uint32_t gt = 0, eq = 0;
-    for (int j = jb; j < je; ++j) {
-        const uint32_t key = keys[j];
-        gt += key > thr;
-        eq += key == thr;
+    for (int x = xb; x < xe; ++x) {
+        const uint4 kk = keys4[x];
+        gt += (kk.x > thr) + (kk.y > thr) + (kk.z > thr) + (kk.w > thr);
+        eq += (kk.x == thr) + (kk.y == thr) + (kk.z == thr) + (kk.w == thr);
     }
     const unsigned long long before =
         block_exclusive_scan<THREADS>(((unsigned long long)gt << 32) | eq, warp_tot, tid, BlockSync{});
     const uint32_t gt_before = (uint32_t)(before >> 32), eq_before = (uint32_t)before;
     uint32_t pos = gt_before + min(eq_before, need), eq_rank = eq_before;
-    for (int j = jb; j < je; ++j) {
-        const uint32_t key = keys[j];
-        if (key > thr) {
-            out[pos++] = j;
-        } else if (key == thr) {
-            if (eq_rank < need) out[pos++] = j;
-            ++eq_rank;
+    for (int x = xb; x < xe; ++x) {
+        const uint4 kk = keys4[x];
+        const uint32_t q[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (q[c] > thr) {
+                out[pos++] = 4 * x + c;
+            } else if (q[c] == thr) {
+                if (eq_rank < need) out[pos++] = 4 * x + c;
+                ++eq_rank;
+            }
         }
     }
     for (int s = keep + tid; s < k; s += THREADS) out[s] = -1;
