@@ -489,7 +489,7 @@ ds4sp_status launch_topk(ds4sp_handle* h, const float* scores, int ld, int t0, i
     const long long mld = h->mask_cols;
     const bool big = ld > 4096;
     if (!h->smem_set[kTopk]) {
-        cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel<256>,
+        cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel<128>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kMaxTopkCandidates * 4 + 64);
         if (e == cudaSuccess)
@@ -517,7 +517,7 @@ ds4sp_status launch_topk(ds4sp_handle* h, const float* scores, int ld, int t0, i
             launch_k(pdl, topk_radix_kernel<1024>, n_q, 1024, smem, stream, scores, ld, t0, n_q, k,
                      ratio, vm, mld, mcols, topk);
         else
-            launch_k(pdl, topk_radix_kernel<256>, n_q, 256, smem, stream, scores, ld, t0, n_q, k,
+            launch_k(pdl, topk_radix_kernel<128>, n_q, 128, smem, stream, scores, ld, t0, n_q, k,
                      ratio, vm, mld, mcols, topk);
     });
 }

@@ -108,45 +108,68 @@ __device__ __forceinline__ void fused_select_row(const uint32_t* keys, int n, in
     uint32_t* s_digit = w_cnt + 2;
     uint32_t* s_above = s_digit + 1;
     unsigned long long* warp_tot = reinterpret_cast<unsigned long long*>(s_above + 1);
+    // Keys four at a time (the row is 16-byte aligned with room to a multiple of 128
+    // keys); j >= n holds stale keys of an earlier unit, read as 0 (no candidate).
+    const int n4 = (n + 3) / 4;
+    auto group = [&](int x) {
+        uint4 kk = reinterpret_cast<const uint4*>(keys)[x];
+        const int j = 4 * x;
+        if (j + 1 >= n) kk.y = 0u;
+        if (j + 2 >= n) kk.z = 0u;
+        if (j + 3 >= n) kk.w = 0u;
+        return kk;
+    };
     uint32_t kor = 0u, kand = 0xffffffffu, cand = 0u;
-    for (int j = tid; j < n; j += NT) {
-        const uint32_t key = keys[j];
-        kor |= key;
-        kand &= key;
-        ++cand;
+    for (int x = tid; x < n4; x += NT) {
+        const uint4 kk = group(x);
+        const uint32_t q[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (q[c]) {
+                kor |= q[c];
+                kand &= q[c];
+                ++cand;
+            }
     }
     uint32_t all_or, all_and, n_cand;
     block_key_stats<NT>(kor, kand, cand, w_or, w_and, w_cnt, all_or, all_and, n_cand, tid, sync);
     RadixSelect<GroupSync> rs(all_or, all_and, (uint32_t)k, tid, sync);
     while (rs.active) {
         rs.clear(hist, NT);
-        for (int j = tid; j < n; j += NT) {
-            const uint32_t key = keys[j];
-            if (key != 0u && (key & rs.digits) == rs.prefix)
-                atomicAdd(&hist[(key >> rs.shift) & 255u], 1u);
+        for (int x = tid; x < n4; x += NT) {
+            const uint4 kk = group(x);
+            const uint32_t q[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (q[c] != 0u && (q[c] & rs.digits) == rs.prefix)
+                    atomicAdd(&hist[(q[c] >> rs.shift) & 255u], 1u);
         }
         rs.step(hist, s_digit, s_above);
     }
     const uint32_t thr = rs.thr, need = rs.need;
-    const int per = (n + NT - 1) / NT;
-    const int jb = min(n, tid * per), je = min(n, jb + per);
+    const int per = (n4 + NT - 1) / NT;
+    const int xb = min(n4, tid * per), xe = min(n4, xb + per);
     uint32_t gt = 0, eq = 0;
-    for (int j = jb; j < je; ++j) {
-        const uint32_t key = keys[j];
-        gt += key > thr;
-        eq += key == thr;
+    for (int x = xb; x < xe; ++x) {
+        const uint4 kk = group(x);
+        gt += (kk.x > thr) + (kk.y > thr) + (kk.z > thr) + (kk.w > thr);
+        eq += (kk.x == thr) + (kk.y == thr) + (kk.z == thr) + (kk.w == thr);
     }
     const unsigned long long before =
         block_exclusive_scan<NT>(((unsigned long long)gt << 32) | eq, warp_tot, tid, sync);
     const uint32_t gt_before = (uint32_t)(before >> 32), eq_before = (uint32_t)before;
     uint32_t pos = gt_before + min(eq_before, need), eq_rank = eq_before;
-    for (int j = jb; j < je; ++j) {
-        const uint32_t key = keys[j];
-        if (key > thr) {
-            out[pos++] = j;
-        } else if (key == thr) {
-            if (eq_rank < need) out[pos++] = j;
-            ++eq_rank;
+    for (int x = xb; x < xe; ++x) {
+        const uint4 kk = group(x);
+        const uint32_t q[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (q[c] > thr) {
+                out[pos++] = 4 * x + c;
+            } else if (q[c] == thr) {
+                if (eq_rank < need) out[pos++] = 4 * x + c;
+                ++eq_rank;
+            }
         }
     }
     // exactly k entries were written (n > k); the scratch is reused by the next row
