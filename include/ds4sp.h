@@ -89,10 +89,11 @@ typedef struct {
                             kernel keeps each token block's scores in shared memory and
                             selects there, so no score reaches global memory. A call takes
                             the fused kernel when no explicit mask is set and a token
-                            block's score rows fit its 64 KB key buffer (256/n_idx_heads
-                            tokens x 128 x ceil(n_vis(last token)/128) x 4 bytes, e.g. up
-                            to 4,096 visible rows at 64 indexer heads) in a call of at most
-                            1,024 token blocks; otherwise the two kernels run. Indices are
+                            block's score rows fit one of its two 40 KB key buffers
+                            (256/n_idx_heads tokens x 128 x ceil(n_vis(last token)/128) x 4
+                            bytes, e.g. up to 2,560 visible rows -- a 10,240-token context
+                            -- at 64 indexer heads) in a call of at most 1,024 token
+                            blocks; otherwise the two kernels run. Indices are
                             the same bits either way. Other values are
                             DS4SP_ERR_INVALID_ARG */
     int kv_format;       /* storage of kv_raw and kv_cmp: 0 = fp16 rows of 576 values

@@ -426,41 +426,54 @@ ds4sp_status launch_fused(ds4sp_handle* h, const void* q_idx, const void* k_idx,
     p.ratio = ratio;
     p.kld = kld;
     // Longest-processing-time assignment of the token blocks to the persistent CTAs: cost
-    // = the block's tiles, plus kSelectCost per token that needs a select (n_vis > k),
-    // in tile-equivalents; blocks go heaviest first to the least loaded CTA.
-    constexpr double kSelectCost = 1.5;
+    // = the block's tiles plus 1.5 tiles per token that needs a select (n_vis > k), kept
+    // in half tiles so that it is an integer; blocks go heaviest first (ties: the later
+    // block first) to the least loaded CTA (ties: the lower CTA). Block costs never fall
+    // with the block index in a launch, so the heaviest-first order is usually the
+    // reverse block order and the sort is skipped.
     const int grid = std::min(n_tb, std::min(h->sm_count, kIndexerMaxGrid));
-    std::vector<std::pair<double, int>> cost(n_tb);
+    struct Item { int cost, tb; };
+    Item items[kFusedMaxBlocks];
+    bool ascending = true;
+    const int t_sel = ratio * (k + 1) - 1;      // tokens t >= t_sel see more than k rows
     for (int tb = 0; tb < n_tb; ++tb) {
         const int tok0 = t0 + tb * C::TB, tok_end = std::min(tok0 + C::TB, t0 + n_q);
         const int tiles = (nvis(tok_end - 1, ratio) + C::BM - 1) / C::BM;
-        int sel = 0;
-        for (int t = tok0; t < tok_end; ++t) sel += nvis(t, ratio) > k;
-        cost[tb] = {tiles + kSelectCost * sel, tb};
+        const int sel = std::max(0, tok_end - std::max(tok0, t_sel));
+        items[tb] = {2 * tiles + 3 * sel, tb};
+        if (tb && items[tb].cost < items[tb - 1].cost) ascending = false;
     }
-    std::sort(cost.begin(), cost.end(), [](const std::pair<double, int>& a, const std::pair<double, int>& b) {
-        return a.first != b.first ? a.first > b.first : a.second > b.second;
-    });
-    std::vector<std::vector<int>> lists(grid);
-    std::vector<std::pair<double, int>> heap;   // (load, cta), min-heap by load then cta
-    for (int c = 0; c < grid; ++c) heap.push_back({0.0, c});
-    auto cmp = [](const std::pair<double, int>& a, const std::pair<double, int>& b) {
-        return a.first != b.first ? a.first > b.first : a.second > b.second;
+    if (ascending)
+        std::reverse(items, items + n_tb);
+    else
+        std::sort(items, items + n_tb, [](const Item& x, const Item& y) {
+            return x.cost != y.cost ? x.cost > y.cost : x.tb > y.tb;
+        });
+    struct Load { long long load; int cta; };
+    Load heap[kIndexerMaxGrid];                 // a min-heap of the CTAs' loads
+    for (int c = 0; c < grid; ++c) heap[c] = {0, c};
+    auto later = [](const Load& x, const Load& y) {
+        return x.load != y.load ? x.load > y.load : x.cta > y.cta;
     };
-    std::make_heap(heap.begin(), heap.end(), cmp);
-    for (const auto& cb : cost) {
-        std::pop_heap(heap.begin(), heap.end(), cmp);
-        auto& top = heap.back();
-        lists[top.second].push_back(cb.second);
-        top.first += cb.first;
-        std::push_heap(heap.begin(), heap.end(), cmp);
+    uint16_t cta_of[kFusedMaxBlocks];
+    int count[kIndexerMaxGrid] = {};
+    for (int u = 0; u < n_tb; ++u) {
+        std::pop_heap(heap, heap + grid, later);
+        Load& top = heap[grid - 1];
+        cta_of[u] = (uint16_t)top.cta;
+        ++count[top.cta];
+        top.load += items[u].cost;
+        std::push_heap(heap, heap + grid, later);
     }
-    int u = 0;
+    int pos[kIndexerMaxGrid];
+    int u_total = 0;
     for (int c = 0; c < grid; ++c) {
-        p.first[c] = (uint16_t)u;
-        for (int tb : lists[c]) p.blk[u++] = (uint16_t)tb;
+        p.first[c] = (uint16_t)u_total;
+        pos[c] = u_total;
+        u_total += count[c];
     }
-    p.first[grid] = (uint16_t)u;
+    p.first[grid] = (uint16_t)u_total;
+    for (int u = 0; u < n_tb; ++u) p.blk[pos[cta_of[u]]++] = (uint16_t)items[u].tb;
     return launch(h, kIndexer, stream, [&] {
         launch_k(h->cfg.dependent_launch != 0, indexer_topk_fused_kernel<D_I, H_I>, grid, C::THREADS,
                  C::SMEM_BYTES, stream, tk, tq, p);

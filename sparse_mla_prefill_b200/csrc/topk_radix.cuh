@@ -39,7 +39,7 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 }
 
 // The select helpers below run on a group of THREADS threads that synchronise through
-// `sync` (the whole block with __syncthreads, or the epilogue warps of the fused indexer
+// `sync` (the whole block with __syncthreads, or a select group of the fused indexer
 // with a named barrier); `tid` is the thread's index inside the group (0 .. THREADS-1),
 // and the group starts on a warp boundary.
 struct BlockSync {
