@@ -138,3 +138,22 @@ def test_quantized_format_limits():
         handle_for(workload("tiny", top_k=1000), kv_format=3)
     assert e.value.status == D.ERR_UNSUPPORTED
     assert D.ds4sp_kv_row_bytes(3, 576) == 912 and D.ds4sp_kv_row_bytes(3, 256) == 0
+
+
+@pytest.mark.parametrize("fmt", [1, 2, 3])
+def test_quantized_cache_few_tokens(fmt):
+    """A call of three tokens (the split attention: one work item per 32-row unit, then
+    the per-token merge) over each quantized cache, against the oracle."""
+    from gpu_common import run_range
+    wl = workload("band")
+    inp = generate(wl)
+    q = 3
+    t0 = wl.T - q
+    dev = _quantized(to_device({n: (v[t0:] if n in ("q", "q_idx", "w") else v)
+                                for n, v in inp.items()}), fmt)
+    with handle_for(wl, kv_format=fmt) as h:
+        topk, out = run_range(h, dev, t0, q, wl.top_k)
+    npi = {k: v.numpy() for k, v in inp.items()}
+    ref = oracle.prefill_tokens_quant(npi, range(t0, wl.T), wl.top_k, wl.n_swa, fmt)
+    assert np.array_equal(topk.cpu().numpy(), ref["topk"])
+    assert_attention_close(out.cpu().numpy(), ref["out"], f"few tokens kv_format {fmt}")
