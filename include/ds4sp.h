@@ -122,8 +122,11 @@ typedef struct {
                             through a 5-slot ring, default); 1 = logits on the tcgen05
                             tensor cores: units of 128 gathered rows as the MMA's M and the
                             16 heads as its N, S = R . Q^T accumulated in TMEM, softmax from
-                            TMEM, P . V on mma.sync (SURVEY's "KV rows as M = 128, heads as
-                            N = 16" form). 1 needs kv_format 0, exp_mode 0 and pv_mode 0
+                            TMEM, P . V on mma.sync (an alternative to the streaming
+                            form, as the pages time a grouped path against the streaming
+                            one: "perf(ds4): unify gfx1151 sparse-prefill stack",
+                            Validation completed). 1 needs kv_format 0, exp_mode 0 and
+                            pv_mode 0
                             (else DS4SP_ERR_UNSUPPORTED) and does not take the few-token
                             split. Other values are DS4SP_ERR_INVALID_ARG */
 } ds4sp_config;
