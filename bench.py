@@ -607,6 +607,7 @@ def run_ours(args, rank, world, local_rank):
 VARIANTS = [
     ("plain_stream_order", dict(dependent_launch=0)),
     ("fused_indexer_topk", dict(topk_mode=1)),
+    ("indexer_cta_pairs", dict(indexer_kernel=1)),
     ("tcgen05_logits", dict(attn_kernel=1)),
     ("exp2f_softmax", dict(exp_mode=1)),
     ("fp32_staged_pv", dict(pv_mode=1)),

@@ -126,9 +126,15 @@ typedef struct {
                             form, as the pages time a grouped path against the streaming
                             one: "perf(ds4): unify gfx1151 sparse-prefill stack",
                             Validation completed). 1 needs kv_format 0, exp_mode 0 and
-                            pv_mode 0
-                            (else DS4SP_ERR_UNSUPPORTED) and does not take the few-token
-                            split. Other values are DS4SP_ERR_INVALID_ARG */
+                            pv_mode 0 (else DS4SP_ERR_UNSUPPORTED) and does not take the
+                            few-token split. Other values are DS4SP_ERR_INVALID_ARG */
+    int indexer_kernel;  /* step 1's kernel in the two-kernel form (topk_mode 0, or a call
+                            the fused kernel does not take): 0 = one CTA per tile, each
+                            tcgen05 MMA 128 rows x 256 (token, head) columns; 1 = CTA pairs
+                            (2-CTA clusters): each MMA 256 rows x 256 columns shared by the
+                            pair (cta_group::2), CTA r holding the rows of its j-tile and
+                            columns 128r .. 128r+127 of the q_idx block. The same scores
+                            either way. Other values are DS4SP_ERR_INVALID_ARG */
 } ds4sp_config;
 
 /* Validate cfg and create a handle bound to the current CUDA device. The handle owns

@@ -20,6 +20,7 @@
 #include "ds4sp.h"
 #include "indexer_tcgen05.cuh"
 #include "indexer_topk_fused.cuh"
+#include "indexer_pair.cuh"
 #include "probe_gather.cuh"
 #include "sparse_attn_mma.cuh"
 #include "sparse_attn_tc.cuh"
@@ -141,8 +142,10 @@ ds4sp_status set_smem_once(ds4sp_handle* h, const void* fn, int bytes, int slot,
 constexpr int indexer_slot(int d_idx, int h_idx) {
     return (d_idx == 128 ? 5 : 0) + (h_idx == 4 ? 0 : h_idx == 8 ? 1 : h_idx == 16 ? 2 : h_idx == 32 ? 3 : 4);
 }
-// Slots 0-9: indexer_tcgen05_kernel; 10-19 (tables of 32): the fused kernel.
+// Slots 0-9: indexer_tcgen05_kernel; 10-19 (tables of 32): the fused kernel; 20-29: the
+// CTA-pair indexer.
 constexpr int fused_slot(int d_idx, int h_idx) { return 10 + indexer_slot(d_idx, h_idx); }
+constexpr int pair_slot(int d_idx, int h_idx) { return 20 + indexer_slot(d_idx, h_idx); }
 
 int score_ld(int t_last, int ratio) {
     const int nv = nvis(t_last, ratio);
@@ -378,10 +381,99 @@ ds4sp_status launch_indexer(ds4sp_handle* h, const void* q_idx, const void* k_id
     });
 }
 
+// The CTA-pair indexer (indexer_pair_kernel): items are (token block, pair of j-tiles),
+// cut into contiguous shares of about equal cost, one per pair of CTAs (a 2-CTA cluster).
+template <int D_I, int H_I>
+ds4sp_status launch_indexer_pair(ds4sp_handle* h, const void* q_idx, const void* k_idx,
+                                 const float* w, int t0, int n_q, float* scores, int ld,
+                                 cudaStream_t stream) {
+    using C = PairTile<D_I, H_I>;
+    const int ratio = h->cfg.ratio;
+    const int n_rows = nvis(t0 + n_q - 1, ratio);
+    if (n_rows == 0) return DS4SP_OK;
+    CUtensorMap tk, tq;
+    if (!make_tmap_2d(&tk, k_idx, D_I, n_rows, C::BM) ||
+        !make_tmap_2d(&tq, q_idx, D_I, n_q * H_I, C::BN_HALF))
+        return fail(DS4SP_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    DS4SP_TRY(set_smem_once(h, reinterpret_cast<const void*>(indexer_pair_kernel<D_I, H_I>),
+                            C::SMEM_BYTES, pair_slot(D_I, H_I), "cudaFuncSetAttribute(indexer pairs)"));
+    IndexerParams p;
+    p.w = w;
+    p.scores = scores;
+    p.wc = next_wait(h);
+    p.t0 = t0;
+    p.n_q = n_q;
+    p.ld = ld;
+    p.ratio = ratio;
+    p.n_tb = (n_q + C::TB - 1) / C::TB;
+    auto block_items = [&](int tb) {
+        const int tiles = (nvis(t0 + std::min((tb + 1) * C::TB, n_q) - 1, ratio) + C::BM - 1) / C::BM;
+        return (tiles + 1) / 2;
+    };
+    long long items = 0;
+    for (int tb = 0; tb < p.n_tb; ++tb) items += block_items(tb);
+    if (items == 0) return DS4SP_OK;
+    const int pairs = (int)std::min<long long>(items, std::min(h->sm_count / 2, kIndexerMaxGrid));
+    if (items > (1 << 30) || p.n_tb > 65535 || (items + p.n_tb) / pairs + 2 > 65535)
+        return fail(DS4SP_ERR_UNSUPPORTED, "indexer launch of %lld tile pairs", items);
+    {
+        // Contiguous shares of about equal cost: one per item, plus kLoadCost for the first
+        // item of each token block (its q_idx load). Every share gets at least one item.
+        constexpr double kLoadCost = 1.0;
+        const double total_cost = (double)items + kLoadCost * p.n_tb;
+        int b = 0, tb = 0, jp = 0, nb = block_items(0);
+        long long left = items;
+        double cost = 0.0;
+        p.start_tb[0] = 0;
+        p.start_jt[0] = 0;
+        int count = 0;
+        while (left > 0) {
+            while (jp >= nb) {
+                ++tb;
+                jp = 0;
+                nb = block_items(tb);
+            }
+            cost += 1.0 + (jp == 0 ? kLoadCost : 0.0);
+            ++count;
+            ++jp;
+            --left;
+            const double target = total_cost * (b + 1) / pairs;
+            if (b + 1 < pairs && (cost >= target || left == pairs - 1 - b)) {
+                p.count[b] = (uint16_t)count;
+                ++b;
+                count = 0;
+                while (jp >= nb && left > 0) {
+                    ++tb;
+                    jp = 0;
+                    nb = block_items(tb);
+                }
+                p.start_tb[b] = (uint16_t)tb;
+                p.start_jt[b] = (uint16_t)jp;
+            }
+        }
+        p.count[b] = (uint16_t)count;
+        if (b != pairs - 1) return fail(DS4SP_ERR_CUDA, "indexer partition: %d of %d shares", b + 1, pairs);
+    }
+    return launch(h, kIndexer, stream, [&] {
+        launch_k_cluster(h->cfg.dependent_launch != 0, 2, indexer_pair_kernel<D_I, H_I>, 2 * pairs,
+                         C::THREADS, C::SMEM_BYTES, stream, tk, tq, p);
+    });
+}
+
 template <int D_I>
 ds4sp_status dispatch_indexer_h(ds4sp_handle* h, const void* q_idx, const void* k_idx,
                                 const float* w, int t0, int n_q, float* scores, int ld,
                                 cudaStream_t s) {
+    if (h->cfg.indexer_kernel == 1) {
+        switch (h->cfg.n_idx_heads) {
+            case 4: return launch_indexer_pair<D_I, 4>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
+            case 8: return launch_indexer_pair<D_I, 8>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
+            case 16: return launch_indexer_pair<D_I, 16>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
+            case 32: return launch_indexer_pair<D_I, 32>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
+            case 64: return launch_indexer_pair<D_I, 64>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
+        }
+        return fail(DS4SP_ERR_UNSUPPORTED, "n_idx_heads %d", h->cfg.n_idx_heads);
+    }
     switch (h->cfg.n_idx_heads) {
         case 4: return launch_indexer<D_I, 4>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
         case 8: return launch_indexer<D_I, 8>(h, q_idx, k_idx, w, t0, n_q, scores, ld, s);
@@ -798,6 +890,9 @@ ds4sp_status ds4sp_create(const ds4sp_config* cfg, ds4sp_handle** out) {
     if (c.attn_kernel != 0 && c.attn_kernel != 1)
         return fail(DS4SP_ERR_INVALID_ARG, "attn_kernel %d (0 = mma.sync streaming, 1 = tcgen05 logits)",
                     c.attn_kernel);
+    if (c.indexer_kernel != 0 && c.indexer_kernel != 1)
+        return fail(DS4SP_ERR_INVALID_ARG, "indexer_kernel %d (0 = one CTA per tile, 1 = CTA pairs)",
+                    c.indexer_kernel);
     if (c.attn_kernel == 1 && (c.kv_format != 0 || c.exp_mode != 0 || c.pv_mode != 0))
         return fail(DS4SP_ERR_UNSUPPORTED, "attn_kernel 1 runs fp16 rows with exp_mode 0 and pv_mode 0");
     if (c.dependent_launch != 0 && c.dependent_launch != 1)
@@ -1301,6 +1396,8 @@ ds4sp_status check_static_config(const ds4sp_config* cfg) {
     if (c.top_k < 0 || c.top_k > attn::MAX_TOPK || c.max_tokens < 1 || c.max_tokens > (1 << 24))
         return fail(DS4SP_ERR_INVALID_ARG, "0 <= top_k <= %d and 1 <= max_tokens <= 2^24 required",
                     attn::MAX_TOPK);
+    if (c.indexer_kernel != 0 && c.indexer_kernel != 1)
+        return fail(DS4SP_ERR_INVALID_ARG, "indexer_kernel %d (0 or 1)", c.indexer_kernel);
     return DS4SP_OK;
 }
 

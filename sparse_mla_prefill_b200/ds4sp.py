@@ -34,7 +34,8 @@ class ds4sp_config(ctypes.Structure):
                 ("max_tokens", ctypes.c_int), ("softmax_scale", ctypes.c_float),
                 ("exp_mode", ctypes.c_int), ("pv_mode", ctypes.c_int),
                 ("topk_mode", ctypes.c_int), ("kv_format", ctypes.c_int),
-                ("dependent_launch", ctypes.c_int), ("attn_kernel", ctypes.c_int)]
+                ("dependent_launch", ctypes.c_int), ("attn_kernel", ctypes.c_int),
+                ("indexer_kernel", ctypes.c_int)]
 
 
 class ds4sp_io(ctypes.Structure):
@@ -157,17 +158,19 @@ def make_config(n_idx_heads: int, d_idx: int, top_k: int, n_swa: int, max_tokens
                 band: int = 2048, softmax_scale: float = 0.0, n_heads: int = 16, d_qk: int = 576,
                 d_v: int = 512, ratio: int = 4, exp_mode: int = 0,
                 pv_mode: int = 0, topk_mode: int = 0, kv_format: int = 0,
-                dependent_launch: int = 1, attn_kernel: int = 0) -> ds4sp_config:
+                dependent_launch: int = 1, attn_kernel: int = 0,
+                indexer_kernel: int = 0) -> ds4sp_config:
     """A ds4sp_config in field order. exp_mode: 0 = ex2.approx, 1 = exp2f for the
     softmax; pv_mode: 0 = fp16 probabilities in P . V, 1 = fp32-staged (hi + lo fp16);
     topk_mode: 0 = scores in the workspace and a separate top-k kernel, 1 = fused
     indexer + top-k where the call qualifies; kv_format: 0 = fp16 KV rows, 1 = Q8_0,
     2 = Q4_0, 3 = Q8 K / Q4 V quantized rows (ds4sp_quantize_kv); dependent_launch:
     1 = each kernel a programmatic dependent of the one before it, 0 = plain order;
-    attn_kernel: 0 = mma.sync streaming attention, 1 = logits on tcgen05 (TMEM)."""
+    attn_kernel: 0 = mma.sync streaming attention, 1 = logits on tcgen05 (TMEM);
+    indexer_kernel: 0 = one CTA per tcgen05 tile, 1 = CTA pairs sharing each MMA."""
     return ds4sp_config(n_heads, d_qk, d_v, ratio, n_idx_heads, d_idx, top_k, n_swa, band,
                         max_tokens, softmax_scale, exp_mode, pv_mode, topk_mode, kv_format,
-                        dependent_launch, attn_kernel)
+                        dependent_launch, attn_kernel, indexer_kernel)
 
 
 def ds4sp_create(cfg: ds4sp_config) -> Handle:

@@ -64,6 +64,7 @@ def _cfg(**kw):
     (dict(kv_format=3, top_k=900), D.ERR_UNSUPPORTED),
     (dict(dependent_launch=2), D.ERR_INVALID_ARG),
     (dict(attn_kernel=2), D.ERR_INVALID_ARG),
+    (dict(indexer_kernel=2), D.ERR_INVALID_ARG),
     (dict(attn_kernel=1, kv_format=2), D.ERR_UNSUPPORTED),
 ])
 def test_create_rejects_bad_config_before_touching_the_device(lib, kw, status):

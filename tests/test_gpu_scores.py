@@ -7,7 +7,8 @@ whatever the summation order; each defined column j < n_vis(t) of every token mu
 have the bits of oracle.indexer_scores_token_exact (int64 arithmetic) converted to
 fp32. Columns j >= n_vis(t) are not defined and are not read. (The handles here use
 topk_mode 0, the path that writes the scores; the fused path keeps them on chip and is
-checked through its indices in test_gpu_fused_topk.py.)
+checked through its indices in test_gpu_fused_topk.py.) Both indexer kernels are run:
+one CTA per tcgen05 tile (indexer_kernel 0) and CTA pairs sharing each MMA (1).
 """
 import numpy as np
 import pytest
@@ -56,22 +57,46 @@ def _check_rows(scores, inp, t0, n_q):
                                  f"got {got[bad[0]]} want {want[bad[0]]}")
 
 
+def _check_rows_sampled(scores, inp, t0, toks):
+    for t in toks:
+        i = t - t0
+        _check_rows(scores[i:i + 1], {"q_idx": inp["q_idx"][i:i + 1], "k_idx": inp["k_idx"],
+                                      "w": inp["w"][i:i + 1]}, t, 1)
+
+
+@pytest.mark.parametrize("indexer_kernel", [0, 1])
 @pytest.mark.parametrize("name", ["tiny", "band"])
-def test_scores_every_token(name):
+def test_scores_every_token(name, indexer_kernel):
     """Every token of the 256-token (4 x 64 indexer) and 2048-token (64 x 128) workloads."""
     wl = workload(name)
     inp = generate(wl)
-    with handle_for(wl, topk_mode=0) as h:
+    with handle_for(wl, topk_mode=0, indexer_kernel=indexer_kernel) as h:
         scores = _scores_of_call(h, to_device(inp), 0, wl.T, wl.top_k)
     _check_rows(scores, inp, 0, wl.T)
 
 
+@pytest.mark.parametrize("indexer_kernel", [0, 1])
 @pytest.mark.parametrize("q", [1, 5])
-def test_scores_verify_width(q):
+def test_scores_verify_width(q, indexer_kernel):
     """The last q tokens of the 122,880-token context: rows of up to 30,720 scores."""
     wl = workload("verify")
     inp = generate(wl)                     # per-token tensors of the last 5 positions
     sl = {k: (v[5 - q:].contiguous() if k in ("q", "q_idx", "w") else v) for k, v in inp.items()}
-    with handle_for(wl, topk_mode=0) as h:
+    with handle_for(wl, topk_mode=0, indexer_kernel=indexer_kernel) as h:
         scores = _scores_of_call(h, to_device(sl), wl.T - q, q, wl.top_k)
     _check_rows(scores, sl, wl.T - q, q)
+
+
+@pytest.mark.parametrize("indexer_kernel", [0, 1])
+def test_scores_10k_last_band_sampled(indexer_kernel):
+    """The last band of the 10K prefill (rows of 2,048-2,560 scores): 48 tokens, among
+    them the band's first and last and both ends of a token block."""
+    wl = workload("10k")
+    inp = generate(wl)
+    t0, n = 8192, 2048
+    sl = {k: (v[t0:t0 + n].contiguous() if k in ("q", "q_idx", "w") else v) for k, v in inp.items()}
+    with handle_for(wl, topk_mode=0, indexer_kernel=indexer_kernel) as h:
+        scores = _scores_of_call(h, to_device(sl), t0, n, wl.top_k)
+    rng = np.random.default_rng(5)
+    toks = sorted({t0, t0 + 3, t0 + 4, t0 + n - 1, *rng.integers(t0, t0 + n, 44).tolist()})
+    _check_rows_sampled(scores, sl, t0, toks)
