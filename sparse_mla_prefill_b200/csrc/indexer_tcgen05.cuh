@@ -15,10 +15,12 @@
 // order. Persistent CTAs (one per SM) each take a contiguous share of about equal cost
 // (a tile, plus the q_idx load of each token block it starts) and process it as one
 // unit per token block it touches.
-// Warp roles (352 threads): warp 10 loads q_idx blocks into two B buffers, up to two
+// Warp roles (384 threads): warp 10 loads q_idx blocks into two B buffers, up to two
 // units ahead; warp 0 streams whole k_idx tiles (one 64-dim TMA box per K sub-tile)
 // into a ring of two (D_i = 128) or four (D_i = 64) stages;
-// warp 1 owns TMEM and issues the MMAs; warps 2-9 run the epilogue (ReLU, head
+// warp 1 owns TMEM and issues the MMAs of even tiles, warp 11 those of odd tiles (so
+// that one issuer's barrier waits, fences and commit between tiles overlap the other's
+// MMAs, which a single issuer left as gaps in the tensor pipe); warps 2-9 run the epilogue (ReLU, head
 // weights, sum, store), two warps per TMEM lane quarter, each on half of the columns,
 // the second 64 of its columns loading from TMEM while the first 64 are reduced.
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i overlap the MMAs
@@ -45,7 +47,8 @@ struct IndexerTile {
     static constexpr int A_STAGES = KSUB == 2 ? 2 : 4;
     static constexpr int EPI_WARPS = 8;
     static constexpr int B_WARP = 2 + EPI_WARPS;                      // q_idx loader
-    static constexpr int THREADS = (3 + EPI_WARPS) * 32;
+    static constexpr int MMA2_WARP = 3 + EPI_WARPS;                   // MMAs of odd tiles
+    static constexpr int THREADS = (4 + EPI_WARPS) * 32;
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int OFF_B = 0;                                   // two B buffers
     static constexpr int OFF_A = 2 * B_BYTES;
@@ -216,10 +219,10 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bfull(i), 1);
-            mbar_init(bempty(i), 1);
+            mbar_init(bempty(i), 2);              // both MMA issuers, once per unit
             mbar_init(tempty(i), C::EPI_WARPS);   // one arrive per epilogue warp
         }
-        mbar_init(done_bar, 1);
+        mbar_init(done_bar, 2);
         fence_mbar_init();
         prefetch_tmap(&tmap_k);
         prefetch_tmap(&tmap_q);
@@ -285,9 +288,14 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 if (a_issued[s]) mbar_wait_drain(afull(s), (a_issued[s] - 1) & 1, p.wc);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == C::MMA2_WARP) {
+        // ------------------------------------------------------------ MMA issuers
+        // Two threads issue the MMAs, warp 1 those of even tiles and the last warp those
+        // of odd tiles (each on its own accumulator buffer): while one waits on its next
+        // tile's barriers, fences and commits, the other's MMAs keep the tensor pipe's
+        // short queue filled.
         if (lane == 0) {
+            const int par = warp == 1 ? 0 : 1;
             // Descriptors differ only in their start-address field (address >> 4 in the low
             // 14 bits), so each stage's is built once and offset per K step.
             const uint64_t a_desc0 = umma_desc_sw128(base + C::OFF_A);
@@ -300,6 +308,7 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 if (!mbar_wait(bfull(bb), (bi >> 1) & 1, p.wc, abort)) break;
                 const uint64_t b_desc = b_desc0 + (uint64_t)((bb * C::B_BYTES) >> 4);
                 for (int it = 0; it < w.n_tiles; ++it, ++tc) {
+                    if ((tc & 1) != par) continue;       // the other issuer's tile
                     const int buf = tc & 1, s = tc % C::A_STAGES;
                     if (!mbar_wait(tempty(buf), ((tc >> 1) & 1) ^ 1, p.wc, abort)) break;
                     if (!mbar_wait(afull(s), (tc / C::A_STAGES) & 1, p.wc, abort)) break;
@@ -317,10 +326,11 @@ indexer_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     // accumulator of this tile is complete.
                     umma_commit(aempty(s));
                 }
-                umma_commit(bempty(bb));                 // B buffer free once the unit's MMAs finish
+                // B buffer free once both issuers' MMAs of the unit finish
+                umma_commit(bempty(bb));
                 ++bi;
             }
-            // All MMAs issued by this thread must finish before TMEM is released (a
+            // All MMAs issued by both threads must finish before TMEM is released (a
             // drain wait: committed MMAs complete on their own).
             umma_commit(done_bar);
             mbar_wait_drain(done_bar, 0, p.wc);
