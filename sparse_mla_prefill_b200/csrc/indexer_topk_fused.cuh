@@ -41,7 +41,8 @@ struct FusedTile {
     using T = IndexerTile<D_I, H_I>;
     static constexpr int BM = T::BM, BN = T::BN, TB = T::TB, KSUB = T::KSUB;
     static constexpr int A_SUB = T::A_SUB, A_STAGE = T::A_STAGE, B_SUB = T::B_SUB;
-    static constexpr int B_BYTES = T::B_BYTES, A_STAGES = T::A_STAGES;
+    static constexpr int B_BYTES = T::B_BYTES;
+    static constexpr int A_STAGES = KSUB == 2 ? 2 : 4;           // k_idx ring
     static constexpr int A_WARP = 0, MMA_WARP = 1, B_WARP = 2;
     static constexpr int EPI_WARP0 = 4, EPI_WARPS = 8, EPI_THREADS = EPI_WARPS * 32;
     static constexpr int SEL_WARP0 = 12, SEL_WARPS = 8, SEL_ALL = SEL_WARPS * 32;
