@@ -67,6 +67,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The same test without suspending: returns at once. A polling loop of it sees a phase
+// complete sooner than try_wait, which may suspend the thread for a system-dependent
+// time, at the cost of issue slots.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // How the pipeline waits of one launch give up. `abort_word` is shared by every launch
 // of a handle; a wait that gives up writes this launch's `epoch` (never 0, new for
 // every launch) into it, and a wait of the same launch that sees its own epoch there
@@ -92,11 +107,14 @@ __device__ __forceinline__ void give_up(const WaitCtl& w) {
 // Wait for the phase of the given parity to complete. Gives up (returns false, records
 // kStatusTimeout and sets `abort`) once w.limit_ns has passed since the first miss, or
 // as soon as another wait of the same launch has given up. Once `abort` is set it
-// returns false at once, so every role drains quickly.
+// returns false at once, so every role drains quickly. kPoll: test with test_wait
+// instead of try_wait (the attention ring measured faster polling; the indexer the same).
+template <bool kPoll = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& w,
                                           bool& abort) {
+    auto test = [&] { return kPoll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity); };
     if (abort) return false;
-    if (mbar_try_wait(bar, parity)) return true;
+    if (test()) return true;
     const unsigned long long t0 = global_ns();
     while (true) {
         if (launch_gave_up(w) || global_ns() - t0 >= w.limit_ns) {
@@ -105,7 +123,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
             return false;
         }
         for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+            if (test()) return true;
     }
 }
 

@@ -537,7 +537,7 @@ __global__ void __launch_bounds__(attn::Roles<KVF>::THREADS, 1) sparse_attn_mma_
         for (int uc = 0; mc.valid(); ++uc, mc.advance(p)) {
             const int s = uc % L::NS_;
             if (!abort &&
-                !__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ((uc / L::NS_) & 1) ^ 1, p.wc, abort)))
+                !__all_sync(0xffffffffu, mbar_wait<true>(empty_bar(s), ((uc / L::NS_) & 1) ^ 1, p.wc, abort)))
                 abort = true;                      // the whole warp gives up together
             const uint32_t dst = sbase + L::OFF_RING + s * L::SLOT_;
             const GroupCursor cu = mc.group(mc.turn);
@@ -638,7 +638,7 @@ __global__ void __launch_bounds__(attn::Roles<KVF>::THREADS, 1) sparse_attn_mma_
         float m_g = -INFINITY, m_g8 = -INFINITY; // reference max, heads g and g+8 (log2 units)
         float l_g = 0.f, l_g8 = 0.f;             // this warp's share of the softmax sums
         auto wait_full = [&](int q) {
-            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(q % L::NS_), (q / L::NS_) & 1, p.wc, abort)))
+            if (!__all_sync(0xffffffffu, mbar_wait<true>(full_bar(q % L::NS_), (q / L::NS_) & 1, p.wc, abort)))
                 flags[2] = 1;
         };
         MergedCursor mc;
