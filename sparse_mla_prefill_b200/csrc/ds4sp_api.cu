@@ -725,9 +725,9 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
         // persistent: one CTA per SM, each walking its share of the work items
         const int grid = std::min(p.n_items, h->sm_count);
         const dim3 g(grid), b(attn::Roles<kFmtF16>::THREADS);
-        const dim3 bs(attn::Roles<kFmtQ8>::THREADS);   // the staged formats' eight producer warps
+        const dim3 bs(attn::Roles<kFmtQ8>::THREADS);   // the quantized formats' eight producer warps
         static_assert(attn::Roles<kFmtQ8>::THREADS == attn::Roles<kFmtQ4>::THREADS &&
-                          attn::Roles<kFmtQ8Q4>::THREADS == attn::Roles<kFmtF16>::THREADS,
+                          attn::Roles<kFmtQ8Q4>::THREADS == attn::Roles<kFmtQ8>::THREADS,
                       "block shapes per format");
         const bool pdl = h->cfg.dependent_launch != 0;
         if (tc) {
@@ -737,7 +737,7 @@ ds4sp_status launch_attn(ds4sp_handle* h, const void* q, const void* kv_raw, con
         } else if (h->cfg.kv_format == kFmtQ4) {
             launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ4>, g, bs, smem, stream, p);
         } else if (h->cfg.kv_format == kFmtQ8Q4) {
-            launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ8Q4>, g, b, smem, stream, p);
+            launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtQ8Q4>, g, bs, smem, stream, p);
         } else {
             switch (2 * h->cfg.pv_mode + h->cfg.exp_mode) {
                 case 0: launch_k(pdl, sparse_attn_mma_kernel<false, false, kFmtF16>, g, b, smem, stream, p); break;

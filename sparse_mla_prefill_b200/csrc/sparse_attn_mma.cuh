@@ -17,8 +17,8 @@
 // tensor-core work. The two groups' unit sequences are merged, one unit of each in
 // turn, into one stream through a 5-slot shared-memory ring with an mbarrier pair
 // per slot; producers and both groups walk the same merged order.
-//   * Warps 8-11 produce (8-15 for the staged Q8_0 / Q4_0 caches, whose dequantization
-//     needs the extra warps). They stage each token's top-k row in shared memory one
+//   * Warps 8-11 produce (8-15 for the quantized caches, whose dequantization needs the
+//     extra warps). They stage each token's top-k row in shared memory one
 //     token ahead per group, resolve and check every row, and copy it in 16-byte chunks
 //     with cp.async; cp.async.mbarrier.arrive.noinc lets the slot's barrier count the
 //     copies without the producer waiting for them. Each producer warp also publishes
@@ -101,9 +101,9 @@ struct RingLayout {
     static constexpr int STAGE = BR * QROW;                 // one staging buffer
     static constexpr int OFF_RING = 0;
     static constexpr int OFF_GROUP = OFF_RING + NS_ * SLOT_;
-    // Row-validity bytes per slot: one per producer warp (four, or eight for the staged
-    // formats' eight producer warps).
-    static constexpr int MASK_STRIDE = STAGED ? 8 : 4;
+    // Row-validity bytes per slot: one per producer warp (four, or eight for the
+    // quantized formats' eight producer warps).
+    static constexpr int MASK_STRIDE = STAGED || SPLIT ? 8 : 4;
     static constexpr int OFF_MASK = OFF_GROUP + GROUPS * G_BYTES;
     static constexpr int OFF_BAR = OFF_MASK + 8 * MASK_STRIDE;      // full[NS_], empty[NS_]
     static constexpr int OFF_STAGE = OFF_BAR + 2 * NS_ * 8;
@@ -128,7 +128,8 @@ __host__ __device__ constexpr int smem_bytes(int k) { return RingLayout<kFmtF16>
 // 200 / 56 at 512.
 template <int KVF>
 struct Roles {
-    static constexpr int PW = RingLayout<KVF>::STAGED ? 8 : 4;   // producer warps
+    // producer warps: eight for the quantized formats, whose producers dequantize
+    static constexpr int PW = RingLayout<KVF>::STAGED || RingLayout<KVF>::SPLIT ? 8 : 4;
     static constexpr int PT = PW * 32;
     static constexpr int THREADS = CTHREADS + PT;
     static constexpr int RPW = BR / PW;          // rows per producer warp
@@ -283,10 +284,11 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
 }
 
 // Producer side of a quantized cache: this lane's blocks of one stored row part (lane l
-// of the row's four takes blocks l, l+4, l+8, ...), loaded as 16-byte words, dequantized
-// to fp16 and stored as four 16-byte chunks per block into ring row r of `pitch` bytes
-// from `base`; a masked row stores zeros. FMT is Q8_0 or Q4_0 and NB the part's blocks.
-template <int FMT, int NB>
+// of the row's LPR takes blocks l, l+LPR, l+2*LPR, ...), loaded as 16-byte words,
+// dequantized to fp16 and stored as four 16-byte chunks per block into ring row r of
+// `pitch` bytes from `base`; a masked row stores zeros. FMT is Q8_0 or Q4_0 and NB the
+// part's blocks.
+template <int FMT, int NB, int LPR>
 __device__ __forceinline__ void dequant_part_to_ring(const uint8_t* rowq, bool ok, uint32_t base,
                                                      int pitch, int r, int sub) {
     using attn::chunk_addr_p;
@@ -294,17 +296,17 @@ __device__ __forceinline__ void dequant_part_to_ring(const uint8_t* rowq, bool o
     constexpr int W = FMT == kFmtQ8 ? 2 : 1;             // 16-byte words per block
     constexpr int BATCH = FMT == kFmtQ8 ? 2 : 3;         // blocks whose loads fly together
     if (!ok) {
-        for (int m = sub; m < NB; m += 4)
+        for (int m = sub; m < NB; m += LPR)
 #pragma unroll
             for (int k = 0; k < 4; ++k) st_shared_v4(chunk_addr_p(base, r, 4 * m + k, pitch), make_uint4(0, 0, 0, 0));
         return;
     }
-    for (int m0 = sub; m0 < NB; m0 += 4 * BATCH) {
+    for (int m0 = sub; m0 < NB; m0 += LPR * BATCH) {
         uint4 c[BATCH][W];
         __half2 d2[BATCH];
 #pragma unroll
         for (int i = 0; i < BATCH; ++i) {
-            const int m = m0 + 4 * i;
+            const int m = m0 + LPR * i;
             if (m < NB) {
                 const uint4* src = reinterpret_cast<const uint4*>(rowq + m * 16 * W);
 #pragma unroll
@@ -314,7 +316,7 @@ __device__ __forceinline__ void dequant_part_to_ring(const uint8_t* rowq, bool o
         }
 #pragma unroll
         for (int i = 0; i < BATCH; ++i) {
-            const int m = m0 + 4 * i;
+            const int m = m0 + LPR * i;
             if (m >= NB) continue;
             if constexpr (FMT == kFmtQ8) {
                 st_shared_v4(chunk_addr_p(base, r, 4 * m + 0, pitch), dequant_q8_chunk(c[i][0].x, c[i][0].y, d2[i]));
@@ -396,18 +398,19 @@ __device__ __forceinline__ void dequant_staged_to_ring(uint32_t srow, bool ok, u
     }
 }
 
-// A stored row of the cache format into ring row r of the slot at `dst`.
-template <int KVF>
+// A stored row of the cache format into ring row r of the slot at `dst` (this lane's
+// blocks: lane `sub` of the row's LPR).
+template <int KVF, int LPR>
 __device__ __forceinline__ void dequant_row_to_ring(const uint8_t* rowq, bool ok, uint32_t dst,
                                                     int r, int sub) {
     using namespace attn;
     constexpr int NB = DQK / kQBlock;                        // 18 key blocks
     if constexpr (KVF == kFmtQ8Q4) {
-        dequant_part_to_ring<kFmtQ8, NB>(rowq, ok, dst, ROW, r, sub);
-        dequant_part_to_ring<kFmtQ4, DV / kQBlock>(rowq + quant_row_bytes(kFmtQ8, DQK), ok,
-                                                   dst + RingLayout<KVF>::VOFF, ROWV, r, sub);
+        dequant_part_to_ring<kFmtQ8, NB, LPR>(rowq, ok, dst, ROW, r, sub);
+        dequant_part_to_ring<kFmtQ4, DV / kQBlock, LPR>(rowq + quant_row_bytes(kFmtQ8, DQK), ok,
+                                                        dst + RingLayout<KVF>::VOFF, ROWV, r, sub);
     } else {
-        dequant_part_to_ring<KVF, NB>(rowq, ok, dst, ROW, r, sub);
+        dequant_part_to_ring<KVF, NB, LPR>(rowq, ok, dst, ROW, r, sub);
     }
 }
 
@@ -590,7 +593,7 @@ __global__ void __launch_bounds__(attn::Roles<KVF>::THREADS, 1) sparse_attn_mma_
                 cp_async_arrive_noinc(full_bar(s));
             } else {
                 const uint8_t* base_q = reinterpret_cast<const uint8_t*>(cmp ? p.kv_cmp : p.kv_raw);
-                dequant_row_to_ring<KVF>(base_q + (size_t)src_row * p.kv_row_bytes, ok, dst, r, sub);
+                dequant_row_to_ring<KVF, R::LPR>(base_q + (size_t)src_row * p.kv_row_bytes, ok, dst, r, sub);
                 mbar_arrive(full_bar(s));          // release: this thread's stores are visible
             }
             const uint32_t bits = __ballot_sync(0xffffffffu, ok && sub == 0);
