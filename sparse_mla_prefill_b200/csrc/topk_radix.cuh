@@ -177,7 +177,7 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan(unsigned long
 }
 
 template <int THREADS>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, THREADS <= 128 ? 16 : 1)
 topk_radix_kernel(const float* __restrict__ scores, int ld, int t0, int n_q, int k, int ratio,
                   const uint8_t* __restrict__ vis_mask, long long mask_ld, int mask_cols,
                   int32_t* __restrict__ topk) {

@@ -67,3 +67,41 @@ def test_band_in_a_graph(topk_mode):
     (rt, ro), (gt, go) = _direct_and_replayed(wl, dev, 0, wl.T, topk_mode=topk_mode)
     assert torch.equal(gt, rt)
     assert torch.equal(go, ro)
+
+
+def test_verify_graph_replays_follow_new_inputs():
+    """A verify step (q = 5: indexer, top-k, split attention and its merge) captured once
+    and replayed while the queries change in place: every replay gives the bits of a
+    direct call on that replay's inputs (nothing of an earlier replay is reused)."""
+    wl = workload("verify")
+    dev = to_device(generate(wl))
+    q = 5
+    t0 = wl.T - q
+    sl = {k: (v.clone() if k in ("q", "q_idx", "w") else v) for k, v in dev.items()}
+    gen = torch.Generator(device="cuda").manual_seed(11)
+    with handle_for(wl) as h:
+        ws = torch.empty(max(D.ds4sp_workspace_bytes(h, t0, q), 256), dtype=torch.uint8,
+                         device="cuda")
+        topk = torch.empty((q, wl.top_k), dtype=torch.int32, device="cuda")
+        out = torch.empty((q, 16, 512), dtype=torch.float32, device="cuda")
+        g = torch.cuda.CUDAGraph()
+        _step(h, sl, t0, q, topk, out, ws)             # warm-up outside the capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            _step(h, sl, t0, q, topk, out, ws)
+        torch.cuda.synchronize()
+        for r in range(4):
+            # new queries in the captured buffers (the rows and index keys stay)
+            sl["q"].copy_((torch.randn(sl["q"].shape, generator=gen, device="cuda") * 0.5).half())
+            g.replay()
+            torch.cuda.synchronize()
+            got_t, got_o = topk.clone(), out.clone()
+            ref_t = torch.empty_like(topk)
+            ref_o = torch.empty_like(out)
+            _step(h, sl, t0, q, ref_t, ref_o, ws)
+            torch.cuda.synchronize()
+            assert torch.equal(got_t, ref_t), r
+            assert torch.equal(got_o, ref_o), r
+        st, bits = D.ds4sp_device_status(h)
+        assert st == D.OK, hex(bits)
+        del g

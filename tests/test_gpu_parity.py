@@ -81,6 +81,25 @@ def test_verify_widths_bit_identical_across_widths():
         assert np.array_equal(results[q][1][-1], results[5][1][-1])
 
 
+def test_split_tokens_equal_across_call_sizes():
+    """Split-mode attention of the 5-token verify step (100 units of 32 rows, fewer than
+    the SMs) and of an 8-token call (160 units, more than the SMs, so a CTA takes two):
+    the tokens both calls hold get the same top-k and output bits."""
+    wl = workload("verify")
+    inp = generate(wl)
+    dev = to_device(inp)
+    T = wl.T
+    with handle_for(wl) as h:
+        # the last 8 tokens: per-token tensors of the verify workload hold 5, so widen them
+        # with 3 earlier tokens' copies of the same draws (positions differ, values repeat)
+        sl8 = {k: (torch.cat([v[:3], v]).contiguous() if k in ("q", "q_idx", "w") else v)
+               for k, v in dev.items()}
+        tk8, out8 = run_range(h, sl8, T - 8, 8, wl.top_k)
+        tk5, out5 = run_range(h, dev, T - 5, 5, wl.top_k)
+    assert torch.equal(tk8[3:], tk5)
+    assert torch.equal(out8[3:], out5)
+
+
 def test_band_path_equals_one_shot_bitwise():
     wl = workload("band", T=2048 + 700, band=1024)
     inp = generate_small(wl.T, wl.H_i, wl.D_i, seed=9)
@@ -140,6 +159,45 @@ def test_all_scores_equal(T, k, band, tail):
     assert (ref["topk"][nv >= k] == np.arange(k)).all()      # the lowest k rows
     assert np.array_equal(topk.cpu().numpy(), ref["topk"])
     assert_attention_close(out.cpu().numpy(), ref["out"], f"equal scores T={T}")
+
+
+def _dim0_scores(T, seed, dim0):
+    """Inputs whose index score of row j is dim0[j] for every token: one index head with
+    weight 1 whose query picks the key's first dimension (dim0 >= 0)."""
+    inp = generate_small(T, 4, 64, seed=seed)
+    k_idx = torch.zeros(T // 4, 64)
+    k_idx[:, 0] = dim0
+    q_idx = torch.zeros(T, 4, 64)
+    q_idx[:, 0, 0] = 1.0
+    w = torch.zeros(T, 4)
+    w[:, 0] = 1.0
+    inp.update(k_idx=k_idx.half(), q_idx=q_idx.half(), w=w)
+    return inp
+
+
+@pytest.mark.parametrize("case", ["ties", "near_equal"])
+def test_topk_radix_candidate_list(case):
+    """The radix select gathers the chosen bucket's keys into a list once a pass leaves at
+    most 512 of them and runs the later passes over the list. "ties": rows 0..599 score 3
+    and the rest 0, so a token that sees more than 512 rows never gets a small enough
+    bucket (every pass scans all keys) and one that sees fewer is listed after the first
+    pass; "near_equal": rows 0..599 score 1024 + j and the rest 1, so the first pass's
+    bucket holds up to 600 keys and the list forms at the second pass. Indices must equal
+    the oracle's (ties to the lower j)."""
+    T, k = 3000, 64
+    n_c = T // 4
+    j = torch.arange(n_c, dtype=torch.float32)
+    dim0 = torch.where(j < 600, torch.full_like(j, 3.0), torch.zeros_like(j)) if case == "ties" \
+        else torch.where(j < 600, 1024.0 + j, torch.ones_like(j))
+    inp = _dim0_scores(T, 21, dim0)
+    wl = Workload(case, T=T, H_i=4, D_i=64, top_k=k, n_swa=16, seed=21)
+    toks = sorted(set(range(0, T, 7)) | set(range(T - 8, T)) | {2047, 2400, 2403})
+    with handle_for(wl) as h:
+        topk, out = run_range(h, to_device(inp), 0, T, k)
+    ref = oracle_tokens(_np(inp), toks, wl)
+    got = topk.cpu().numpy()[toks]
+    assert np.array_equal(got, ref["topk"])
+    assert_attention_close(out.cpu().numpy()[toks], ref["out"], case)
 
 
 def test_causal_reduction_against_sdpa():
