@@ -75,9 +75,11 @@ typedef struct {
     int band;            /* tokens per band (2048) */
     int max_tokens;      /* sequence length T the KV buffers hold */
     float softmax_scale; /* <= 0 selects 1/sqrt(d_qk) */
-    int exp_mode;        /* softmax exponentials: 0 = ex2.approx (default, about 2^-22
-                            relative error), 1 = exp2f (CUDA's precise function); other
-                            values are DS4SP_ERR_INVALID_ARG */
+    int exp_mode;        /* softmax exponentials: 0 = ex2.approx (about 2^-22 relative
+                            error), 1 = exp2f (CUDA's precise function; measured the
+                            faster of the two in the streaming kernel, and the Python
+                            binding's default where the configuration allows it: fp16
+                            rows, attn_kernel 0); other values are DS4SP_ERR_INVALID_ARG */
     int pv_mode;         /* probabilities entering P . V: 0 = one fp16 term (default),
                             1 = fp32-staged: P = hi + lo, two fp16 terms (hi = fp16(p),
                             lo = fp16(p - hi)), about 22 significant bits, at twice the
@@ -94,7 +96,8 @@ typedef struct {
                             bytes, e.g. up to 2,560 visible rows -- a 10,240-token context
                             -- at 64 indexer heads) in a call of at most 1,024 token
                             blocks; otherwise the two kernels run. Indices are
-                            the same bits either way. Other values are
+                            the same bits either way; 1 is the faster prefill and
+                            the Python binding's default. Other values are
                             DS4SP_ERR_INVALID_ARG */
     int kv_format;       /* storage of kv_raw and kv_cmp: 0 = fp16 rows of 576 values
                             (1152 bytes); 1 = Q8_0 and 2 = Q4_0 quantized rows (one row

@@ -156,18 +156,21 @@ class Handle:
 
 def make_config(n_idx_heads: int, d_idx: int, top_k: int, n_swa: int, max_tokens: int,
                 band: int = 2048, softmax_scale: float = 0.0, n_heads: int = 16, d_qk: int = 576,
-                d_v: int = 512, ratio: int = 4, exp_mode: int = 0,
-                pv_mode: int = 0, topk_mode: int = 0, kv_format: int = 0,
+                d_v: int = 512, ratio: int = 4, exp_mode: Optional[int] = None,
+                pv_mode: int = 0, topk_mode: int = 1, kv_format: int = 0,
                 dependent_launch: int = 1, attn_kernel: int = 0,
                 indexer_kernel: int = 0) -> ds4sp_config:
     """A ds4sp_config in field order. exp_mode: 0 = ex2.approx, 1 = exp2f for the
-    softmax; pv_mode: 0 = fp16 probabilities in P . V, 1 = fp32-staged (hi + lo fp16);
-    topk_mode: 0 = scores in the workspace and a separate top-k kernel, 1 = fused
-    indexer + top-k where the call qualifies; kv_format: 0 = fp16 KV rows, 1 = Q8_0,
+    softmax (unset: 1 where the configuration supports it, fp16 rows on the streaming
+    kernel, where it measured faster; else 0); pv_mode: 0 = fp16 probabilities in P . V, 1 = fp32-staged (hi + lo fp16);
+    topk_mode: 1 (the default) = fused indexer + top-k where the call qualifies, 0 =
+    scores in the workspace and a separate top-k kernel; kv_format: 0 = fp16 KV rows, 1 = Q8_0,
     2 = Q4_0, 3 = Q8 K / Q4 V quantized rows (ds4sp_quantize_kv); dependent_launch:
     1 = each kernel a programmatic dependent of the one before it, 0 = plain order;
     attn_kernel: 0 = mma.sync streaming attention, 1 = logits on tcgen05 (TMEM);
     indexer_kernel: 0 = one CTA per tcgen05 tile, 1 = CTA pairs sharing each MMA."""
+    if exp_mode is None:
+        exp_mode = 1 if kv_format == 0 and attn_kernel == 0 else 0
     return ds4sp_config(n_heads, d_qk, d_v, ratio, n_idx_heads, d_idx, top_k, n_swa, band,
                         max_tokens, softmax_scale, exp_mode, pv_mode, topk_mode, kv_format,
                         dependent_launch, attn_kernel, indexer_kernel)

@@ -1,4 +1,5 @@
-"""Softmax exponentials: ex2.approx (default) against CUDA's exp2f (exp_mode 1). Both
+"""Softmax exponentials: ex2.approx (exp_mode 0) against CUDA's exp2f (exp_mode 1, the
+binding's default for fp16 rows). Both
 must meet the attention tolerance against the float64 oracle on the band workload,
 select the same rows, and differ from each other by no more than the tolerance; the
 precise mode must not be less accurate than the fast one by more than rounding noise.

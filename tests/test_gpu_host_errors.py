@@ -118,15 +118,21 @@ def test_bad_topk_index_is_skipped_and_reported(setup):
     assert st == D.OK and bits == 0
 
 
-def test_profile_counts_launches(setup):
-    h, inp, topk, out, ws = setup
-    D.ds4sp_profile_enable(h, True)
-    D.prefill(h, inp, WL.T, topk, out, ws)
-    prof = D.ds4sp_profile_read(h)
-    assert prof["indexer"][1] == 3 and prof["topk"][1] == 3 and prof["attention"][1] == 3
-    assert all(ms > 0 for ms, _ in prof.values())
-    assert all(n == 0 for _, n in D.ds4sp_profile_read(h).values())
-    D.ds4sp_profile_enable(h, False)
+@pytest.mark.parametrize("topk_mode", [0, 1])
+def test_profile_counts_launches(setup, topk_mode):
+    """Three bands: three launches of each kernel, or, with the fused indexer + top-k,
+    three of it (timed as the indexer) and none of the separate top-k."""
+    _, inp, topk, out, _ = setup
+    with handle_for(WL, topk_mode=topk_mode) as h:
+        ws = D.band_workspace(h, WL.T, "cuda")
+        D.ds4sp_profile_enable(h, True)
+        D.prefill(h, inp, WL.T, topk, out, ws)
+        prof = D.ds4sp_profile_read(h)
+        n_topk = 3 if topk_mode == 0 else 0
+        assert prof["indexer"][1] == 3 and prof["topk"][1] == n_topk and prof["attention"][1] == 3
+        assert all(ms > 0 for ms, n in prof.values() if n > 0)
+        assert all(n == 0 for _, n in D.ds4sp_profile_read(h).values())
+        D.ds4sp_profile_enable(h, False)
 
 
 def test_destroy_waits_for_work_in_flight():

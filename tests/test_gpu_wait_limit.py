@@ -3,7 +3,8 @@
 Every pipeline wait inside the kernels has a limit (about one second by default). A
 test cannot make a healthy pipeline stall, so it lowers the limit instead:
 ds4sp_debug_set_wait_limit_ns(h, 0) makes every wait give up at its first miss. The
-2048-token band then runs with waits that give up: the calls must return, the kernels
+2048-token band then runs with waits that give up, in both top-k forms (the fused
+indexer + top-k kernel and the two-kernel form): the calls must return, the kernels
 must end (the test would hang otherwise), the status word must carry bit 1 (a wait gave
 up), and once the default limit is back the next prefill must give the same bits as
 the one before, which is itself checked against the oracle on a sample of tokens.
@@ -27,11 +28,12 @@ def _lib(cuda_ok):
     D.load_library()
 
 
-def test_wait_give_up_is_reported_and_the_handle_recovers():
+@pytest.mark.parametrize("topk_mode", [0, 1])
+def test_wait_give_up_is_reported_and_the_handle_recovers(topk_mode):
     wl = workload("band")
     inp = generate(wl)
     dev = to_device(inp)
-    with handle_for(wl) as h:
+    with handle_for(wl, topk_mode=topk_mode) as h:
         topk1, out1 = run_prefill(h, dev, wl.T, wl.top_k)          # asserts status 0
         toks = sample_tokens(wl.T, wl.band, 32, seed=11)
         ref = oracle_tokens({k: v.numpy() for k, v in inp.items()}, toks, wl)
