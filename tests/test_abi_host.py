@@ -75,6 +75,20 @@ def test_create_rejects_bad_config_before_touching_the_device(lib, kw, status):
     assert lib.ds4sp_last_error()
 
 
+def test_binding_defaults():
+    """make_config's defaults: the fused indexer + top-k, and exp2f for the softmax where
+    the configuration runs it (fp16 rows on the streaming kernel), else ex2.approx, so
+    that every default configuration is one ds4sp_create accepts."""
+    base = dict(n_idx_heads=64, d_idx=128, top_k=512, n_swa=128, max_tokens=10240)
+    c = D.make_config(**base)
+    assert c.topk_mode == 1 and c.exp_mode == 1 and c.pv_mode == 0 and c.kv_format == 0
+    for kv in (1, 2, 3):
+        assert D.make_config(**base, kv_format=kv).exp_mode == 0
+    assert D.make_config(**base, attn_kernel=1).exp_mode == 0
+    assert D.make_config(**base, exp_mode=0).exp_mode == 0          # explicit wins
+    assert D.make_config(**base, topk_mode=0).topk_mode == 0
+
+
 def test_null_handle_paths(lib):
     assert lib.ds4sp_destroy(None) == D.OK
     assert lib.ds4sp_workspace_bytes(None, 0, 10) == 0
