@@ -571,7 +571,8 @@ def run_ours(args, rank, world, local_rank):
         attn_ms, attn_n = prof["attention"]
         head_launches = attn_n + prof["indexer"][1] + prof["topk"][1]
         fused = None
-        if split is not None:
+        # (a headline step with separate top-k launches did not take the fused kernel)
+        if split is not None and prof["topk"][1] == 0:
             f_ms, f_n = prof["indexer"]           # the fused kernel's launches
             f_tf = alg["indexer_flops"] * args.steps / (f_ms / 1e3) / 1e12
             fused = {"ms_per_step": f_ms / args.steps, "launches": f_n,
