@@ -64,3 +64,24 @@ def test_traffic_figure_needs_matching_kernel_sources(tmp_path, monkeypatch):
     assert bench.attention_traffic() == 123456
     (csrc / "sparse_attn_mma.cuh").write_text("// changed\n")
     assert bench.attention_traffic() is None
+
+
+def test_every_variant_is_an_accepted_configuration():
+    """Each configuration bench.py times (the headline, the two-kernel pass and every
+    entry of VARIANTS) passes ds4sp_create's checks. Without a GPU, create reports a
+    CUDA error once the configuration is accepted and a validation status otherwise."""
+    import ctypes
+
+    from sparse_mla_prefill_b200 import ds4sp as D
+    lib = D.load_library()
+    wl = workload("10k")
+    base = dict(n_idx_heads=wl.H_i, d_idx=wl.D_i, top_k=wl.top_k, n_swa=wl.n_swa,
+                max_tokens=wl.T, band=wl.band)
+    configs = [("headline", {}), ("two-kernel pass", dict(topk_mode=0))] + list(bench.VARIANTS)
+    for name, modes in configs:
+        cfg = D.make_config(**base, **modes)
+        out = ctypes.c_void_p()
+        st = lib.ds4sp_create(ctypes.byref(cfg), ctypes.byref(out))
+        assert st not in (D.ERR_INVALID_ARG, D.ERR_UNSUPPORTED), (name, modes, st)
+        if st == D.OK:                       # a GPU is present: the handle is real
+            lib.ds4sp_destroy(out)
