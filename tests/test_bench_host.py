@@ -1,7 +1,8 @@
 """Host-side pieces of bench.py, on CPU: the algorithmic byte and FLOP counts behind the
 roofline (against closed forms), the sampled parity check (passes on the oracle's own
-result, fails on a planted error), and the rule that an ncu traffic figure is used only
-for the kernel sources it was captured on."""
+result, fails on a planted error), the rule that an ncu traffic figure is used only
+for the kernel sources it was captured on, and that every configuration the bench times
+is one the library accepts."""
 import hashlib
 
 import numpy as np
